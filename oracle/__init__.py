@@ -1,0 +1,22 @@
+"""fp64 CPU oracle for DeltaLog decoding -- TEST INFRASTRUCTURE ONLY.
+
+This package is the plain, slow, eager definition of the three recurrences
+DeltaLog decodes (GDN, KDA, RWKV6), written in float64 numpy.  It is what the
+GPU path must reproduce: DeltaLog's claim is that the model observes the same
+dense state as eager decoding ("DeltaLog: Deferred Materialization of
+Recurrent States for Linear Attention Decoding", Abstract), so the oracle is
+the eager recurrence itself, with no log and no merge.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU
+baseline and reference arm) may import it.  The library never does: it shares
+no code with the CUDA path and imports nothing from it.
+
+Parity is not pinned to printed values: the pages print no worked example.
+The oracle is pinned instead by closed forms, exact rational hand examples,
+invariants and an exact-arithmetic brute force of the log form (see
+``tests/test_oracle_pins.py``).
+"""
+
+from .recurrence import (  # noqa: F401
+    gdn_step, kda_step, rwkv6_step, run_eager, EagerResult,
+)
