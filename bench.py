@@ -1,0 +1,523 @@
+"""Decode state-update throughput of DeltaLog on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--L 16] [--merge fused|separate]
+                    [--impl ours|reference] [--sweep]
+
+Workload: GDN decode, B=512 sequences, H=32 heads, d_k=d_v=128, fp32 state
+(1 GiB), bf16 q/k/v, ragged batch whose sequences start at log fill offsets
+U{0..L-1} (so merges are staggered), L=16.  One step = one decode step of the
+whole batch (one layer, all heads) including the merges it triggers; the
+timed loop cycles a device ring of 16 pre-drawn steps.  tokens/s = B * K /
+time.  The state (1 GiB) is far larger than L2 (126 MB), so no L2 flush is
+needed between steps.
+
+The JSON line also carries: the roofline of the dominant kernel (the step
+kernel, HBM-bound: algorithmic bytes per launch / its mean CUDA-event
+duration, against the measured copy bandwidth), the eager dense step kernel
+timed the same way, an end-to-end figure (host inputs in pinned memory
+copied in and o copied out every step), the fp64 CPU oracle timed on a
+bounded sample of the same workload, and SM clocks sampled during the timed
+region.
+
+With --gpus N > 1 (one process per GPU under torchrun) every rank decodes its
+own B=512 batch (weak scaling, no data-path collective); the time is the
+maximum over ranks and the value counts all ranks' tokens.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_recurrent_deltalog_b200 import workloads as wl  # noqa: E402
+
+METRIC = "decode state-update tokens/s (B=512,H=32,d=128); HBM GB/s vs 8 TB/s peak"
+UNIT = "tokens/s"
+RING = 16
+L2_BYTES = 126 * 2**20
+FALLBACK_HBM_GBS = 6650.0
+
+# Step kernel source files: a traffic figure taken by ncu is reported only
+# while these are unchanged.
+KERNEL_SOURCES = ("linear_attention_recurrent_deltalog_b200/csrc/dl_kernels.cuh",
+                  "linear_attention_recurrent_deltalog_b200/csrc/dl_device.cuh")
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = os.environ.get("DL_BENCH_BACKEND", "nccl")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Maximum of a host float over all ranks (the bench's timing rule)."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(tokens_per_rank: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / max_seconds
+
+
+# ------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ byte model
+
+def step_bytes(cfg, fills: np.ndarray, fused: bool) -> tuple:
+    """Algorithmic bytes one step-kernel launch must move (read, write).
+
+    Per head with f log entries before the step (GDN, fp32 state):
+      read : S_b (d_v*d_k*4) + q,k,v + decay,beta + fill + f log entries
+      write: o (d_v*4) + fill + the appended entry, or (fused merge, f = L-1)
+             the merged S_b instead of the entry.
+    """
+    ein = 2 if cfg.in_dtype == "bf16" else 4
+    dk, dv, H = cfg.d_k, cfg.d_v, cfg.H
+    gw = 1 if cfg.variant == "gdn" else dk
+    uin = ein if cfg.variant == "rwkv6" else 4
+    entry = dv * uin + dk * ein + gw * 4
+    tile = dv * dk * 4
+    vec = (2 * dk + dv) * ein + (4 if cfg.variant == "gdn" else dk * 4) + (4 if cfg.variant != "rwkv6" else 0)
+    f = fills.astype(np.int64)
+    merging = (f == cfg.L - 1) if fused else np.zeros_like(f, dtype=bool)
+    rd = H * (tile + vec + 4 + f * entry)
+    wr = H * (dv * 4 + 4 + np.where(merging, tile, entry))
+    return int(rd.sum()), int(wr.sum())
+
+
+def merge_bytes(cfg, fills_after_step: np.ndarray) -> tuple:
+    """Algorithmic bytes of a separate merge launch (sequences with f == L)."""
+    ein = 2 if cfg.in_dtype == "bf16" else 4
+    dk, dv, H = cfg.d_k, cfg.d_v, cfg.H
+    gw = 1 if cfg.variant == "gdn" else dk
+    uin = ein if cfg.variant == "rwkv6" else 4
+    entry = dv * uin + dk * ein + gw * 4
+    tile = dv * dk * 4
+    n = int((fills_after_step == cfg.L).sum())
+    allfill = fills_after_step.size * H * 4
+    return allfill + n * H * (tile + cfg.L * entry), n * H * (tile + 4)
+
+
+def eager_bytes(cfg) -> tuple:
+    ein = 2 if cfg.in_dtype == "bf16" else 4
+    dk, dv = cfg.d_k, cfg.d_v
+    tile = dv * dk * 4
+    vec = (2 * dk + dv) * ein + 8
+    return cfg.heads * (tile + vec), cfg.heads * (tile + dv * 4)
+
+
+# ------------------------------------------------------------ our arm
+
+def to_dev(s, device):
+    def up(x):
+        if x is None:
+            return None
+        if x.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(device).view(torch.bfloat16).reshape(-1)
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device).reshape(-1)
+    return (up(s.device_array("q")), up(s.device_array("k")), up(s.device_array("v")),
+            up(s.decay), up(s.beta))
+
+
+def run_ours(args, world, rank, local):
+    from linear_attention_recurrent_deltalog_b200 import deltalog as dlb
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    fused = args.merge == "fused"
+    w = wl.WORKLOADS["gdn_serving"].replace(L=args.L)
+    cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=fused)
+    stream = torch.cuda.current_stream(device)
+
+    # inputs: a device ring of RING pre-drawn steps (the generator's recipe)
+    host_steps = list(wl.StepStream(w, RING, workers=args.gen_workers))
+    ring = [to_dev(s, device) for s in host_steps]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    S0 = (torch.randn(w.heads * w.d_v * w.d_k, generator=gen, device=device) * w.s0_std).contiguous()
+    fill0 = wl.fill_offsets(w)
+
+    st = dlb.DeltaLogState(cfg, device=device)
+    st.reset(S0, fill0.tolist())
+    o = torch.empty(w.heads * w.d_v, dtype=torch.float32, device=device)
+
+    def one_step(i, ev=None):
+        q, k, v, dec, beta = ring[i % RING]
+        if ev is not None:
+            ev[0].record(stream)
+        st.step(q, k, v, dec, beta, None, o)
+        if ev is not None:
+            ev[1].record(stream)
+        if not fused:
+            st.merge(dlb.DL_MERGE_FULL)
+
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize(device)
+
+    # algorithmic bytes of the timed steps, from the host fill mirror
+    fills = np.array(st.fill(), dtype=np.int64)
+    rd = wr = mrd = mwr = 0
+    for i in range(args.steps):
+        r_, w_ = step_bytes(cfg, fills, fused)
+        rd, wr = rd + r_, wr + w_
+        fills = fills + 1
+        if not fused:
+            a, b = merge_bytes(cfg, fills)
+            mrd, mwr = mrd + a, mwr + b
+        fills[fills == cfg.L] = 0
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = dlb.dl_launch_count()
+    dist_barrier(world)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            one_step(args.warmup + i, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    dist_barrier(world)
+    launches = dlb.dl_launch_count() - n0
+    elapsed = start.elapsed_time(end) / 1e3
+    step_kernel_s = sum(a.elapsed_time(b) for a, b in evs) / 1e3
+    code, head = st.device_error()
+    if code != 0:
+        raise RuntimeError(f"device error {code} at head {head}")
+    max_elapsed = max_over_ranks(elapsed, world, device)
+    tokens = w.B * args.steps
+    value = aggregate_value(tokens, world, max_elapsed)
+
+    peak, peak_kind = hbm_peak()
+    step_avg = step_kernel_s / args.steps
+    step_bytes_avg = (rd + wr) / args.steps
+    achieved = step_bytes_avg / step_avg / 1e9
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "step_kernel_traffic.json")
+    if os.path.exists(tfile):
+        try:
+            t = json.load(open(tfile))
+            if t.get("kernel_hash") == kernel_hash() and t.get("L") == args.L and t.get("merge") == args.merge:
+                traffic = t.get("bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    # eager dense step on a separate 1 GiB state, same inputs
+    S_e = S0.clone()
+    for i in range(args.warmup):
+        q, k, v, dec, beta = ring[i % RING]
+        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, None, o)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        q, k, v, dec, beta = ring[i % RING]
+        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, None, o)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    eager_s = e0.elapsed_time(e1) / 1e3
+    erd, ewr = eager_bytes(cfg)
+    del S_e
+
+    # end to end: pinned host inputs in, o out, every step
+    pinned = []
+    for s in host_steps:
+        arrs = [s.device_array("q"), s.device_array("k"), s.device_array("v"), s.decay, s.beta]
+        ts = []
+        for a in arrs:
+            if a.dtype == np.uint16:
+                ts.append(torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).reshape(-1).pin_memory())
+            else:
+                ts.append(torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).reshape(-1).pin_memory())
+        pinned.append(ts)
+    dbuf = [torch.empty(t.numel(), dtype=t.dtype, device=device) for t in pinned[0]]
+    o_host = torch.empty(o.numel(), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned[0])
+    d2h = o_host.numel() * 4
+
+    def e2e_step(i):
+        for d, h in zip(dbuf, pinned[i % RING]):
+            d.copy_(h, non_blocking=True)
+        q = dbuf[0].view(torch.bfloat16)
+        k = dbuf[1].view(torch.bfloat16)
+        v = dbuf[2].view(torch.bfloat16)
+        st.step(q, k, v, dbuf[3], dbuf[4], None, o)
+        if not fused:
+            st.merge(dlb.DL_MERGE_FULL)
+        o_host.copy_(o, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize(device)
+    dist_barrier(world)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    x1.record(stream)
+    torch.cuda.synchronize(device)
+    dist_barrier(world)
+    e2e_s = max_over_ranks(x0.elapsed_time(x1) / 1e3, world, device)
+    st.close()
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_elapsed * 1e3 / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"GDN decode B=512 H=32 d_k=d_v=128 fp32 state, bf16 q/k/v, "
+                               f"ragged fills, L={args.L}, merge={args.merge}",
+                   "B": w.B, "H": w.H, "d": w.d_k, "L": args.L, "merge": args.merge,
+                   "global_batch": w.B * world, "parallelism": f"replicas x{world} (dp, no collective)",
+                   "l2": "state 1 GiB > 126 MB L2 on every step: no flush needed",
+                   "input_ring_steps": RING},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": f"{peak_kind} copy bandwidth",
+                     "kernel": "dl_step_kernel", "algorithmic_bytes_per_launch": int(step_bytes_avg),
+                     "launch_ms": round(step_avg * 1e3, 5)},
+        "gpu_launches": int(launches),
+        "e2e": {"value": round(aggregate_value(tokens, world, e2e_s), 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "clocks": clk.summary(),
+        "hbm_gbs_step_plus_merge": round(((rd + wr + mrd + mwr) / args.steps) / (max_elapsed / args.steps) / 1e9, 1),
+        "write_bytes_per_token": {"deltalog": round((wr + mwr) / args.steps / w.B, 1),
+                                  "eager": round(ewr / w.B, 1),
+                                  "reduction": round(ewr / ((wr + mwr) / args.steps), 3)},
+        "eager": {"value": round(aggregate_value(tokens, 1, eager_s), 1), "unit": UNIT,
+                  "achieved_gbs": round((erd + ewr) / (eager_s / args.steps) / 1e9, 1),
+                  "frac": round((erd + ewr) / (eager_s / args.steps) / 1e9 / peak, 4),
+                  "speedup_of_deltalog": round(eager_s / elapsed, 3)},
+    }
+    return line
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_tokens_per_s(target_s: float, seqs: int = 2, steps_cap: int = 10**6):
+    """The fp64 oracle as it stands on a bounded sample of the workload:
+    the first ``seqs`` sequences (all 32 heads each), successive steps,
+    until ``target_s`` seconds of CPU work have run.  Returns (tokens/s,
+    steps, seconds, threads)."""
+    import oracle
+    from oracle import recurrence as rec  # noqa: F401
+    w = wl.WORKLOADS["gdn_serving"]
+    heads = np.arange(seqs * w.H)
+    S = np.random.default_rng(w.seed).standard_normal((heads.size, w.d_v, w.d_k)) * w.s0_std
+    steps = 0
+    t0 = time.perf_counter()
+    el = 0.0
+    t = 0
+    while el < target_s and steps < steps_cap:
+        s = wl.step_inputs(w, t)  # drawing is not timed
+        sl = lambda x: x.reshape((w.heads,) + x.shape[2:])[heads][:, None]
+        import types
+        st = types.SimpleNamespace(q=sl(s.q), k=sl(s.k), v=sl(s.v), decay=sl(s.decay), beta=sl(s.beta))
+        a = time.perf_counter()
+        S = oracle.run_eager("gdn", S, [st]).S
+        el += time.perf_counter() - a
+        steps += 1
+        t += 1
+    threads = None
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        threads = max((i.get("num_threads", 1) for i in info), default=None)
+    except Exception:
+        threads = os.cpu_count()
+    return seqs * steps / el, steps, el, threads
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    target = min(20.0, max(2.0, 0.02 * (args.steps + args.warmup)))
+    v, steps, el, threads = oracle_tokens_per_s(target)
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": 0, "ms_per_step": round(el * 1e3 / steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"GDN decode B=512 H=32 d_k=d_v=128, L={args.L} (oracle: eager fp64)",
+                   "B": 512, "H": 32, "d": 128, "L": args.L},
+        "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"first 2 of 512 sequences (64 heads), {steps} steps, "
+                                   f"{el:.1f} s of fp64 eager oracle time"},
+        "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--L", type=int, default=16)
+    ap.add_argument("--merge", choices=("fused", "separate"), default="fused")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gen-workers", type=int, default=None)
+    ap.add_argument("--sweep", action="store_true", help="also print one line per L in 4..64")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+            return
+        line = run_ours(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            v, steps, el, threads = oracle_tokens_per_s(args.cpu_seconds)
+            line["cpu_baseline"] = {"value": round(v, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"first 2 of 512 sequences (64 heads), {steps} steps, "
+                                              f"{el:.1f} s of fp64 eager oracle time"}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if args.sweep:
+            for L in wl.SERVING_L_SWEEP:
+                for merge in ("fused", "separate"):
+                    a2 = argparse.Namespace(**vars(args))
+                    a2.L, a2.merge = L, merge
+                    a2.steps = min(args.steps, 500)
+                    l2 = run_ours(a2, world, rank, local)
+                    if rank == 0:
+                        print(json.dumps({"sweep": True, "L": L, "merge": merge, "value": l2["value"],
+                                          "roofline": l2["roofline"], "eager": l2["eager"],
+                                          "write_bytes_per_token": l2["write_bytes_per_token"],
+                                          "hbm_gbs_step_plus_merge": l2["hbm_gbs_step_plus_merge"]}),
+                              flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+/*
+ * deltalog.h -- C ABI of the DeltaLog decode library for B200 (sm_100a).
+ *
+ * DeltaLog ("DeltaLog: Deferred Materialization of Recurrent States for
+ * Linear Attention Decoding", Abstract and AI Summary) keeps each head's
+ * recurrent state as a dense base plus a bounded log of recent compact
+ * updates.  A decode step reads base + log, appends one compact factor
+ * instead of writing the whole state back, and a periodic merge folds the
+ * log into the base.  The model observes the same dense state as eager
+ * decoding (up to floating-point rounding order).
+ *
+ * Recurrences (state S is d_v x d_k per head, row = value index, contiguous
+ * along the key index):
+ *   GDN   S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t
+ *   KDA   S_t = S_{t-1} Diag(a_t) (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t
+ *   RWKV6 (stored as the transpose of its d_k x d_v matrix)
+ *         S_t = S_{t-1} Diag(w_t) + v_t k_t^T,
+ *         o_t = S_{t-1} r_t + (sum_c r_c u_c k_c) v_t
+ * With gamma_t the decay accumulated since the base was last merged and
+ * u_t = b_t (v_t - a_t S_{t-1} k_t) (GDN; KDA uses S_{t-1}(a_t o k_t)),
+ *   S_t = S_b Diag(gamma_t) + sum_i u_i (k_i o gamma_t / gamma_i)^T,
+ * so one log entry is (u_i, k_i, log gamma_i); RWKV6 stores u_i = v_i.
+ *
+ * Conventions for every call:
+ *   - Returns DL_OK (0) or a negative DL_ERR_* code.  Arguments are checked
+ *     on the host before anything is enqueued; a failed check enqueues
+ *     nothing and changes no state.
+ *   - Device pointers are plain CUDA device addresses owned by the caller.
+ *     The library never allocates device memory and never frees caller
+ *     memory; a dl_state borrows the three buffers sized by dl_state_bytes
+ *     for its whole life.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on it and never synchronize, except
+ *     dl_state_reset and dl_device_error, which say so.
+ *   - One dl_state is used from one host thread and one stream at a time.
+ *   - Floating-point results equal eager decoding up to rounding order, not
+ *     bitwise: the log and the merge sum in a different order.
+ */
+#ifndef DELTALOG_H
+#define DELTALOG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Recurrence family ("We implement DeltaLog for GDN, KDA, and RWKV6"). */
+enum dl_variant { DL_GDN = 0, DL_KDA = 1, DL_RWKV6 = 2 };
+
+/* Element type of q (r), k and v as stored by the caller. */
+enum dl_dtype { DL_F32 = 0, DL_BF16 = 1 };
+
+/* Status codes. */
+enum dl_status {
+  DL_OK = 0,
+  DL_ERR_ARG = -1,         /* null pointer, bad size, bad enum, bad mode   */
+  DL_ERR_ALIGN = -2,       /* a pointer violates the alignment rule        */
+  DL_ERR_LOG_FULL = -3,    /* a sequence's log holds L entries: merge first */
+  DL_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed          */
+  DL_ERR_UNSUPPORTED = -5, /* valid but not built (head size, dtype)        */
+  DL_ERR_DEVICE = -6       /* a kernel recorded an error (dl_device_error)  */
+};
+
+/* dl_merge modes. */
+enum dl_merge_mode {
+  DL_MERGE_FULL = 0, /* fold the logs of sequences whose log holds L entries */
+  DL_MERGE_ALL = 1   /* fold every non-empty log                            */
+};
+
+/* dl_config.flags */
+enum dl_flags {
+  /* The step kernel merges in place: a head whose append would fill its
+   * log writes the merged base instead and leaves an empty log, so the log
+   * is never full and dl_merge(DL_MERGE_FULL) has nothing to do. */
+  DL_FLAG_FUSED_MERGE = 1
+};
+
+/* Layer configuration.  d_k, d_v in {64, 128}; 1 <= L <= 64; B, H >= 1 and
+ * B*H*d_v*d_k < 2^40.  `flags` is a bitwise OR of dl_flags. */
+typedef struct dl_config {
+  int32_t variant;  /* enum dl_variant */
+  int32_t B;        /* sequences in the batch */
+  int32_t H;        /* heads per sequence */
+  int32_t d_k;      /* key (and q / r) size per head */
+  int32_t d_v;      /* value size per head */
+  int32_t L;        /* log capacity: entries per head before a merge */
+  int32_t in_dtype; /* enum dl_dtype of q/r, k, v */
+  int32_t flags;    /* enum dl_flags */
+} dl_config;
+
+typedef struct dl_state dl_state;
+
+/* Sizes in bytes of the three device buffers a state borrows:
+ *   base: fp32 [B, H, d_v, d_k]                 the dense base S_b
+ *   log : per head L entries of u (fp32 [d_v]; in_dtype for RWKV6),
+ *         k (in_dtype [d_k]) and log-decay g (fp32, [1] for GDN, [d_k]
+ *         otherwise), laid out as three arrays [B,H,L,.], each 256-B aligned
+ *   meta: int32 fill [B, H] plus a device error word, 256-B padded.
+ * Any output pointer may be NULL.  Errors: DL_ERR_ARG, DL_ERR_UNSUPPORTED. */
+int dl_state_bytes(const dl_config* cfg, size_t* base_bytes, size_t* log_bytes,
+                   size_t* meta_bytes);
+
+/* Creates a state over caller-owned device buffers of at least the sizes
+ * above, each 256-byte aligned (else DL_ERR_ALIGN).  The contents are
+ * undefined until dl_state_reset.  Enqueues nothing.  The handle (host
+ * memory) is owned by the library until dl_state_destroy. */
+int dl_state_create(const dl_config* cfg, void* base, void* log, void* meta,
+                    dl_state** out);
+
+/* Loads a dense state and starts every log.  S0: fp32 [B, H, d_v, d_k]
+ * device buffer 16-B aligned, or NULL for a zero state.  fill0: host int32
+ * [B] with 0 <= fill0[b] < L, or NULL for zeros; sequence b starts with
+ * fill0[b] log entries that change nothing (u = 0, k = 0, g = 0), so its
+ * first merge comes after L - fill0[b] steps (ragged batches sit at
+ * different merge phases).  Clears the device error word.  Synchronizes
+ * `stream` before returning (it copies the fill counts from host memory). */
+int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* stream);
+
+/* One decode step for all B*H heads (one kernel launch).
+ *   q: q_t (r_t for RWKV6)  [B, H, d_k] in_dtype
+ *   k: k_t                  [B, H, d_k] in_dtype
+ *   v: v_t                  [B, H, d_v] in_dtype
+ *   decay: fp32, GDN alpha_t [B, H]; KDA alpha_t [B, H, d_k];
+ *          RWKV6 w_t [B, H, d_k]; every value in (0, 1]
+ *   beta: fp32 [B, H] for GDN/KDA; ignored (may be NULL) for RWKV6
+ *   bonus: fp32 [H, d_k] RWKV6 u; ignored (may be NULL) otherwise
+ *   o: fp32 [B, H, d_v] output o_t
+ * All pointers 16-byte aligned device addresses.  Without
+ * DL_FLAG_FUSED_MERGE, returns DL_ERR_LOG_FULL (enqueuing nothing) when
+ * some sequence's log already holds L entries: call dl_merge first. */
+int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v,
+                   const float* decay, const float* beta, const float* bonus,
+                   float* o, void* stream);
+
+/* Folds logs into the base: S_b <- S_b Diag(gamma) + sum_i u_i (k_i o
+ * gamma / gamma_i)^T, then empties those logs.  mode DL_MERGE_FULL folds
+ * the sequences whose log holds L entries, DL_MERGE_ALL every non-empty
+ * log.  Enqueues nothing when no sequence qualifies. */
+int dl_merge(dl_state* st, int mode, void* stream);
+
+/* Writes the dense state S_t = base folded with the log to S_out (fp32
+ * [B, H, d_v, d_k], 16-B aligned, must not alias the base) without changing
+ * the state. */
+int dl_materialize(const dl_state* st, float* S_out, void* stream);
+
+/* Eager dense step, the comparison point: reads and writes the whole fp32
+ * state S [B, H, d_v, d_k] (16-B aligned) in place, same recurrence and
+ * arguments as dl_decode_step.  cfg->L and cfg->flags are ignored. */
+int dl_eager_step(const dl_config* cfg, float* S, const void* q, const void* k,
+                  const void* v, const float* decay, const float* beta,
+                  const float* bonus, float* o, void* stream);
+
+/* Copies the host-side fill counts (entries per sequence, int32 [B]). */
+int dl_state_fill(const dl_state* st, int32_t* fill_out);
+
+/* Releases the handle (not the borrowed buffers).  NULL is accepted. */
+int dl_state_destroy(dl_state* st);
+
+/* Reads and optionally clears the device error word that kernels set when
+ * a bounded wait gives up or a device-side check fails (code 0 = none;
+ * *head = first failing head).  `st` NULL reads the word the eager kernel
+ * uses on the current device.  Synchronizes `stream`. */
+int dl_device_error(dl_state* st, int32_t* code, int32_t* head, int clear, void* stream);
+
+/* Total kernels this library has launched in this process. */
+uint64_t dl_launch_count(void);
+
+/* Static text for a status code. */
+const char* dl_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DELTALOG_H */

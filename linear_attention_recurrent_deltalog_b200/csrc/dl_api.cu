@@ -1,0 +1,384 @@
+// dl_api.cu -- the C ABI of the DeltaLog library (declared in deltalog.h).
+//
+// Host side only: argument checks, the buffer layout a state borrows, the
+// host mirror of every sequence's log fill (so merge scheduling and the
+// "log full" check need no device round trip), and kernel launches.
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "deltalog.h"
+#include "dl_launch.cuh"
+
+namespace {
+
+using dl::Shape;
+
+std::atomic<uint64_t> g_launches{0};
+
+// Error word used by kernels that run without a state (the eager step).
+__device__ int g_dev_err[2];
+
+constexpr size_t kAlign = 256;
+
+size_t pad(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Layout {
+  size_t base, u_off, u_bytes, k_off, k_bytes, g_off, g_bytes, log, fill_bytes, err_off, meta;
+};
+
+int u_elem_size(const dl_config& c) {
+  return (c.variant == DL_RWKV6) ? (c.in_dtype == DL_BF16 ? 2 : 4) : 4;
+}
+int in_elem_size(const dl_config& c) { return c.in_dtype == DL_BF16 ? 2 : 4; }
+
+Layout layout_of(const dl_config& c) {
+  const size_t bh = size_t(c.B) * size_t(c.H);
+  const size_t gw = (c.variant == DL_GDN) ? 1 : size_t(c.d_k);
+  Layout l{};
+  l.base = pad(bh * c.d_v * c.d_k * 4);
+  l.u_off = 0;
+  l.u_bytes = pad(bh * c.L * c.d_v * u_elem_size(c));
+  l.k_off = l.u_off + l.u_bytes;
+  l.k_bytes = pad(bh * c.L * c.d_k * in_elem_size(c));
+  l.g_off = l.k_off + l.k_bytes;
+  l.g_bytes = pad(bh * c.L * gw * 4);
+  l.log = l.g_off + l.g_bytes;
+  l.fill_bytes = pad(bh * 4);
+  l.err_off = l.fill_bytes;
+  l.meta = l.err_off + kAlign;
+  return l;
+}
+
+bool head_size_ok(int d) { return d == 64 || d == 128; }
+
+// Shape checks shared by every call.  `need_L`: whether L matters.
+int check_config(const dl_config* c, bool need_L) {
+  if (c == nullptr) return DL_ERR_ARG;
+  if (c->variant < DL_GDN || c->variant > DL_RWKV6) return DL_ERR_ARG;
+  if (c->B < 1 || c->H < 1 || c->d_k < 1 || c->d_v < 1) return DL_ERR_ARG;
+  if (c->in_dtype != DL_F32 && c->in_dtype != DL_BF16) return DL_ERR_ARG;
+  if (need_L && (c->L < 1 || c->L > 64)) return DL_ERR_ARG;
+  if (need_L && (c->flags & ~int32_t(DL_FLAG_FUSED_MERGE)) != 0) return DL_ERR_ARG;
+  const uint64_t bh = uint64_t(c->B) * uint64_t(c->H);
+  if (bh > 0x7fffffffull) return DL_ERR_ARG;  // one CTA per head in a 1-D grid
+  if (bh * uint64_t(c->d_v) * uint64_t(c->d_k) >= (1ull << 40)) return DL_ERR_ARG;
+  if (!head_size_ok(c->d_k) || !head_size_ok(c->d_v)) return DL_ERR_UNSUPPORTED;
+  return DL_OK;
+}
+
+Shape shape_of(const dl_config& c) { return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0}; }
+
+cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, cudaStream_t s) {
+  const unsigned n = unsigned(size_t(c.B) * c.H);
+  const bool fused = (c.flags & DL_FLAG_FUSED_MERGE) != 0;
+  switch (c.variant) {
+    case DL_GDN: return dl::launch_step<dl::kVarGDN>(shape_of(c), fused, p, n, s);
+    case DL_KDA: return dl::launch_step<dl::kVarKDA>(shape_of(c), fused, p, n, s);
+    default: return dl::launch_step<dl::kVarRWKV6>(shape_of(c), fused, p, n, s);
+  }
+}
+
+cudaError_t launch_merge(const dl_config& c, const dl::MergeParams& p, cudaStream_t s) {
+  const unsigned n = unsigned(size_t(c.B) * c.H);
+  switch (c.variant) {
+    case DL_GDN: return dl::launch_merge<dl::kVarGDN>(shape_of(c), p, n, s);
+    case DL_KDA: return dl::launch_merge<dl::kVarKDA>(shape_of(c), p, n, s);
+    default: return dl::launch_merge<dl::kVarRWKV6>(shape_of(c), p, n, s);
+  }
+}
+
+cudaError_t launch_eager(const dl_config& c, const dl::EagerParams& p, cudaStream_t s) {
+  const unsigned n = unsigned(size_t(c.B) * c.H);
+  switch (c.variant) {
+    case DL_GDN: return dl::launch_eager<dl::kVarGDN>(shape_of(c), p, n, s);
+    case DL_KDA: return dl::launch_eager<dl::kVarKDA>(shape_of(c), p, n, s);
+    default: return dl::launch_eager<dl::kVarRWKV6>(shape_of(c), p, n, s);
+  }
+}
+
+// Device address of g_dev_err on the current device (cached per device).
+int* global_err_word() {
+  static std::atomic<int*> cache[dl::kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= dl::kMaxDevices) return nullptr;
+  int* p = cache[dev].load(std::memory_order_acquire);
+  if (p != nullptr) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_dev_err) != cudaSuccess) return nullptr;
+  cache[dev].store(static_cast<int*>(addr), std::memory_order_release);
+  return static_cast<int*>(addr);
+}
+
+// Checks shared by dl_decode_step and dl_eager_step.
+int check_step_args(const dl_config& c, const void* q, const void* k, const void* v,
+                    const float* decay, const float* beta, const float* bonus, const float* o) {
+  if (!q || !k || !v || !decay || !o) return DL_ERR_ARG;
+  if (c.variant == DL_RWKV6 ? (bonus == nullptr) : (beta == nullptr)) return DL_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(decay, 16) ||
+      !aligned(o, 16))
+    return DL_ERR_ALIGN;
+  if (c.variant == DL_RWKV6 ? !aligned(bonus, 16) : !aligned(beta, 16)) return DL_ERR_ALIGN;
+  return DL_OK;
+}
+
+}  // namespace
+
+struct dl_state {
+  dl_config cfg;
+  Layout lay;
+  float* base;
+  unsigned char* log;
+  unsigned char* meta;
+  std::vector<int32_t> fill;        // host mirror, entries per sequence
+  std::vector<int32_t> fill_stage;  // [B*H] staging for reset uploads
+  int n_full;                       // sequences whose log holds L entries
+  int n_nonempty;                   // sequences whose log holds >= 1 entry
+
+  int* dev_fill() const { return reinterpret_cast<int*>(meta); }
+  int* dev_err() const { return reinterpret_cast<int*>(meta + lay.err_off); }
+  void* logU() const { return log + lay.u_off; }
+  void* logK() const { return log + lay.k_off; }
+  float* logG() const { return reinterpret_cast<float*>(log + lay.g_off); }
+  void recount() {
+    n_full = n_nonempty = 0;
+    for (int32_t f : fill) {
+      n_full += (f == cfg.L);
+      n_nonempty += (f > 0);
+    }
+  }
+};
+
+extern "C" {
+
+int dl_state_bytes(const dl_config* cfg, size_t* base_bytes, size_t* log_bytes,
+                   size_t* meta_bytes) {
+  const int rc = check_config(cfg, true);
+  if (rc != DL_OK) return rc;
+  const Layout l = layout_of(*cfg);
+  if (base_bytes) *base_bytes = l.base;
+  if (log_bytes) *log_bytes = l.log;
+  if (meta_bytes) *meta_bytes = l.meta;
+  return DL_OK;
+}
+
+int dl_state_create(const dl_config* cfg, void* base, void* log, void* meta, dl_state** out) {
+  if (out == nullptr) return DL_ERR_ARG;
+  *out = nullptr;
+  const int rc = check_config(cfg, true);
+  if (rc != DL_OK) return rc;
+  if (!base || !log || !meta) return DL_ERR_ARG;
+  if (!aligned(base, kAlign) || !aligned(log, kAlign) || !aligned(meta, kAlign))
+    return DL_ERR_ALIGN;
+  const Shape sh = shape_of(*cfg);
+  size_t need = 0;
+  switch (cfg->variant) {
+    case DL_GDN:
+      need = dl::step_smem_bytes<dl::kVarGDN>(sh, cfg->L);
+      need = need > dl::merge_smem_bytes<dl::kVarGDN>(sh, cfg->L) ? need
+                                                                : dl::merge_smem_bytes<dl::kVarGDN>(sh, cfg->L);
+      break;
+    case DL_KDA:
+      need = dl::step_smem_bytes<dl::kVarKDA>(sh, cfg->L);
+      need = need > dl::merge_smem_bytes<dl::kVarKDA>(sh, cfg->L) ? need
+                                                                : dl::merge_smem_bytes<dl::kVarKDA>(sh, cfg->L);
+      break;
+    default:
+      need = dl::step_smem_bytes<dl::kVarRWKV6>(sh, cfg->L);
+      need = need > dl::merge_smem_bytes<dl::kVarRWKV6>(sh, cfg->L) ? need
+                                                                  : dl::merge_smem_bytes<dl::kVarRWKV6>(sh, cfg->L);
+  }
+  if (need == 0 || need > size_t(dl::kMaxSmemOptIn)) return DL_ERR_UNSUPPORTED;
+  dl_state* st = new (std::nothrow) dl_state();
+  if (st == nullptr) return DL_ERR_ARG;
+  st->cfg = *cfg;
+  st->lay = layout_of(*cfg);
+  st->base = static_cast<float*>(base);
+  st->log = static_cast<unsigned char*>(log);
+  st->meta = static_cast<unsigned char*>(meta);
+  st->fill.assign(size_t(cfg->B), 0);
+  st->fill_stage.assign(size_t(cfg->B) * cfg->H, 0);
+  st->recount();
+  *out = st;
+  return DL_OK;
+}
+
+int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* stream) {
+  if (st == nullptr) return DL_ERR_ARG;
+  const dl_config& c = st->cfg;
+  if (S0 != nullptr && !aligned(S0, 16)) return DL_ERR_ALIGN;
+  if (S0 != nullptr && S0 == st->base) return DL_ERR_ARG;
+  if (fill0 != nullptr)
+    for (int b = 0; b < c.B; ++b)
+      if (fill0[b] < 0 || fill0[b] >= c.L) return DL_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t state_bytes = size_t(c.B) * c.H * c.d_v * c.d_k * 4;
+  cudaError_t e = (S0 != nullptr)
+                      ? cudaMemcpyAsync(st->base, S0, state_bytes, cudaMemcpyDeviceToDevice, s)
+                      : cudaMemsetAsync(st->base, 0, state_bytes, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->log, 0, st->lay.log, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->meta, 0, st->lay.meta, s);
+  for (int b = 0; b < c.B; ++b)
+    for (int h = 0; h < c.H; ++h)
+      st->fill_stage[size_t(b) * c.H + h] = fill0 ? fill0[b] : 0;
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(st->dev_fill(), st->fill_stage.data(), st->fill_stage.size() * 4,
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return DL_ERR_CUDA;
+  for (int b = 0; b < c.B; ++b) st->fill[b] = fill0 ? fill0[b] : 0;
+  st->recount();
+  return DL_OK;
+}
+
+int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v, const float* decay,
+                   const float* beta, const float* bonus, float* o, void* stream) {
+  if (st == nullptr) return DL_ERR_ARG;
+  const dl_config& c = st->cfg;
+  int rc = check_step_args(c, q, k, v, decay, beta, bonus, o);
+  if (rc != DL_OK) return rc;
+  const bool fused = (c.flags & DL_FLAG_FUSED_MERGE) != 0;
+  if (st->n_full > 0) return DL_ERR_LOG_FULL;
+  dl::StepParams p{};
+  p.base = st->base;
+  p.logU = st->logU();
+  p.logK = st->logK();
+  p.logG = st->logG();
+  p.fill = st->dev_fill();
+  p.err = st->dev_err();
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.decay = decay;
+  p.beta = beta;
+  p.bonus = bonus;
+  p.o = o;
+  p.H = c.H;
+  p.L = c.L;
+  if (launch_step(c, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  for (int32_t& f : st->fill) {
+    f += 1;
+    if (fused && f == c.L) f = 0;
+  }
+  st->recount();
+  return DL_OK;
+}
+
+int dl_merge(dl_state* st, int mode, void* stream) {
+  if (st == nullptr) return DL_ERR_ARG;
+  if (mode != DL_MERGE_FULL && mode != DL_MERGE_ALL) return DL_ERR_ARG;
+  if (mode == DL_MERGE_FULL ? st->n_full == 0 : st->n_nonempty == 0) return DL_OK;
+  const dl_config& c = st->cfg;
+  dl::MergeParams p{};
+  p.base = st->base;
+  p.logU = st->logU();
+  p.logK = st->logK();
+  p.logG = st->logG();
+  p.fill = st->dev_fill();
+  p.err = st->dev_err();
+  p.out = st->base;
+  p.L = c.L;
+  p.mode = mode;
+  if (launch_merge(c, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  for (int32_t& f : st->fill)
+    if (mode == DL_MERGE_ALL || f == c.L) f = 0;
+  st->recount();
+  return DL_OK;
+}
+
+int dl_materialize(const dl_state* st, float* S_out, void* stream) {
+  if (st == nullptr || S_out == nullptr) return DL_ERR_ARG;
+  if (!aligned(S_out, 16)) return DL_ERR_ALIGN;
+  if (S_out == st->base) return DL_ERR_ARG;
+  const dl_config& c = st->cfg;
+  dl::MergeParams p{};
+  p.base = st->base;
+  p.logU = st->logU();
+  p.logK = st->logK();
+  p.logG = st->logG();
+  p.fill = st->dev_fill();
+  p.err = st->dev_err();
+  p.out = S_out;
+  p.L = c.L;
+  p.mode = 2;
+  if (launch_merge(c, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DL_OK;
+}
+
+int dl_eager_step(const dl_config* cfg, float* S, const void* q, const void* k, const void* v,
+                  const float* decay, const float* beta, const float* bonus, float* o,
+                  void* stream) {
+  int rc = check_config(cfg, false);
+  if (rc != DL_OK) return rc;
+  if (S == nullptr) return DL_ERR_ARG;
+  if (!aligned(S, 16)) return DL_ERR_ALIGN;
+  rc = check_step_args(*cfg, q, k, v, decay, beta, bonus, o);
+  if (rc != DL_OK) return rc;
+  dl::EagerParams p{};
+  p.S = S;
+  p.err = global_err_word();
+  if (p.err == nullptr) return DL_ERR_CUDA;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.decay = decay;
+  p.beta = beta;
+  p.bonus = bonus;
+  p.o = o;
+  p.H = cfg->H;
+  if (launch_eager(*cfg, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DL_OK;
+}
+
+int dl_state_fill(const dl_state* st, int32_t* fill_out) {
+  if (st == nullptr || fill_out == nullptr) return DL_ERR_ARG;
+  std::memcpy(fill_out, st->fill.data(), st->fill.size() * sizeof(int32_t));
+  return DL_OK;
+}
+
+int dl_state_destroy(dl_state* st) {
+  delete st;
+  return DL_OK;
+}
+
+int dl_device_error(dl_state* st, int32_t* code, int32_t* head, int clear, void* stream) {
+  int* word = (st != nullptr) ? st->dev_err() : global_err_word();
+  if (word == nullptr) return DL_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int host[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(host, word, sizeof(host), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(word, 0, sizeof(host), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return DL_ERR_CUDA;
+  if (code) *code = host[0];
+  if (head) *head = host[1];
+  return DL_OK;
+}
+
+uint64_t dl_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* dl_status_string(int status) {
+  switch (status) {
+    case DL_OK: return "ok";
+    case DL_ERR_ARG: return "invalid argument";
+    case DL_ERR_ALIGN: return "pointer alignment";
+    case DL_ERR_LOG_FULL: return "log full: merge before the next step";
+    case DL_ERR_CUDA: return "CUDA runtime error";
+    case DL_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DL_ERR_DEVICE: return "device-side error recorded";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,190 @@
+// dl_device.cuh -- device-side building blocks shared by the DeltaLog kernels:
+// bulk-copy (TMA) and mbarrier wrappers with bounded waits, element
+// conversion, and the warp reduction that turns per-lane row partials into
+// finished row dot products.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace dl {
+
+constexpr int kVarGDN = 0;
+constexpr int kVarKDA = 1;
+constexpr int kVarRWKV6 = 2;
+
+// Device error codes written to the error word.
+constexpr int kDevErrTimeout = 1;   // a bounded mbarrier wait gave up
+constexpr int kDevErrFill = 2;      // a fill counter outside [0, L]
+
+// A bounded wait gives up after this many SM clock cycles (~1 s at 2 GHz).
+constexpr long long kWaitCycles = 2000000000LL;
+
+// ------------------------------------------------------------ conversions
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  __device__ static float to_f(float x) { return x; }
+  __device__ static float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  __device__ static float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  __device__ static __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x) { return Elem<T>::to_f(x); }
+
+// Four consecutive elements as fp32 (16-B or 8-B vector load).
+__device__ __forceinline__ float4 load4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  uint2 r = *reinterpret_cast<const uint2*>(p);
+  float4 f;
+  f.x = __uint_as_float(r.x << 16);
+  f.y = __uint_as_float(r.x & 0xffff0000u);
+  f.z = __uint_as_float(r.y << 16);
+  f.w = __uint_as_float(r.y & 0xffff0000u);
+  return f;
+}
+
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+
+// ------------------------------------------------------- mbarrier + TMA
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes the mbarrier initialisations visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// One arrival that also announces `bytes` of transactions to come.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait on phase `parity`.  Returns false (and records the error) if
+// the phase did not complete within kWaitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int head) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) {
+      if (err != nullptr && atomicCAS(err, 0, kDevErrTimeout) == 0) err[1] = head;
+      return false;
+    }
+  }
+  return true;
+}
+
+// Bulk global -> shared copy (non-tensor TMA), completing on `bar`.
+// dst, src 16-B aligned; bytes a multiple of 16.
+__device__ __forceinline__ void tma_load_1d(void* dst, const void* src, uint32_t bytes,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Same, with an L2 evict-first policy: streamed data that is not reused.
+__device__ __forceinline__ void tma_load_1d_stream(void* dst, const void* src, uint32_t bytes,
+                                                   uint64_t* bar) {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// --------------------------------------------------------- row reduction
+//
+// A warp covers rows of a d_v x d_k tile: LPR lanes per row, each lane
+// holding 4 consecutive columns, so 32/LPR rows per warp instruction.  After
+// a lane has accumulated NV partial sums (one per row it touched), this
+// butterfly leaves every lane with one finished row sum: at each level a
+// lane keeps half of its partials and trades the other half with its
+// partner, so NV partials need log2(NV) exchanges of shrinking size instead
+// of NV full warp reductions.  Requires LPR == 2 * NV: the last level adds
+// the pair (lane, lane ^ 1), which then hold the same row.
+template <int NV, int LPR>
+__device__ __forceinline__ float reduce_rows(float (&v)[NV], int lane) {
+  static_assert(LPR == 2 * NV, "layout: two lanes finish each row");
+#pragma unroll
+  for (int n = NV, o = LPR / 2; n > 1; n >>= 1, o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = upper ? v[i] : v[i + n / 2];
+      const float keep = upper ? v[i + n / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+// Which of the NV partials `reduce_rows` leaves in this lane.
+template <int NV, int LPR>
+__device__ __forceinline__ int reduced_index(int lane) {
+  int p = 0;
+#pragma unroll
+  for (int n = NV, o = LPR / 2; n > 1; n >>= 1, o >>= 1)
+    if (lane & o) p += n / 2;
+  return p;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Tile geometry for a d_v x d_k fp32 tile handled by DV/16 warps of 16 rows.
+template <int DK, int DV>
+struct Tile {
+  static_assert(DK == 64 || DK == 128, "d_k in {64,128}");
+  static_assert(DV == 64 || DV == 128, "d_v in {64,128}");
+  static constexpr int kWarps = DV / 16;           // 16 rows per warp
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kRowsPerWarp = 16;
+  static constexpr int kLPR = DK / 4;              // lanes per row (float4 each)
+  static constexpr int kRPI = 32 / kLPR;           // rows per warp instruction
+  static constexpr int kNV = kRowsPerWarp / kRPI;  // partials per lane
+  static constexpr int kChunkRows = 32;            // rows per bulk copy
+  static constexpr int kChunks = DV / kChunkRows;
+  static constexpr uint32_t kChunkBytes = kChunkRows * DK * 4;
+  static constexpr size_t kTileBytes = size_t(DV) * DK * 4;
+  static constexpr int kCPL = DK / 32;              // key columns per lane in 32-lane dots
+  static_assert(kLPR == 2 * kNV, "row reduction layout");
+};
+
+}  // namespace dl

@@ -1,0 +1,652 @@
+// dl_kernels.cuh -- the DeltaLog kernels for sm_100a.
+//
+// Notation ("DeltaLog: Deferred Materialization of Recurrent States for Linear
+// Attention Decoding", Abstract): each head keeps a dense base S_b (fp32,
+// d_v x d_k, row = value index) and a bounded log of f < L compact entries
+// (u_i, k_i, g_i), g_i = log of the decay accumulated since the base was
+// merged (a scalar for GDN, a d_k vector for KDA and RWKV6).  The dense state
+// the model sees is
+//     S = S_b Diag(e^{g}) + sum_i u_i (k_i o e^{g - g_i})^T,
+// g being the newest accumulated log-decay.  Keeping log-decay and forming
+// only differences g - g_i <= 0 keeps every factor in (0, 1], so long runs of
+// strong decay (RWKV6) cannot overflow or lose the ratio to underflow.
+//
+// Kernels (one CTA per (sequence, head), blockIdx.x = b*H + h):
+//   dl_step_kernel   : decode step. Streams S_b into shared memory with bulk
+//                      copies (TMA), forms S_b k-hat and S_b q-hat with one
+//                      pass over the tile, adds the log correction from the
+//                      log entries staged in shared memory, writes o_t and
+//                      appends (u_t, k_t, g_t).  With FUSED, a head whose
+//                      append would fill the log writes the merged base
+//                      instead (it already holds S_b and the whole log).
+//   dl_merge_kernel  : folds a log into the base (or into a separate output
+//                      for materialize) -- a rank-f update of the tile.
+//   dl_eager_kernel  : the dense read-modify-write step eager decoding does.
+#pragma once
+
+#include "dl_device.cuh"
+
+namespace dl {
+
+struct StepParams {
+  float* base;   // [BH, DV, DK]
+  void* logU;    // [BH, L, DV]  fp32 (in_dtype for RWKV6)
+  void* logK;    // [BH, L, DK]  in_dtype
+  float* logG;   // [BH, L, GW]
+  int* fill;     // [BH]
+  int* err;      // device error word (2 ints)
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* decay;
+  const float* beta;
+  const float* bonus;
+  float* o;
+  int H;
+  int L;
+};
+
+struct MergeParams {
+  float* base;
+  const void* logU;
+  const void* logK;
+  const float* logG;
+  int* fill;
+  int* err;
+  float* out;    // merge: == base; materialize: caller buffer
+  int L;
+  int mode;      // 0 merge full logs, 1 merge every non-empty log, 2 materialize
+};
+
+struct EagerParams {
+  float* S;
+  int* err;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* decay;
+  const float* beta;
+  const float* bonus;
+  float* o;
+  int H;
+};
+
+template <int VAR, typename TIn>
+struct LogU { using type = float; };
+template <typename TIn>
+struct LogU<kVarRWKV6, TIn> { using type = TIn; };  // RWKV6 logs v itself
+
+__host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ step
+
+template <int VAR, int DK, int DV, typename TIn>
+struct StepLayout {
+  using TU = typename LogU<VAR, TIn>::type;
+  static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
+  size_t offU, offK, offG, offVec, offW, offZ, offScal, offBar, total;
+  __host__ __device__ explicit StepLayout(int L) {
+    offU = Tile<DK, DV>::kTileBytes;
+    offK = offU + align_up(size_t(L) * DV * sizeof(TU), 128);
+    offG = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
+    offVec = offG + align_up(size_t(L) * GW * 4, 128);
+    // k, q (raw), k-hat, q-hat [DK] each; v [DV]; g_t, g_{t-1} [GW] each
+    offW = offVec + align_up(size_t(4 * DK + DV + 2 * GW) * 4, 128);
+    offZ = offW + align_up(size_t(L) * 4, 16);
+    offScal = offZ + align_up(size_t(L) * 4, 16);
+    offBar = offScal + 64;
+    total = offBar + 8 * (Tile<DK, DV>::kChunks + 1);
+  }
+};
+
+template <int VAR, int DK, int DV, typename TIn, bool FUSED>
+__global__ void __launch_bounds__(Tile<DK, DV>::kThreads)
+dl_step_kernel(const StepParams p) {
+  using Tl = Tile<DK, DV>;
+  using TU = typename LogU<VAR, TIn>::type;
+  constexpr int GW = StepLayout<VAR, DK, DV, TIn>::GW;
+  constexpr int NT = Tl::kThreads;
+  constexpr int NW = Tl::kWarps;
+  constexpr int NV = Tl::kNV;
+  constexpr int LPR = Tl::kLPR;
+  constexpr int RPI = Tl::kRPI;
+  constexpr int CPL = Tl::kCPL;
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int L = p.L;
+  const StepLayout<VAR, DK, DV, TIn> lay(L);
+  float* sS = reinterpret_cast<float*>(smem);
+  TU* sU = reinterpret_cast<TU*>(smem + lay.offU);
+  TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);
+  float* sG = reinterpret_cast<float*>(smem + lay.offG);
+  float* sk = reinterpret_cast<float*>(smem + lay.offVec);  // raw k_t
+  float* sq = sk + DK;                                       // raw q_t / r_t
+  float* sKh = sq + DK;                                      // GEMV vector for a
+  float* sQh = sKh + DK;                                     // GEMV vector for b
+  float* sV = sQh + DK;                                      // v_t
+  float* sGt = sV + DV;                                      // g_t
+  float* sGp = sGt + GW;                                     // g_{t-1}
+  float* sW = reinterpret_cast<float*>(smem + lay.offW);     // per-entry weights on k
+  float* sZ = reinterpret_cast<float*>(smem + lay.offZ);     // per-entry weights on q / r
+  float* sScal = reinterpret_cast<float*>(smem + lay.offScal);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const size_t head = blockIdx.x;
+  const int h = static_cast<int>(head % static_cast<size_t>(p.H));
+  const int f = p.fill[head];
+  if (f < 0 || f >= L) {  // the host never launches a step on a full log
+    if (tid == 0 && p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
+    return;
+  }
+  const bool merge_now = FUSED && (f + 1 == L);
+
+  const float* gS = p.base + head * size_t(DV) * DK;
+  TU* gU = static_cast<TU*>(p.logU) + head * size_t(L) * DV;
+  TIn* gK = static_cast<TIn*>(p.logK) + head * size_t(L) * DK;
+  float* gG = p.logG + head * size_t(L) * GW;
+  uint64_t* barLog = &bars[Tl::kChunks];
+
+  if (tid == 0) {
+#pragma unroll
+    for (int c = 0; c <= Tl::kChunks; ++c) mbar_init(&bars[c], 1);
+    fence_mbar_init();
+    if (f > 0) {
+      const uint32_t bu = uint32_t(f) * DV * sizeof(TU);
+      const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
+      const uint32_t bg = (GW > 1) ? uint32_t(f) * GW * 4 : 0u;
+      mbar_arrive_expect_tx(barLog, bu + bk + bg);
+      tma_load_1d(sU, gU, bu, barLog);
+      tma_load_1d(sK, gK, bk, barLog);
+      if (GW > 1) tma_load_1d(sG, gG, bg, barLog);
+    }
+#pragma unroll
+    for (int c = 0; c < Tl::kChunks; ++c) {
+      mbar_arrive_expect_tx(&bars[c], Tl::kChunkBytes);
+      tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
+                         Tl::kChunkBytes, &bars[c]);
+    }
+  }
+
+  // ---- per-head vectors while the tile streams in
+  const TIn* gq = static_cast<const TIn*>(p.q) + head * DK;
+  const TIn* gk = static_cast<const TIn*>(p.k) + head * DK;
+  const TIn* gv = static_cast<const TIn*>(p.v) + head * DV;
+  for (int c = tid; c < DK; c += NT) {
+    const float kc = to_f(gk[c]);
+    const float qc = to_f(gq[c]);
+    sk[c] = kc;
+    sq[c] = qc;
+    if (VAR == kVarGDN) {
+      sKh[c] = kc;
+      sQh[c] = qc;
+    } else {
+      const float gp = (f > 0) ? gG[size_t(f - 1) * GW + c] : 0.f;
+      const float gt = gp + logf(p.decay[head * DK + c]);
+      sGp[c] = gp;
+      sGt[c] = gt;
+      if (VAR == kVarKDA) {
+        const float e = expf(gt);
+        sKh[c] = e * kc;
+        sQh[c] = e * qc;
+      } else {  // RWKV6 reads S_{t-1}: decay up to the previous step
+        sKh[c] = kc;
+        sQh[c] = expf(gp) * qc;
+      }
+    }
+    if (merge_now) {
+      sK[size_t(f) * DK + c] = gk[c];
+    } else {
+      gK[size_t(f) * DK + c] = gk[c];
+      if (GW > 1) gG[size_t(f) * GW + c] = sGt[c];
+    }
+  }
+  for (int j = tid; j < DV; j += NT) sV[j] = to_f(gv[j]);
+  if (VAR == kVarGDN) {
+    for (int i = tid; i < f; i += NT) sG[i] = gG[i];
+    if (tid == 0) {
+      const float gp = (f > 0) ? gG[f - 1] : 0.f;
+      const float gt = gp + logf(p.decay[head]);
+      sGp[0] = gp;
+      sGt[0] = gt;
+      sScal[2] = expf(gt);
+      if (!merge_now) gG[f] = gt;
+    }
+  }
+  if (tid == 0) sScal[1] = (VAR == kVarRWKV6) ? 0.f : p.beta[head];
+  __syncthreads();
+  // Every thread has read fill[head] before the barrier above, and no other
+  // CTA reads it, so advancing it here is race-free.
+  if (tid == 0) p.fill[head] = merge_now ? 0 : f + 1;
+
+  // ---- log prologue: one weight per entry and query vector
+  bool ok = true;
+  if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
+  if (!__syncthreads_and(ok)) {
+    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
+    return;
+  }
+  for (int i = warp; i < f; i += NW) {
+    float x = 0.f, y = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) {
+      const int c = lane * CPL + cc;
+      const float ki = to_f(sK[size_t(i) * DK + c]);
+      if (VAR == kVarGDN) {
+        x = fmaf(ki, sk[c], x);
+        y = fmaf(ki, sq[c], y);
+      } else if (VAR == kVarKDA) {
+        const float e = expf(sGt[c] - sG[size_t(i) * DK + c]);
+        x = fmaf(ki * e, sk[c], x);
+        y = fmaf(ki * e, sq[c], y);
+      } else {
+        const float e = expf(sGp[c] - sG[size_t(i) * DK + c]);
+        y = fmaf(ki * e, sq[c], y);
+      }
+    }
+    if (VAR != kVarRWKV6) x = warp_sum(x);
+    y = warp_sum(y);
+    if (VAR == kVarGDN) {
+      const float e = expf(sGt[0] - sG[i]);
+      x *= e;
+      y *= e;
+    }
+    if (lane == 0) {
+      sW[i] = x;
+      sZ[i] = y;
+    }
+  }
+  if (warp == NW - 1) {
+    // GDN/KDA: k_t . q_t (the current entry's own weight on q);
+    // RWKV6: the bonus sum_c r_c u_c k_c.
+    float x = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) {
+      const int c = lane * CPL + cc;
+      x = (VAR == kVarRWKV6) ? fmaf(sq[c] * p.bonus[size_t(h) * DK + c], sk[c], x)
+                             : fmaf(sk[c], sq[c], x);
+    }
+    x = warp_sum(x);
+    if (lane == 0) sScal[0] = x;
+  }
+  __syncthreads();
+
+  // ---- one pass over this warp's 16 rows of S_b
+  const int j0 = warp * Tl::kRowsPerWarp;
+  uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
+  if (!mbar_wait(barMine, 0, p.err, int(head))) {
+    mbar_wait(barMine, 0, nullptr, 0);
+    return;
+  }
+  const int c0 = (lane % LPR) * 4;
+  const int rsub = lane / LPR;
+  const float4 kh4 = *reinterpret_cast<const float4*>(sKh + c0);
+  const float4 qh4 = *reinterpret_cast<const float4*>(sQh + c0);
+  float pa[NV], pb[NV];
+#pragma unroll
+  for (int pi = 0; pi < NV; ++pi) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
+    pa[pi] = (VAR == kVarRWKV6) ? 0.f : dot4(s4, kh4);
+    pb[pi] = dot4(s4, qh4);
+  }
+  const float a = (VAR == kVarRWKV6) ? 0.f : reduce_rows<NV, LPR>(pa, lane);
+  const float b = reduce_rows<NV, LPR>(pb, lane);
+  const int j = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;
+
+  // ---- log correction, delta-rule correction and readout for row j
+  float ck = 0.f, cq = 0.f;
+  for (int i = 0; i < f; ++i) {
+    const float uij = to_f(sU[size_t(i) * DV + j]);
+    if (VAR != kVarRWKV6) ck = fmaf(sW[i], uij, ck);
+    cq = fmaf(sZ[i], uij, cq);
+  }
+  const float vj = sV[j];
+  const float sdot = sScal[0];
+  float u, o;
+  if (VAR == kVarGDN) {
+    const float gamma = sScal[2];
+    u = sScal[1] * (vj - gamma * a - ck);
+    o = gamma * b + cq + sdot * u;
+  } else if (VAR == kVarKDA) {
+    u = sScal[1] * (vj - a - ck);
+    o = b + cq + sdot * u;
+  } else {
+    u = vj;
+    o = b + cq + sdot * vj;
+  }
+  if ((lane & 1) == 0) {
+    p.o[head * DV + j] = o;
+    if (merge_now)
+      sU[size_t(f) * DV + j] = Elem<TU>::from_f(u);
+    else
+      gU[size_t(f) * DV + j] = Elem<TU>::from_f(u);
+  }
+  if (!merge_now) return;
+
+  // ---- fused merge: S_b <- S_b Diag(e^{g_t}) + sum_{i<=f} u_i (k_i o e^{g_t-g_i})^T
+  __syncwarp();
+  float4 dec;
+  if (VAR == kVarGDN) {
+    dec.x = dec.y = dec.z = dec.w = sScal[2];
+  } else {
+    dec = make_float4(expf(sGt[c0]), expf(sGt[c0 + 1]), expf(sGt[c0 + 2]), expf(sGt[c0 + 3]));
+  }
+  float4 acc[NV];
+#pragma unroll
+  for (int pi = 0; pi < NV; ++pi) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
+    acc[pi] = make_float4(s4.x * dec.x, s4.y * dec.y, s4.z * dec.z, s4.w * dec.w);
+  }
+  for (int i = 0; i <= f; ++i) {
+    float4 k4 = load4(sK + size_t(i) * DK + c0);
+    if (i < f) {
+      if (VAR == kVarGDN) {
+        const float e = expf(sGt[0] - sG[i]);
+        k4.x *= e; k4.y *= e; k4.z *= e; k4.w *= e;
+      } else {
+        const float* gi = sG + size_t(i) * DK + c0;
+        k4.x *= expf(sGt[c0] - gi[0]);
+        k4.y *= expf(sGt[c0 + 1] - gi[1]);
+        k4.z *= expf(sGt[c0 + 2] - gi[2]);
+        k4.w *= expf(sGt[c0 + 3] - gi[3]);
+      }
+    }
+#pragma unroll
+    for (int pi = 0; pi < NV; ++pi) {
+      const float ui = to_f(sU[size_t(i) * DV + j0 + pi * RPI + rsub]);
+      acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
+      acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
+      acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
+      acc[pi].w = fmaf(ui, k4.w, acc[pi].w);
+    }
+  }
+  float* gSw = p.base + head * size_t(DV) * DK;
+#pragma unroll
+  for (int pi = 0; pi < NV; ++pi)
+    *reinterpret_cast<float4*>(gSw + size_t(j0 + pi * RPI + rsub) * DK + c0) = acc[pi];
+}
+
+// ----------------------------------------------------------- merge / materialize
+
+template <int VAR, int DK, int DV, typename TIn>
+struct MergeLayout {
+  using TU = typename LogU<VAR, TIn>::type;
+  static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
+  size_t offU, offK, offKt, offG, offDec, offBar, total;
+  __host__ __device__ explicit MergeLayout(int L) {
+    offU = Tile<DK, DV>::kTileBytes;
+    offK = offU + align_up(size_t(L) * DV * sizeof(TU), 128);
+    offKt = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
+    offG = offKt + align_up(size_t(L) * DK * 4, 128);
+    offDec = offG + align_up(size_t(L) * GW * 4, 128);
+    offBar = offDec + align_up(size_t(DK) * 4, 128);
+    total = offBar + 8 * (Tile<DK, DV>::kChunks + 1);
+  }
+};
+
+template <int VAR, int DK, int DV, typename TIn>
+__global__ void __launch_bounds__(Tile<DK, DV>::kThreads)
+dl_merge_kernel(const MergeParams p) {
+  using Tl = Tile<DK, DV>;
+  using TU = typename LogU<VAR, TIn>::type;
+  constexpr int GW = MergeLayout<VAR, DK, DV, TIn>::GW;
+  constexpr int NT = Tl::kThreads;
+  constexpr int NV = Tl::kNV;
+  constexpr int LPR = Tl::kLPR;
+  constexpr int RPI = Tl::kRPI;
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int L = p.L;
+  const size_t head = blockIdx.x;
+  const int f = p.fill[head];
+  if (f < 0 || f > L) {
+    if (threadIdx.x == 0 && p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0)
+      p.err[1] = int(head);
+    return;
+  }
+  if (p.mode == 0 && f != L) return;
+  if (p.mode == 1 && f == 0) return;
+
+  const MergeLayout<VAR, DK, DV, TIn> lay(L);
+  float* sS = reinterpret_cast<float*>(smem);
+  TU* sU = reinterpret_cast<TU*>(smem + lay.offU);
+  TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);
+  float* sKt = reinterpret_cast<float*>(smem + lay.offKt);
+  float* sG = reinterpret_cast<float*>(smem + lay.offG);
+  float* sDec = reinterpret_cast<float*>(smem + lay.offDec);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
+  uint64_t* barLog = &bars[Tl::kChunks];
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const float* gS = p.base + head * size_t(DV) * DK;
+  const TU* gU = static_cast<const TU*>(p.logU) + head * size_t(L) * DV;
+  const TIn* gK = static_cast<const TIn*>(p.logK) + head * size_t(L) * DK;
+  const float* gG = p.logG + head * size_t(L) * GW;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int c = 0; c <= Tl::kChunks; ++c) mbar_init(&bars[c], 1);
+    fence_mbar_init();
+    if (f > 0) {
+      const uint32_t bu = uint32_t(f) * DV * sizeof(TU);
+      const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
+      const uint32_t bg = (GW > 1) ? uint32_t(f) * GW * 4 : 0u;
+      mbar_arrive_expect_tx(barLog, bu + bk + bg);
+      tma_load_1d(sU, gU, bu, barLog);
+      tma_load_1d(sK, gK, bk, barLog);
+      if (GW > 1) tma_load_1d(sG, gG, bg, barLog);
+    }
+#pragma unroll
+    for (int c = 0; c < Tl::kChunks; ++c) {
+      mbar_arrive_expect_tx(&bars[c], Tl::kChunkBytes);
+      tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
+                         Tl::kChunkBytes, &bars[c]);
+    }
+  }
+  if (GW == 1)
+    for (int i = tid; i < f; i += NT) sG[i] = gG[i];
+  __syncthreads();
+  bool ok = true;
+  if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
+  if (!__syncthreads_and(ok)) {
+    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
+    return;
+  }
+  // decay of the base and decayed keys k-tilde_i = k_i o e^{g_last - g_i}
+  for (int c = tid; c < DK; c += NT) {
+    const float gl = (f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f;
+    sDec[c] = expf(gl);
+    for (int i = 0; i < f; ++i)
+      sKt[size_t(i) * DK + c] = to_f(sK[size_t(i) * DK + c]) * expf(gl - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
+  }
+  if (tid == 0 && p.mode != 2) p.fill[head] = 0;
+  __syncthreads();
+
+  const int j0 = warp * Tl::kRowsPerWarp;
+  uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
+  if (!mbar_wait(barMine, 0, p.err, int(head))) {
+    mbar_wait(barMine, 0, nullptr, 0);
+    return;
+  }
+  const int c0 = (lane % LPR) * 4;
+  const int rsub = lane / LPR;
+  const float4 dec = *reinterpret_cast<const float4*>(sDec + c0);
+  float4 acc[NV];
+#pragma unroll
+  for (int pi = 0; pi < NV; ++pi) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
+    acc[pi] = make_float4(s4.x * dec.x, s4.y * dec.y, s4.z * dec.z, s4.w * dec.w);
+  }
+  for (int i = 0; i < f; ++i) {
+    const float4 k4 = *reinterpret_cast<const float4*>(sKt + size_t(i) * DK + c0);
+#pragma unroll
+    for (int pi = 0; pi < NV; ++pi) {
+      const float ui = to_f(sU[size_t(i) * DV + j0 + pi * RPI + rsub]);
+      acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
+      acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
+      acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
+      acc[pi].w = fmaf(ui, k4.w, acc[pi].w);
+    }
+  }
+  float* gO = p.out + head * size_t(DV) * DK;
+#pragma unroll
+  for (int pi = 0; pi < NV; ++pi)
+    *reinterpret_cast<float4*>(gO + size_t(j0 + pi * RPI + rsub) * DK + c0) = acc[pi];
+}
+
+// ------------------------------------------------------------------ eager
+
+template <int DK, int DV>
+struct EagerLayout {
+  size_t offVec, offUrow, offScal, offBar, total;
+  __host__ __device__ EagerLayout() {
+    offVec = Tile<DK, DV>::kTileBytes;
+    offUrow = offVec + align_up(size_t(5 * DK + DV) * 4, 128);  // k, q, kh, qh, dec; v
+    offScal = offUrow + align_up(size_t(DV) * 4, 128);
+    offBar = offScal + 64;
+    total = offBar + 8 * Tile<DK, DV>::kChunks;
+  }
+};
+
+template <int VAR, int DK, int DV, typename TIn>
+__global__ void __launch_bounds__(Tile<DK, DV>::kThreads)
+dl_eager_kernel(const EagerParams p) {
+  using Tl = Tile<DK, DV>;
+  constexpr int NT = Tl::kThreads;
+  constexpr int NW = Tl::kWarps;
+  constexpr int NV = Tl::kNV;
+  constexpr int LPR = Tl::kLPR;
+  constexpr int RPI = Tl::kRPI;
+  constexpr int CPL = Tl::kCPL;
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const EagerLayout<DK, DV> lay;
+  float* sS = reinterpret_cast<float*>(smem);
+  float* sk = reinterpret_cast<float*>(smem + lay.offVec);
+  float* sq = sk + DK;
+  float* sKh = sq + DK;
+  float* sQh = sKh + DK;
+  float* sDec = sQh + DK;
+  float* sV = sDec + DK;
+  float* sUrow = reinterpret_cast<float*>(smem + lay.offUrow);
+  float* sScal = reinterpret_cast<float*>(smem + lay.offScal);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const size_t head = blockIdx.x;
+  const int h = static_cast<int>(head % static_cast<size_t>(p.H));
+  float* gS = p.S + head * size_t(DV) * DK;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_init(&bars[c], 1);
+    fence_mbar_init();
+#pragma unroll
+    for (int c = 0; c < Tl::kChunks; ++c) {
+      mbar_arrive_expect_tx(&bars[c], Tl::kChunkBytes);
+      tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
+                         Tl::kChunkBytes, &bars[c]);
+    }
+  }
+  const TIn* gq = static_cast<const TIn*>(p.q) + head * DK;
+  const TIn* gk = static_cast<const TIn*>(p.k) + head * DK;
+  const TIn* gv = static_cast<const TIn*>(p.v) + head * DV;
+  for (int c = tid; c < DK; c += NT) {
+    const float kc = to_f(gk[c]);
+    const float qc = to_f(gq[c]);
+    const float dc = (VAR == kVarGDN) ? p.decay[head] : p.decay[head * DK + c];
+    sk[c] = kc;
+    sq[c] = qc;
+    sDec[c] = dc;
+    if (VAR == kVarKDA) {  // S Diag(alpha) k and S Diag(alpha) q
+      sKh[c] = dc * kc;
+      sQh[c] = dc * qc;
+    } else {               // GDN scales after the GEMV; RWKV6 reads S_{t-1}
+      sKh[c] = kc;
+      sQh[c] = qc;
+    }
+  }
+  for (int j = tid; j < DV; j += NT) sV[j] = to_f(gv[j]);
+  __syncthreads();
+  if (warp == NW - 1) {
+    float x = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) {
+      const int c = lane * CPL + cc;
+      x = (VAR == kVarRWKV6) ? fmaf(sq[c] * p.bonus[size_t(h) * DK + c], sk[c], x)
+                             : fmaf(sk[c], sq[c], x);
+    }
+    x = warp_sum(x);
+    if (lane == 0) {
+      sScal[0] = x;
+      sScal[1] = (VAR == kVarRWKV6) ? 0.f : p.beta[head];
+      sScal[2] = (VAR == kVarGDN) ? p.decay[head] : 1.f;
+    }
+  }
+  __syncthreads();
+
+  const int j0 = warp * Tl::kRowsPerWarp;
+  uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
+  if (!mbar_wait(barMine, 0, p.err, int(head))) {
+    mbar_wait(barMine, 0, nullptr, 0);
+    return;
+  }
+  const int c0 = (lane % LPR) * 4;
+  const int rsub = lane / LPR;
+  const float4 kh4 = *reinterpret_cast<const float4*>(sKh + c0);
+  const float4 qh4 = *reinterpret_cast<const float4*>(sQh + c0);
+  float pa[NV], pb[NV];
+#pragma unroll
+  for (int pi = 0; pi < NV; ++pi) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
+    pa[pi] = (VAR == kVarRWKV6) ? 0.f : dot4(s4, kh4);
+    pb[pi] = dot4(s4, qh4);
+  }
+  const float a = (VAR == kVarRWKV6) ? 0.f : reduce_rows<NV, LPR>(pa, lane);
+  const float b = reduce_rows<NV, LPR>(pb, lane);
+  const int j = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;
+  const float vj = sV[j];
+  const float sdot = sScal[0];
+  float u, o;
+  if (VAR == kVarGDN) {
+    const float alpha = sScal[2];
+    u = sScal[1] * (vj - alpha * a);
+    o = alpha * b + sdot * u;
+  } else if (VAR == kVarKDA) {
+    u = sScal[1] * (vj - a);
+    o = b + sdot * u;
+  } else {
+    u = vj;
+    o = b + sdot * vj;
+  }
+  if ((lane & 1) == 0) {
+    p.o[head * DV + j] = o;
+    sUrow[j] = u;
+  }
+  __syncwarp();
+  // S <- S Diag(decay) + u k^T  (GDN: alpha S + u k^T)
+  const float4 k4 = *reinterpret_cast<const float4*>(sk + c0);
+  const float4 d4 = *reinterpret_cast<const float4*>(sDec + c0);
+#pragma unroll
+  for (int pi = 0; pi < NV; ++pi) {
+    const int row = j0 + pi * RPI + rsub;
+    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(row) * DK + c0);
+    const float ur = sUrow[row];
+    float4 r;
+    r.x = fmaf(ur, k4.x, s4.x * d4.x);
+    r.y = fmaf(ur, k4.y, s4.y * d4.y);
+    r.z = fmaf(ur, k4.z, s4.z * d4.z);
+    r.w = fmaf(ur, k4.w, s4.w * d4.w);
+    *reinterpret_cast<float4*>(gS + size_t(row) * DK + c0) = r;
+  }
+}
+
+}  // namespace dl

@@ -1,0 +1,202 @@
+// dl_launch.cuh -- host-side launchers for the DeltaLog kernels.  Each
+// variant's launchers are instantiated in their own translation unit
+// (dl_kernels_<variant>.cu) so the builds run in parallel.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "dl_kernels.cuh"
+
+namespace dl {
+
+// Shapes the launchers are built for.
+struct Shape {
+  int dk;
+  int dv;
+  int bf16;  // 1: q/k/v are bf16, 0: fp32
+};
+
+// Dynamic shared memory each kernel may use; set once per device.
+constexpr int kMaxSmemOptIn = 227 * 1024;
+constexpr int kMaxDevices = 64;
+
+template <typename Kern>
+inline cudaError_t prepare_kernel(Kern kern, std::atomic<unsigned long long>& done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long bit = 1ull << dev;
+  if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmemOptIn);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return cudaSuccess;
+}
+
+template <int VAR, int DK, int DV, typename TIn, bool FUSED>
+cudaError_t launch_step_t(const StepParams& p, unsigned nheads, cudaStream_t s) {
+  static std::atomic<unsigned long long> done{0};
+  auto kern = dl_step_kernel<VAR, DK, DV, TIn, FUSED>;
+  cudaError_t e = prepare_kernel(kern, done);
+  if (e != cudaSuccess) return e;
+  const size_t smem = StepLayout<VAR, DK, DV, TIn>(p.L).total;
+  kern<<<nheads, Tile<DK, DV>::kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int VAR, int DK, int DV, typename TIn>
+cudaError_t launch_merge_t(const MergeParams& p, unsigned nheads, cudaStream_t s) {
+  static std::atomic<unsigned long long> done{0};
+  auto kern = dl_merge_kernel<VAR, DK, DV, TIn>;
+  cudaError_t e = prepare_kernel(kern, done);
+  if (e != cudaSuccess) return e;
+  const size_t smem = MergeLayout<VAR, DK, DV, TIn>(p.L).total;
+  kern<<<nheads, Tile<DK, DV>::kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int VAR, int DK, int DV, typename TIn>
+cudaError_t launch_eager_t(const EagerParams& p, unsigned nheads, cudaStream_t s) {
+  static std::atomic<unsigned long long> done{0};
+  auto kern = dl_eager_kernel<VAR, DK, DV, TIn>;
+  cudaError_t e = prepare_kernel(kern, done);
+  if (e != cudaSuccess) return e;
+  const size_t smem = EagerLayout<DK, DV>().total;
+  kern<<<nheads, Tile<DK, DV>::kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+// Shape dispatch: calls F::template run<DK, DV, TIn>() for the runtime shape.
+template <typename F>
+inline cudaError_t dispatch_shape(const Shape& sh, F&& f) {
+#define DL_SHAPE_CASE(DK_, DV_)                                                  \
+  if (sh.dk == DK_ && sh.dv == DV_)                                              \
+    return sh.bf16 ? f.template run<DK_, DV_, __nv_bfloat16>()                   \
+                   : f.template run<DK_, DV_, float>();
+  DL_SHAPE_CASE(64, 64)
+  DL_SHAPE_CASE(128, 128)
+  DL_SHAPE_CASE(64, 128)
+  DL_SHAPE_CASE(128, 64)
+#undef DL_SHAPE_CASE
+  return cudaErrorInvalidValue;
+}
+
+// Per-variant entry points (defined in dl_kernels_<variant>.cu).
+template <int VAR>
+cudaError_t launch_step(const Shape& sh, bool fused, const StepParams& p, unsigned nheads,
+                        cudaStream_t s);
+template <int VAR>
+cudaError_t launch_merge(const Shape& sh, const MergeParams& p, unsigned nheads, cudaStream_t s);
+template <int VAR>
+cudaError_t launch_eager(const Shape& sh, const EagerParams& p, unsigned nheads, cudaStream_t s);
+
+// Shared-memory bytes a launch needs (host-side check before launching).
+template <int VAR>
+size_t step_smem_bytes(const Shape& sh, int L);
+template <int VAR>
+size_t merge_smem_bytes(const Shape& sh, int L);
+
+#define DL_DECLARE_VARIANT_LAUNCHERS(VAR)                                                     \
+  template <>                                                                                 \
+  cudaError_t launch_step<VAR>(const Shape&, bool, const StepParams&, unsigned, cudaStream_t); \
+  template <>                                                                                 \
+  cudaError_t launch_merge<VAR>(const Shape&, const MergeParams&, unsigned, cudaStream_t);    \
+  template <>                                                                                 \
+  cudaError_t launch_eager<VAR>(const Shape&, const EagerParams&, unsigned, cudaStream_t);    \
+  template <>                                                                                 \
+  size_t step_smem_bytes<VAR>(const Shape&, int);                                             \
+  template <>                                                                                 \
+  size_t merge_smem_bytes<VAR>(const Shape&, int);
+
+DL_DECLARE_VARIANT_LAUNCHERS(kVarGDN)
+DL_DECLARE_VARIANT_LAUNCHERS(kVarKDA)
+DL_DECLARE_VARIANT_LAUNCHERS(kVarRWKV6)
+
+// Functors the shape dispatch calls (namespace scope: local classes cannot
+// have member templates).
+template <int VAR>
+struct StepRun {
+  const StepParams& p;
+  unsigned n;
+  cudaStream_t s;
+  bool fused;
+  template <int DK, int DV, typename T>
+  cudaError_t run() {
+    return fused ? launch_step_t<VAR, DK, DV, T, true>(p, n, s)
+                 : launch_step_t<VAR, DK, DV, T, false>(p, n, s);
+  }
+};
+template <int VAR>
+struct MergeRun {
+  const MergeParams& p;
+  unsigned n;
+  cudaStream_t s;
+  template <int DK, int DV, typename T>
+  cudaError_t run() { return launch_merge_t<VAR, DK, DV, T>(p, n, s); }
+};
+template <int VAR>
+struct EagerRun {
+  const EagerParams& p;
+  unsigned n;
+  cudaStream_t s;
+  template <int DK, int DV, typename T>
+  cudaError_t run() { return launch_eager_t<VAR, DK, DV, T>(p, n, s); }
+};
+template <int VAR>
+struct StepSmem {
+  int L;
+  size_t out;
+  template <int DK, int DV, typename T>
+  cudaError_t run() {
+    out = StepLayout<VAR, DK, DV, T>(L).total;
+    return cudaSuccess;
+  }
+};
+template <int VAR>
+struct MergeSmem {
+  int L;
+  size_t out;
+  template <int DK, int DV, typename T>
+  cudaError_t run() {
+    out = MergeLayout<VAR, DK, DV, T>(L).total;
+    return cudaSuccess;
+  }
+};
+
+#define DL_DEFINE_VARIANT_LAUNCHERS(VAR)                                                   \
+  template <>                                                                              \
+  cudaError_t launch_step<VAR>(const Shape& sh, bool fused, const StepParams& p,           \
+                               unsigned nheads, cudaStream_t s) {                          \
+    StepRun<VAR> f{p, nheads, s, fused};                                                   \
+    return dispatch_shape(sh, f);                                                          \
+  }                                                                                        \
+  template <>                                                                              \
+  cudaError_t launch_merge<VAR>(const Shape& sh, const MergeParams& p, unsigned nheads,    \
+                                cudaStream_t s) {                                          \
+    MergeRun<VAR> f{p, nheads, s};                                                         \
+    return dispatch_shape(sh, f);                                                          \
+  }                                                                                        \
+  template <>                                                                              \
+  cudaError_t launch_eager<VAR>(const Shape& sh, const EagerParams& p, unsigned nheads,    \
+                                cudaStream_t s) {                                          \
+    EagerRun<VAR> f{p, nheads, s};                                                         \
+    return dispatch_shape(sh, f);                                                          \
+  }                                                                                        \
+  template <>                                                                              \
+  size_t step_smem_bytes<VAR>(const Shape& sh, int L) {                                    \
+    StepSmem<VAR> f{L, 0};                                                                 \
+    return dispatch_shape(sh, f) == cudaSuccess ? f.out : 0;                               \
+  }                                                                                        \
+  template <>                                                                              \
+  size_t merge_smem_bytes<VAR>(const Shape& sh, int L) {                                   \
+    MergeSmem<VAR> f{L, 0};                                                                \
+    return dispatch_shape(sh, f) == cudaSuccess ? f.out : 0;                               \
+  }
+
+}  // namespace dl

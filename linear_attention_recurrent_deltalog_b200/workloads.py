@@ -222,3 +222,49 @@ def sample_heads(w: Workload, n: int, seed: int = 0) -> np.ndarray:
     n = min(n, w.heads)
     g = _rng(w.seed, 0, 3 + seed)
     return np.sort(g.choice(w.heads, size=n, replace=False)).astype(np.int64)
+
+
+# ----------------------------------------------------------------- prefetch
+
+def _step_job(args):
+    w, t = args
+    return step_inputs(w, t)
+
+
+class StepStream:
+    """Yields step_inputs(w, t) for t in [start, start + T) in order,
+    drawing ahead in a pool of worker processes started with ``spawn`` (safe
+    after CUDA is initialised in the parent).  ``workers=0`` draws inline."""
+
+    def __init__(self, w: Workload, T: Optional[int] = None, start: int = 0,
+                 workers: Optional[int] = None, ahead: int = 0):
+        import os
+        self.w = w
+        self.T = w.T if T is None else T
+        self.start = start
+        if workers is None:
+            workers = min(16, max(0, (os.cpu_count() or 1) - 1))
+        self.workers = workers if self.T > 4 else 0
+        self.ahead = ahead or 2 * max(1, self.workers)
+
+    def __iter__(self) -> Iterator[StepInputs]:
+        if self.workers <= 0:
+            yield from iter_steps(self.w, self.T, self.start)
+            return
+        import collections
+        import concurrent.futures as cf
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        with cf.ProcessPoolExecutor(max_workers=self.workers, mp_context=ctx) as ex:
+            pending = collections.deque()
+            nxt = self.start
+            end = self.start + self.T
+            while nxt < end and len(pending) < self.ahead:
+                pending.append(ex.submit(_step_job, (self.w, nxt)))
+                nxt += 1
+            while pending:
+                s = pending.popleft().result()
+                if nxt < end:
+                    pending.append(ex.submit(_step_job, (self.w, nxt)))
+                    nxt += 1
+                yield s

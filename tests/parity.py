@@ -1,0 +1,173 @@
+"""GPU-vs-oracle parity harness (test infrastructure).
+
+Runs the library's decode paths through the C ABI on the seeded inputs of a
+workload, and the fp64 oracle on the same inputs for a sample of heads (every
+head is an independent recurrence, so a sample checks the full launch
+exactly), then reports the relative errors north of which a test fails:
+
+  state : max |S_gpu - S_ref| / max |S_ref| over the checked heads, taken
+          at every snapshot step (every ``snap_every`` steps and at T);
+  output: max over steps t of max |o_gpu - o_ref| / max |o_ref| (over the
+          checked heads and value rows).
+
+Several "arms" run in one pass over the inputs so the draws are made once:
+  "log"    DeltaLog step + dl_merge(DL_MERGE_FULL) after every step
+  "fused"  DeltaLog step with the merge fused into the step kernel
+  "eager"  the dense eager step kernel
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import types
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+import torch
+
+import oracle
+from linear_attention_recurrent_deltalog_b200 import deltalog as dlb
+from linear_attention_recurrent_deltalog_b200 import workloads as wl
+
+STATE_TOL = 1e-4
+OUT_TOL = 1e-3
+
+
+def host_to_device(x: np.ndarray, dev) -> torch.Tensor:
+    """numpy array as the kernel reads it (uint16 -> bf16 bits, else fp32)."""
+    if x.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(dev).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev)
+
+
+def step_to_device(s: wl.StepInputs, dev):
+    q = host_to_device(s.device_array("q"), dev).reshape(-1)
+    k = host_to_device(s.device_array("k"), dev).reshape(-1)
+    v = host_to_device(s.device_array("v"), dev).reshape(-1)
+    dec = host_to_device(s.decay, dev).reshape(-1)
+    beta = None if s.beta is None else host_to_device(s.beta, dev).reshape(-1)
+    return q, k, v, dec, beta
+
+
+@dataclasses.dataclass
+class ArmResult:
+    state_err: float
+    out_err: float
+    outputs: List[np.ndarray]
+    states: Dict[int, np.ndarray]
+
+
+_S0_CACHE: Dict[tuple, np.ndarray] = {}
+
+
+def cached_initial_state(w: wl.Workload) -> np.ndarray:
+    """wl.initial_state(w), memoised: it does not depend on L, and the 1 GiB
+    draw of the serving batch takes several seconds."""
+    key = (w.seed, w.B, w.H, w.d_v, w.d_k, w.s0_std)
+    if key not in _S0_CACHE:
+        if len(_S0_CACHE) > 2:
+            _S0_CACHE.clear()
+        _S0_CACHE[key] = wl.initial_state(w)
+    return _S0_CACHE[key]
+
+
+def _rel(a: np.ndarray, ref: np.ndarray) -> float:
+    den = float(np.max(np.abs(ref)))
+    return float(np.max(np.abs(a - ref))) / (den if den > 0 else 1.0)
+
+
+def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence[int]] = None,
+               arms=("log", "fused", "eager"), snap_every: int = 64, L: Optional[int] = None,
+               merge_all_at: Sequence[int] = (), workers: Optional[int] = None,
+               device="cuda") -> Dict[str, ArmResult]:
+    """Runs the given arms and the oracle; returns per-arm errors."""
+    if L is not None:
+        w = w.replace(L=L)
+    T = w.T if T is None else T
+    BH, dk, dv = w.heads, w.d_k, w.d_v
+    heads = np.arange(BH) if heads is None else np.asarray(heads, dtype=np.int64)
+    heads_t = torch.from_numpy(heads).to(device)
+    S0 = cached_initial_state(w)
+    fill0 = wl.fill_offsets(w)
+    bonus = wl.rwkv6_bonus(w) if w.variant == wl.RWKV6 else None
+    bonus_d = None if bonus is None else torch.from_numpy(bonus).to(device).reshape(-1)
+    S0_d = torch.from_numpy(S0).to(device).reshape(-1)
+    snaps = sorted(set([t for t in range(snap_every, T + 1, snap_every)] + [T]))
+
+    states = {}
+    dense = {}
+    for arm in arms:
+        if arm == "eager":
+            dense[arm] = S0_d.clone()
+        else:
+            cfg = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype, fused_merge=(arm == "fused"))
+            st = dlb.DeltaLogState(cfg, device=device)
+            st.reset(S0_d, fill0.tolist())
+            states[arm] = st
+    cfg_e = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype)
+    out = {arm: [] for arm in arms}
+    snap_gpu = {arm: {} for arm in arms}
+    recs = []
+    o = torch.empty(BH * dv, dtype=torch.float32, device=device)
+    S_out = torch.empty(BH * dv * dk, dtype=torch.float32, device=device)
+    for s in wl.StepStream(w, T, workers=workers):
+        q, k, v, dec, beta = step_to_device(s, device)
+        n = s.t + 1
+        for arm in arms:
+            if arm == "eager":
+                dlb.dl_eager_step(cfg_e, dense[arm], q, k, v, dec, beta, bonus_d, o)
+            else:
+                st = states[arm]
+                st.step(q, k, v, dec, beta, bonus_d, o)
+                if arm == "log":
+                    st.merge(dlb.DL_MERGE_FULL)
+                if n in merge_all_at:
+                    st.merge(dlb.DL_MERGE_ALL)
+            out[arm].append(o.view(BH, dv).index_select(0, heads_t).cpu().numpy().astype(np.float64))
+            if n in snaps:
+                if arm == "eager":
+                    S = dense[arm]
+                else:
+                    states[arm].materialize(S_out)
+                    S = S_out
+                snap_gpu[arm][n] = (S.view(BH, dv, dk).index_select(0, heads_t).cpu().numpy()
+                                    .astype(np.float64))
+        flat = lambda x: None if x is None else x.reshape((BH,) + x.shape[2:])[heads][:, None]
+        recs.append(types.SimpleNamespace(q=flat(s.q), k=flat(s.k), v=flat(s.v),
+                                          decay=flat(s.decay), beta=flat(s.beta)))
+    torch.cuda.synchronize()
+    for arm, st in states.items():
+        code, head = st.device_error()
+        assert code == 0, f"device error {code} at head {head} ({arm})"
+        st.close()
+
+    S0h = S0.reshape(BH, dv, dk)[heads].astype(np.float64)
+    if w.variant == wl.RWKV6:
+        S0h = S0h.transpose(0, 2, 1)
+    bon = None if bonus is None else bonus[heads % w.H]
+    ref = oracle.run_eager(w.variant, S0h, recs, bonus=bon, snapshot_at=snaps)
+    result = {}
+    for arm in arms:
+        out_err = max(_rel(a, r) for a, r in zip(out[arm], ref.outputs))
+        st_err = 0.0
+        for n in snaps:
+            Sr = ref.states[n]
+            if w.variant == wl.RWKV6:
+                Sr = Sr.transpose(0, 2, 1)
+            st_err = max(st_err, _rel(snap_gpu[arm][n], Sr))
+        result[arm] = ArmResult(st_err, out_err, out[arm], snap_gpu[arm])
+    return result
+
+
+def heads_covering_phases(w: wl.Workload, n: int, L: Optional[int] = None) -> np.ndarray:
+    """A seeded head sample that contains every fill offset present."""
+    if L is not None:
+        w = w.replace(L=L)
+    fill = wl.fill_offsets(w)
+    picked = []
+    for f in sorted(set(fill.tolist())):
+        b = int(np.nonzero(fill == f)[0][0])
+        picked.append(b * w.H + (f % w.H))
+    rest = wl.sample_heads(w, n)
+    allh = np.unique(np.concatenate([np.array(picked, dtype=np.int64), rest]))
+    return allh

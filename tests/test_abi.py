@@ -1,0 +1,156 @@
+"""The C ABI library without a GPU (CPU only): it loads, exports every
+declared symbol, sizes buffers, and rejects bad arguments on the host before
+any CUDA call."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_recurrent_deltalog_b200 import deltalog as dlb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "deltalog.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dl_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(dlb.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"missing export {n}"
+    assert sorted(dlb.EXPORTED) == names
+
+
+def test_status_strings():
+    assert dlb.dl_status_string(0) == "ok"
+    assert "merge" in dlb.dl_status_string(dlb.DL_ERR_LOG_FULL)
+    assert dlb.dl_status_string(-99) == "unknown status"
+
+
+def cfg(**kw):
+    base = dict(variant="gdn", B=4, H=2, d_k=128, d_v=128, L=16, in_dtype="bf16")
+    base.update(kw)
+    return dlb.Config(**base)
+
+
+def test_state_bytes_layout():
+    c = cfg()
+    nb, nl, nm = dlb.dl_state_bytes(c)
+    BH = 8
+    assert nb == BH * 128 * 128 * 4
+    # u fp32 + k bf16 + scalar g, each array 256-B padded
+    pad = lambda x: (x + 255) // 256 * 256
+    assert nl == pad(BH * 16 * 128 * 4) + pad(BH * 16 * 128 * 2) + pad(BH * 16 * 4)
+    assert nm == pad(BH * 4) + 256
+    # KDA: vector log-decay; RWKV6: u stored in the input dtype
+    _, nl_kda, _ = dlb.dl_state_bytes(cfg(variant="kda"))
+    assert nl_kda == pad(BH * 16 * 128 * 4) + pad(BH * 16 * 128 * 2) + pad(BH * 16 * 128 * 4)
+    _, nl_rw, _ = dlb.dl_state_bytes(cfg(variant="rwkv6", d_k=64, d_v=64, L=32))
+    assert nl_rw == pad(BH * 32 * 64 * 2) + pad(BH * 32 * 64 * 2) + pad(BH * 32 * 64 * 4)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(variant="gdn", d_k=96), dlb.DL_ERR_UNSUPPORTED),
+    (dict(L=0), dlb.DL_ERR_ARG),
+    (dict(L=65), dlb.DL_ERR_ARG),
+    (dict(B=0), dlb.DL_ERR_ARG),
+    (dict(H=-1), dlb.DL_ERR_ARG),
+])
+def test_state_bytes_rejects(bad, code):
+    with pytest.raises(dlb.DeltaLogError) as e:
+        dlb.dl_state_bytes(cfg(**bad))
+    assert e.value.status == code
+
+
+def test_bad_enums_rejected():
+    c = cfg().c()
+    c.variant = 7
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+    c = cfg().c()
+    c.in_dtype = 3
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+    c = cfg().c()
+    c.flags = 4
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+
+
+def test_create_checks_pointers_without_touching_cuda():
+    c = cfg()
+    # fake device addresses: create only validates and stores them
+    with pytest.raises(dlb.DeltaLogError) as e:
+        dlb.dl_state_create(c, 0x1000, 0x2000, 0x3008)
+    assert e.value.status == dlb.DL_ERR_ALIGN
+    with pytest.raises(dlb.DeltaLogError) as e:
+        dlb.dl_state_create(c, 0x1000, None, 0x3000)
+    assert e.value.status == dlb.DL_ERR_ARG
+    h = dlb.dl_state_create(c, 0x100000, 0x200000, 0x300000)
+    try:
+        assert dlb.dl_state_fill(h, c) == [0] * c.B
+        # step argument checks happen before any launch
+        st = dlb._lib.dl_decode_step
+        assert st(h, None, 0x1000, 0x1000, 0x1000, 0x1000, None, 0x1000, None) == dlb.DL_ERR_ARG
+        assert st(h, 0x1008, 0x1000, 0x1000, 0x1000, 0x1000, None, 0x1000, None) == dlb.DL_ERR_ALIGN
+        # GDN needs beta
+        assert st(h, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x1000, None) == dlb.DL_ERR_ARG
+        assert dlb._lib.dl_merge(h, 5, None) == dlb.DL_ERR_ARG
+        # nothing to merge: no launch, OK even without a GPU
+        assert dlb._lib.dl_merge(h, dlb.DL_MERGE_FULL, None) == 0
+        assert dlb._lib.dl_merge(h, dlb.DL_MERGE_ALL, None) == 0
+        assert dlb._lib.dl_materialize(h, None, None) == dlb.DL_ERR_ARG
+        assert dlb._lib.dl_materialize(h, 0x1004, None) == dlb.DL_ERR_ALIGN
+        assert dlb._lib.dl_materialize(h, 0x100000, None) == dlb.DL_ERR_ARG  # aliases the base
+        # reset rejects fill offsets outside [0, L)
+        bad = (ctypes.c_int32 * c.B)(0, 16, 0, 0)
+        assert dlb._lib.dl_state_reset(h, None, bad, None) == dlb.DL_ERR_ARG
+    finally:
+        dlb.dl_state_destroy(h)
+    dlb.dl_state_destroy(None)
+
+
+def test_rwkv6_needs_bonus():
+    c = cfg(variant="rwkv6", d_k=64, d_v=64, L=32)
+    h = dlb.dl_state_create(c, 0x100000, 0x200000, 0x300000)
+    try:
+        st = dlb._lib.dl_decode_step
+        assert st(h, 0x1000, 0x1000, 0x1000, 0x1000, None, None, 0x1000, None) == dlb.DL_ERR_ARG
+    finally:
+        dlb.dl_state_destroy(h)
+    ec = cfg(variant="rwkv6", d_k=64, d_v=64).c()
+    assert dlb._lib.dl_eager_step(ctypes.byref(ec), 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None,
+                                  None, 0x1000, None) == dlb.DL_ERR_ARG
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="host without a GPU only")
+def test_launch_failure_leaves_host_mirror_unchanged():
+    # Without a device the launch fails with DL_ERR_CUDA; the fill mirror
+    # must not advance.
+    c = cfg()
+    h = dlb.dl_state_create(c, 0x100000, 0x200000, 0x300000)
+    try:
+        rc = dlb._lib.dl_decode_step(h, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, None, 0x1000, None)
+        assert rc == dlb.DL_ERR_CUDA
+        assert dlb.dl_state_fill(h, c) == [0] * c.B
+    finally:
+        dlb.dl_state_destroy(h)
+
+
+def test_binding_rejects_undersized_tensors():
+    import torch
+    c = cfg(B=2, H=2)
+    small = torch.zeros(3, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dlb._check_step_tensors(c, small, small, small, torch.zeros(4), torch.zeros(4), None,
+                                torch.zeros(512))
+    with pytest.raises(TypeError):
+        dlb._check_step_tensors(c, torch.zeros(512), torch.zeros(512), torch.zeros(512),
+                                torch.zeros(4), torch.zeros(4), None, torch.zeros(512))
