@@ -236,8 +236,9 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     fused = args.merge == "fused"
-    w = wl.WORKLOADS["gdn_serving"].replace(L=args.L)
-    cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=fused)
+    w = wl.WORKLOADS["gdn_serving"].replace(L=args.L, B=args.B)
+    cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=fused,
+                     step_split=args.split)
     stream = torch.cuda.current_stream(device)
 
     # inputs: a device ring of RING pre-drawn steps (the generator's recipe)
@@ -315,6 +316,14 @@ def run_ours(args, world, rank, local):
         except Exception:
             traffic = None
 
+    if args.only_step:
+        st.close()
+        return {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "only_step": True,
+                "config": {"B": w.B, "L": args.L, "merge": args.merge, "split": args.split},
+                "roofline": {"achieved": round(achieved, 1), "peak": peak,
+                             "frac": round(achieved / peak, 4), "launch_ms": round(step_avg * 1e3, 5)}}
+
     # eager dense step on a separate 1 GiB state, same inputs
     S_e = S0.clone()
     for i in range(args.warmup):
@@ -389,6 +398,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": f"GDN decode B=512 H=32 d_k=d_v=128 fp32 state, bf16 q/k/v, "
                                f"ragged fills, L={args.L}, merge={args.merge}",
                    "B": w.B, "H": w.H, "d": w.d_k, "L": args.L, "merge": args.merge,
+                   "step_split": args.split,
                    "global_batch": w.B * world, "parallelism": f"replicas x{world} (dp, no collective)",
                    "l2": "state 1 GiB > 126 MB L2 on every step: no flush needed",
                    "input_ring_steps": RING},
@@ -475,6 +485,11 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--L", type=int, default=16)
+    ap.add_argument("--B", type=int, default=512, help="sequences (profiling runs use fewer)")
+    ap.add_argument("--split", type=int, default=0,
+                    help="CTAs per head in the step kernel (0 = library default)")
+    ap.add_argument("--only-step", action="store_true",
+                    help="time the DeltaLog step only (profiling); not a bench line")
     ap.add_argument("--merge", choices=("fused", "separate"), default="fused")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -493,7 +508,7 @@ def main():
                 print(json.dumps(line), flush=True)
             return
         line = run_ours(args, world, rank, local)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.only_step:
             v, steps, el, threads = oracle_tokens_per_s(args.cpu_seconds)
             line["cpu_baseline"] = {"value": round(v, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
                                     "sample": f"first 2 of 512 sequences (64 heads), {steps} steps, "

@@ -78,16 +78,20 @@ enum dl_flags {
 };
 
 /* Layer configuration.  d_k, d_v in {64, 128}; 1 <= L <= 64; B, H >= 1 and
- * B*H*d_v*d_k < 2^40.  `flags` is a bitwise OR of dl_flags. */
+ * B*H*d_v*d_k < 2^40.  `flags` is a bitwise OR of dl_flags.  `step_split`
+ * is how many CTAs share one head's rows in the step kernel: 0 picks the
+ * library's default, otherwise 1, 2 or 4 with d_v / step_split >= 32 (a
+ * performance knob only: results do not depend on it). */
 typedef struct dl_config {
-  int32_t variant;  /* enum dl_variant */
-  int32_t B;        /* sequences in the batch */
-  int32_t H;        /* heads per sequence */
-  int32_t d_k;      /* key (and q / r) size per head */
-  int32_t d_v;      /* value size per head */
-  int32_t L;        /* log capacity: entries per head before a merge */
-  int32_t in_dtype; /* enum dl_dtype of q/r, k, v */
-  int32_t flags;    /* enum dl_flags */
+  int32_t variant;    /* enum dl_variant */
+  int32_t B;          /* sequences in the batch */
+  int32_t H;          /* heads per sequence */
+  int32_t d_k;        /* key (and q / r) size per head */
+  int32_t d_v;        /* value size per head */
+  int32_t L;          /* log capacity: entries per head before a merge */
+  int32_t in_dtype;   /* enum dl_dtype of q/r, k, v */
+  int32_t flags;      /* enum dl_flags */
+  int32_t step_split; /* 0 (default), 1, 2 or 4 */
 } dl_config;
 
 typedef struct dl_state dl_state;
@@ -97,7 +101,8 @@ typedef struct dl_state dl_state;
  *   log : per head L entries of u (fp32 [d_v]; in_dtype for RWKV6),
  *         k (in_dtype [d_k]) and log-decay g (fp32, [1] for GDN, [d_k]
  *         otherwise), laid out as three arrays [B,H,L,.], each 256-B aligned
- *   meta: int32 fill [B, H] plus a device error word, 256-B padded.
+ *   meta: two int32 fill arrays [B, H] (read and written alternately by
+ *         successive steps) and a device error word, each 256-B padded.
  * Any output pointer may be NULL.  Errors: DL_ERR_ARG, DL_ERR_UNSUPPORTED. */
 int dl_state_bytes(const dl_config* cfg, size_t* base_bytes, size_t* log_bytes,
                    size_t* meta_bytes);

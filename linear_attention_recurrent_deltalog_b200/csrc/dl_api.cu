@@ -34,6 +34,10 @@ struct Layout {
   size_t base, u_off, u_bytes, k_off, k_bytes, g_off, g_bytes, log, fill_bytes, err_off, meta;
 };
 
+// Default CTAs per head for the step kernel.
+int default_split(const dl_config& c) { return c.d_v >= 128 ? 2 : 1; }
+int split_of(const dl_config& c) { return c.step_split == 0 ? default_split(c) : c.step_split; }
+
 int u_elem_size(const dl_config& c) {
   return (c.variant == DL_RWKV6) ? (c.in_dtype == DL_BF16 ? 2 : 4) : 4;
 }
@@ -41,7 +45,6 @@ int in_elem_size(const dl_config& c) { return c.in_dtype == DL_BF16 ? 2 : 4; }
 
 Layout layout_of(const dl_config& c) {
   const size_t bh = size_t(c.B) * size_t(c.H);
-  const size_t gw = (c.variant == DL_GDN) ? 1 : size_t(c.d_k);
   Layout l{};
   l.base = pad(bh * c.d_v * c.d_k * 4);
   l.u_off = 0;
@@ -49,10 +52,10 @@ Layout layout_of(const dl_config& c) {
   l.k_off = l.u_off + l.u_bytes;
   l.k_bytes = pad(bh * c.L * c.d_k * in_elem_size(c));
   l.g_off = l.k_off + l.k_bytes;
-  l.g_bytes = pad(bh * c.L * gw * 4);
+  l.g_bytes = pad(bh * size_t(dl::g_stride(c.variant, c.L, c.d_k)) * 4);
   l.log = l.g_off + l.g_bytes;
   l.fill_bytes = pad(bh * 4);
-  l.err_off = l.fill_bytes;
+  l.err_off = 2 * l.fill_bytes;
   l.meta = l.err_off + kAlign;
   return l;
 }
@@ -71,10 +74,13 @@ int check_config(const dl_config* c, bool need_L) {
   if (bh > 0x7fffffffull) return DL_ERR_ARG;  // one CTA per head in a 1-D grid
   if (bh * uint64_t(c->d_v) * uint64_t(c->d_k) >= (1ull << 40)) return DL_ERR_ARG;
   if (!head_size_ok(c->d_k) || !head_size_ok(c->d_v)) return DL_ERR_UNSUPPORTED;
+  if (c->step_split != 0 && !dl::split_ok(c->d_v, c->step_split)) return DL_ERR_ARG;
   return DL_OK;
 }
 
-Shape shape_of(const dl_config& c) { return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0}; }
+Shape shape_of(const dl_config& c) {
+  return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0, split_of(c)};
+}
 
 cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, cudaStream_t s) {
   const unsigned n = unsigned(size_t(c.B) * c.H);
@@ -141,8 +147,12 @@ struct dl_state {
   std::vector<int32_t> fill_stage;  // [B*H] staging for reset uploads
   int n_full;                       // sequences whose log holds L entries
   int n_nonempty;                   // sequences whose log holds >= 1 entry
+  int parity;                       // which fill array holds the current counts
 
-  int* dev_fill() const { return reinterpret_cast<int*>(meta); }
+  int* dev_fill(int which) const {
+    return reinterpret_cast<int*>(meta + size_t(which) * lay.fill_bytes);
+  }
+  int* dev_fill() const { return dev_fill(parity); }
   int* dev_err() const { return reinterpret_cast<int*>(meta + lay.err_off); }
   void* logU() const { return log + lay.u_off; }
   void* logK() const { return log + lay.k_off; }
@@ -204,6 +214,7 @@ int dl_state_create(const dl_config* cfg, void* base, void* log, void* meta, dl_
   st->log = static_cast<unsigned char*>(log);
   st->meta = static_cast<unsigned char*>(meta);
   st->fill.assign(size_t(cfg->B), 0);
+  st->parity = 0;
   st->fill_stage.assign(size_t(cfg->B) * cfg->H, 0);
   st->recount();
   *out = st;
@@ -229,11 +240,12 @@ int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* st
     for (int h = 0; h < c.H; ++h)
       st->fill_stage[size_t(b) * c.H + h] = fill0 ? fill0[b] : 0;
   if (e == cudaSuccess)
-    e = cudaMemcpyAsync(st->dev_fill(), st->fill_stage.data(), st->fill_stage.size() * 4,
+    e = cudaMemcpyAsync(st->dev_fill(0), st->fill_stage.data(), st->fill_stage.size() * 4,
                         cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return DL_ERR_CUDA;
   for (int b = 0; b < c.B; ++b) st->fill[b] = fill0 ? fill0[b] : 0;
+  st->parity = 0;
   st->recount();
   return DL_OK;
 }
@@ -251,7 +263,8 @@ int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v, co
   p.logU = st->logU();
   p.logK = st->logK();
   p.logG = st->logG();
-  p.fill = st->dev_fill();
+  p.fill_in = st->dev_fill(st->parity);
+  p.fill_out = st->dev_fill(st->parity ^ 1);
   p.err = st->dev_err();
   p.q = q;
   p.k = k;
@@ -264,6 +277,7 @@ int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v, co
   p.L = c.L;
   if (launch_step(c, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
+  st->parity ^= 1;
   for (int32_t& f : st->fill) {
     f += 1;
     if (fused && f == c.L) f = 0;

@@ -168,21 +168,22 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// Tile geometry for a d_v x d_k fp32 tile handled by DV/16 warps of 16 rows.
-template <int DK, int DV>
+// Tile geometry: ROWS rows (value indices) of a d_v x d_k fp32 tile, d_k
+// columns, handled by ROWS/16 warps of 16 rows each.
+template <int DK, int ROWS>
 struct Tile {
   static_assert(DK == 64 || DK == 128, "d_k in {64,128}");
-  static_assert(DV == 64 || DV == 128, "d_v in {64,128}");
-  static constexpr int kWarps = DV / 16;           // 16 rows per warp
+  static_assert(ROWS == 32 || ROWS == 64 || ROWS == 128, "rows per CTA in {32,64,128}");
+  static constexpr int kWarps = ROWS / 16;         // 16 rows per warp
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kRowsPerWarp = 16;
   static constexpr int kLPR = DK / 4;              // lanes per row (float4 each)
   static constexpr int kRPI = 32 / kLPR;           // rows per warp instruction
   static constexpr int kNV = kRowsPerWarp / kRPI;  // partials per lane
   static constexpr int kChunkRows = 32;            // rows per bulk copy
-  static constexpr int kChunks = DV / kChunkRows;
+  static constexpr int kChunks = ROWS / kChunkRows;
   static constexpr uint32_t kChunkBytes = kChunkRows * DK * 4;
-  static constexpr size_t kTileBytes = size_t(DV) * DK * 4;
+  static constexpr size_t kTileBytes = size_t(ROWS) * DK * 4;
   static constexpr int kCPL = DK / 32;              // key columns per lane in 32-lane dots
   static_assert(kLPR == 2 * kNV, "row reduction layout");
 };

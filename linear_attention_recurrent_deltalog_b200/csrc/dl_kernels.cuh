@@ -33,7 +33,8 @@ struct StepParams {
   void* logU;    // [BH, L, DV]  fp32 (in_dtype for RWKV6)
   void* logK;    // [BH, L, DK]  in_dtype
   float* logG;   // [BH, L, GW]
-  int* fill;     // [BH]
+  const int* fill_in;  // [BH] entries before this step
+  int* fill_out;       // [BH] entries after it (the other buffer of a pair)
   int* err;      // device error word (2 ints)
   const void* q;
   const void* k;
@@ -78,90 +79,111 @@ struct LogU<kVarRWKV6, TIn> { using type = TIn; };  // RWKV6 logs v itself
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// ------------------------------------------------------------------ step
+// Per-head stride of the log-decay array: GDN keeps one scalar per entry,
+// padded to a multiple of 4 entries so a head's block starts 16-B aligned and
+// can be fetched by a bulk copy; KDA and RWKV6 keep d_k values per entry.
+__host__ __device__ constexpr int g_stride(int variant, int L, int dk) {
+  return variant == kVarGDN ? ((L + 3) / 4) * 4 : L * dk;
+}
 
-template <int VAR, int DK, int DV, typename TIn>
+// Bytes of the first f log-decay entries a bulk copy fetches (whole
+// 16-B groups for GDN's scalars).
+template <int VAR, int DK>
+__device__ __forceinline__ uint32_t g_copy_bytes(int f) {
+  return VAR == kVarGDN ? uint32_t((f + 3) / 4) * 16u : uint32_t(f) * DK * 4u;
+}
+
+// ------------------------------------------------------------------ step
+//
+// A head's rows may be split over SPLIT = DV / ROWS CTAs (blockIdx.x =
+// head * SPLIT + part).  Rows are independent in the GEMV, the correction
+// and the readout; every part recomputes the per-head scalars (cheap) and
+// stages all f log keys but only its own rows of the log's u vectors.  The
+// smaller shared-memory footprint lets more CTAs -- and more bytes in
+// flight -- sit on each SM.  Part 0 appends k_t and g_t and advances the
+// fill; fills are double-buffered by step parity (read fill_in, write
+// fill_out), so no CTA ever reads a counter another CTA of the same launch
+// writes.
+//
+// Order inside a CTA: the tile's bulk copies go out first (they do not
+// depend on anything), then the fill is read and the log's copies go out;
+// the per-head vectors are loaded meanwhile.  After one barrier, the
+// log-decay bookkeeping and the per-entry weights are computed together, a
+// second barrier publishes them, and each warp streams its rows.
+
+template <int VAR, int DK, int DV, int ROWS, typename TIn>
 struct StepLayout {
   using TU = typename LogU<VAR, TIn>::type;
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
   size_t offU, offK, offG, offVec, offW, offZ, offScal, offBar, total;
   __host__ __device__ explicit StepLayout(int L) {
-    offU = Tile<DK, DV>::kTileBytes;
-    offK = offU + align_up(size_t(L) * DV * sizeof(TU), 128);
+    offU = Tile<DK, ROWS>::kTileBytes;
+    offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
     offG = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
-    offVec = offG + align_up(size_t(L) * GW * 4, 128);
-    // k, q (raw), k-hat, q-hat [DK] each; v [DV]; g_t, g_{t-1} [GW] each
-    offW = offVec + align_up(size_t(4 * DK + DV + 2 * GW) * 4, 128);
+    offVec = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
+    // k, q (raw), k-hat, q-hat, decay [DK] each; v [ROWS]; g_t, g_{t-1} [GW]
+    offW = offVec + align_up(size_t(5 * DK + ROWS + 2 * GW) * 4, 128);
     offZ = offW + align_up(size_t(L) * 4, 16);
     offScal = offZ + align_up(size_t(L) * 4, 16);
     offBar = offScal + 64;
-    total = offBar + 8 * (Tile<DK, DV>::kChunks + 1);
+    total = offBar + 8 * (Tile<DK, ROWS>::kChunks + 1);
   }
 };
 
-template <int VAR, int DK, int DV, typename TIn, bool FUSED>
-__global__ void __launch_bounds__(Tile<DK, DV>::kThreads)
+template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
+__global__ void __launch_bounds__(Tile<DK, ROWS>::kThreads)
 dl_step_kernel(const StepParams p) {
-  using Tl = Tile<DK, DV>;
+  using Tl = Tile<DK, ROWS>;
   using TU = typename LogU<VAR, TIn>::type;
-  constexpr int GW = StepLayout<VAR, DK, DV, TIn>::GW;
+  constexpr int SPLIT = DV / ROWS;
+  constexpr int GW = StepLayout<VAR, DK, DV, ROWS, TIn>::GW;
   constexpr int NT = Tl::kThreads;
   constexpr int NW = Tl::kWarps;
   constexpr int NV = Tl::kNV;
   constexpr int LPR = Tl::kLPR;
   constexpr int RPI = Tl::kRPI;
   constexpr int CPL = Tl::kCPL;
+  static_assert(DV % ROWS == 0, "rows split evenly");
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int L = p.L;
-  const StepLayout<VAR, DK, DV, TIn> lay(L);
-  float* sS = reinterpret_cast<float*>(smem);
-  TU* sU = reinterpret_cast<TU*>(smem + lay.offU);
-  TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);
-  float* sG = reinterpret_cast<float*>(smem + lay.offG);
-  float* sk = reinterpret_cast<float*>(smem + lay.offVec);  // raw k_t
-  float* sq = sk + DK;                                       // raw q_t / r_t
-  float* sKh = sq + DK;                                      // GEMV vector for a
-  float* sQh = sKh + DK;                                     // GEMV vector for b
-  float* sV = sQh + DK;                                      // v_t
-  float* sGt = sV + DV;                                      // g_t
-  float* sGp = sGt + GW;                                     // g_{t-1}
-  float* sW = reinterpret_cast<float*>(smem + lay.offW);     // per-entry weights on k
-  float* sZ = reinterpret_cast<float*>(smem + lay.offZ);     // per-entry weights on q / r
+  const int GS = g_stride(VAR, L, DK);
+  const StepLayout<VAR, DK, DV, ROWS, TIn> lay(L);
+  float* sS = reinterpret_cast<float*>(smem);                 // [ROWS][DK]
+  TU* sU = reinterpret_cast<TU*>(smem + lay.offU);            // [L][ROWS]
+  TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);          // [L][DK]
+  float* sG = reinterpret_cast<float*>(smem + lay.offG);      // [L][GW]
+  float* sk = reinterpret_cast<float*>(smem + lay.offVec);    // raw k_t
+  float* sq = sk + DK;                                        // raw q_t / r_t
+  float* sKh = sq + DK;                                       // GEMV vector for a
+  float* sQh = sKh + DK;                                      // GEMV vector for b
+  float* sDec = sQh + DK;                                     // decay_t
+  float* sV = sDec + DK;                                      // v_t (this part's rows)
+  float* sGt = sV + ROWS;                                     // g_t
+  float* sGp = sGt + GW;                                      // g_{t-1}
+  float* sW = reinterpret_cast<float*>(smem + lay.offW);      // per-entry weights on k
+  float* sZ = reinterpret_cast<float*>(smem + lay.offZ);      // per-entry weights on q / r
   float* sScal = reinterpret_cast<float*>(smem + lay.offScal);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
+  uint64_t* barLog = &bars[Tl::kChunks];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const size_t head = blockIdx.x;
+  const size_t head = blockIdx.x / SPLIT;
+  const int part = static_cast<int>(blockIdx.x % SPLIT);
+  const int r0 = part * ROWS;  // first value row of this CTA
   const int h = static_cast<int>(head % static_cast<size_t>(p.H));
-  const int f = p.fill[head];
-  if (f < 0 || f >= L) {  // the host never launches a step on a full log
-    if (tid == 0 && p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
-    return;
-  }
-  const bool merge_now = FUSED && (f + 1 == L);
 
-  const float* gS = p.base + head * size_t(DV) * DK;
+  const float* gS = p.base + (head * size_t(DV) + r0) * DK;
   TU* gU = static_cast<TU*>(p.logU) + head * size_t(L) * DV;
   TIn* gK = static_cast<TIn*>(p.logK) + head * size_t(L) * DK;
-  float* gG = p.logG + head * size_t(L) * GW;
-  uint64_t* barLog = &bars[Tl::kChunks];
+  float* gG = p.logG + head * size_t(GS);
 
   if (tid == 0) {
 #pragma unroll
     for (int c = 0; c <= Tl::kChunks; ++c) mbar_init(&bars[c], 1);
     fence_mbar_init();
-    if (f > 0) {
-      const uint32_t bu = uint32_t(f) * DV * sizeof(TU);
-      const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
-      const uint32_t bg = (GW > 1) ? uint32_t(f) * GW * 4 : 0u;
-      mbar_arrive_expect_tx(barLog, bu + bk + bg);
-      tma_load_1d(sU, gU, bu, barLog);
-      tma_load_1d(sK, gK, bk, barLog);
-      if (GW > 1) tma_load_1d(sG, gG, bg, barLog);
-    }
 #pragma unroll
     for (int c = 0; c < Tl::kChunks; ++c) {
       mbar_arrive_expect_tx(&bars[c], Tl::kChunkBytes);
@@ -169,94 +191,116 @@ dl_step_kernel(const StepParams p) {
                          Tl::kChunkBytes, &bars[c]);
     }
   }
+  const int f = p.fill_in[head];
+  if (f < 0 || f >= L) {  // the host never launches a step on a full log
+    if (tid == 0) {
+      if (p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
+      for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
+    }
+    return;
+  }
+  const bool merge_now = FUSED && (f + 1 == L);
+  const bool appender = (part == 0) && !merge_now;
+  if (tid == 0 && f > 0) {
+    const uint32_t bu = uint32_t(ROWS) * sizeof(TU);
+    const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
+    const uint32_t bg = g_copy_bytes<VAR, DK>(f);
+    mbar_arrive_expect_tx(barLog, bu * uint32_t(f) + bk + bg);
+    tma_load_1d(sK, gK, bk, barLog);
+    tma_load_1d(sG, gG, bg, barLog);
+    for (int i = 0; i < f; ++i)
+      tma_load_1d(sU + size_t(i) * ROWS, gU + size_t(i) * DV + r0, bu, barLog);
+  }
 
-  // ---- per-head vectors while the tile streams in
+  // ---- per-head vectors while the tile and the log stream in
   const TIn* gq = static_cast<const TIn*>(p.q) + head * DK;
   const TIn* gk = static_cast<const TIn*>(p.k) + head * DK;
-  const TIn* gv = static_cast<const TIn*>(p.v) + head * DV;
+  const TIn* gv = static_cast<const TIn*>(p.v) + head * DV + r0;
   for (int c = tid; c < DK; c += NT) {
-    const float kc = to_f(gk[c]);
-    const float qc = to_f(gq[c]);
-    sk[c] = kc;
-    sq[c] = qc;
-    if (VAR == kVarGDN) {
-      sKh[c] = kc;
-      sQh[c] = qc;
-    } else {
-      const float gp = (f > 0) ? gG[size_t(f - 1) * GW + c] : 0.f;
-      const float gt = gp + logf(p.decay[head * DK + c]);
+    const TIn kraw = gk[c];
+    sk[c] = to_f(kraw);
+    sq[c] = to_f(gq[c]);
+    sDec[c] = (GW > 1) ? p.decay[head * DK + c] : 0.f;
+    if (merge_now)
+      sK[size_t(f) * DK + c] = kraw;
+    else if (appender)
+      gK[size_t(f) * DK + c] = kraw;
+  }
+  for (int j = tid; j < ROWS; j += NT) sV[j] = to_f(gv[j]);
+  if (tid == 0) {
+    if (GW == 1) sDec[0] = p.decay[head];
+    sScal[1] = (VAR == kVarRWKV6) ? 0.f : p.beta[head];
+    if (part == 0) p.fill_out[head] = merge_now ? 0 : f + 1;
+  }
+  __syncthreads();
+
+  // ---- log-decay bookkeeping and per-entry weights (needs the log)
+  bool ok = true;
+  if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
+  if (GW == 1) {
+    if (tid == 0) {
+      const float gp = (f > 0) ? sG[f - 1] : 0.f;
+      const float gt = gp + logf(sDec[0]);
+      sGp[0] = gp;
+      sGt[0] = gt;
+      sScal[2] = expf(gt);
+      if (appender) gG[f] = gt;
+    }
+  } else {
+    for (int c = tid; c < DK; c += NT) {
+      const float gp = (f > 0) ? sG[size_t(f - 1) * DK + c] : 0.f;
+      const float gt = gp + logf(sDec[c]);
       sGp[c] = gp;
       sGt[c] = gt;
       if (VAR == kVarKDA) {
         const float e = expf(gt);
-        sKh[c] = e * kc;
-        sQh[c] = e * qc;
+        sKh[c] = e * sk[c];
+        sQh[c] = e * sq[c];
       } else {  // RWKV6 reads S_{t-1}: decay up to the previous step
-        sKh[c] = kc;
-        sQh[c] = expf(gp) * qc;
+        sQh[c] = expf(gp) * sq[c];
       }
-    }
-    if (merge_now) {
-      sK[size_t(f) * DK + c] = gk[c];
-    } else {
-      gK[size_t(f) * DK + c] = gk[c];
-      if (GW > 1) gG[size_t(f) * GW + c] = sGt[c];
+      if (appender) gG[size_t(f) * DK + c] = gt;
     }
   }
-  for (int j = tid; j < DV; j += NT) sV[j] = to_f(gv[j]);
-  if (VAR == kVarGDN) {
-    for (int i = tid; i < f; i += NT) sG[i] = gG[i];
-    if (tid == 0) {
-      const float gp = (f > 0) ? gG[f - 1] : 0.f;
-      const float gt = gp + logf(p.decay[head]);
-      sGp[0] = gp;
-      sGt[0] = gt;
-      sScal[2] = expf(gt);
-      if (!merge_now) gG[f] = gt;
-    }
-  }
-  if (tid == 0) sScal[1] = (VAR == kVarRWKV6) ? 0.f : p.beta[head];
-  __syncthreads();
-  // Every thread has read fill[head] before the barrier above, and no other
-  // CTA reads it, so advancing it here is race-free.
-  if (tid == 0) p.fill[head] = merge_now ? 0 : f + 1;
-
-  // ---- log prologue: one weight per entry and query vector
-  bool ok = true;
-  if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
-  if (!__syncthreads_and(ok)) {
-    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
-    for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
-    return;
-  }
-  for (int i = warp; i < f; i += NW) {
-    float x = 0.f, y = 0.f;
-#pragma unroll
-    for (int cc = 0; cc < CPL; ++cc) {
-      const int c = lane * CPL + cc;
-      const float ki = to_f(sK[size_t(i) * DK + c]);
-      if (VAR == kVarGDN) {
-        x = fmaf(ki, sk[c], x);
-        y = fmaf(ki, sq[c], y);
-      } else if (VAR == kVarKDA) {
-        const float e = expf(sGt[c] - sG[size_t(i) * DK + c]);
-        x = fmaf(ki * e, sk[c], x);
-        y = fmaf(ki * e, sq[c], y);
-      } else {
-        const float e = expf(sGp[c] - sG[size_t(i) * DK + c]);
-        y = fmaf(ki * e, sq[c], y);
-      }
-    }
-    if (VAR != kVarRWKV6) x = warp_sum(x);
-    y = warp_sum(y);
+  if (f > 0) {
+    // g_t (KDA) or g_{t-1} (RWKV6) for this lane's key columns, and g_t for GDN
+    float gl[CPL];
+    float gt0 = 0.f;
     if (VAR == kVarGDN) {
-      const float e = expf(sGt[0] - sG[i]);
-      x *= e;
-      y *= e;
+      gt0 = sG[f - 1] + logf(sDec[0]);
+    } else {
+#pragma unroll
+      for (int cc = 0; cc < CPL; ++cc) {
+        const int c = lane * CPL + cc;
+        gl[cc] = sG[size_t(f - 1) * DK + c] + (VAR == kVarKDA ? logf(sDec[c]) : 0.f);
+      }
     }
-    if (lane == 0) {
-      sW[i] = x;
-      sZ[i] = y;
+    for (int i = warp; i < f; i += NW) {
+      float x = 0.f, y = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < CPL; ++cc) {
+        const int c = lane * CPL + cc;
+        const float ki = to_f(sK[size_t(i) * DK + c]);
+        if (VAR == kVarGDN) {
+          x = fmaf(ki, sk[c], x);
+          y = fmaf(ki, sq[c], y);
+        } else {
+          const float kie = ki * expf(gl[cc] - sG[size_t(i) * DK + c]);
+          if (VAR == kVarKDA) x = fmaf(kie, sk[c], x);
+          y = fmaf(kie, sq[c], y);
+        }
+      }
+      if (VAR != kVarRWKV6) x = warp_sum(x);
+      y = warp_sum(y);
+      if (VAR == kVarGDN) {
+        const float e = expf(gt0 - sG[i]);
+        x *= e;
+        y *= e;
+      }
+      if (lane == 0) {
+        sW[i] = x;
+        sZ[i] = y;
+      }
     }
   }
   if (warp == NW - 1) {
@@ -272,10 +316,14 @@ dl_step_kernel(const StepParams p) {
     x = warp_sum(x);
     if (lane == 0) sScal[0] = x;
   }
-  __syncthreads();
+  if (!__syncthreads_and(ok)) {
+    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
+    return;
+  }
 
   // ---- one pass over this warp's 16 rows of S_b
-  const int j0 = warp * Tl::kRowsPerWarp;
+  const int j0 = warp * Tl::kRowsPerWarp;  // local row index
   uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
   if (!mbar_wait(barMine, 0, p.err, int(head))) {
     mbar_wait(barMine, 0, nullptr, 0);
@@ -283,8 +331,10 @@ dl_step_kernel(const StepParams p) {
   }
   const int c0 = (lane % LPR) * 4;
   const int rsub = lane / LPR;
-  const float4 kh4 = *reinterpret_cast<const float4*>(sKh + c0);
-  const float4 qh4 = *reinterpret_cast<const float4*>(sQh + c0);
+  const float* vA = (VAR == kVarGDN) ? sk : sKh;
+  const float* vB = (VAR == kVarGDN) ? sq : sQh;
+  const float4 kh4 = *reinterpret_cast<const float4*>(vA + c0);
+  const float4 qh4 = *reinterpret_cast<const float4*>(vB + c0);
   float pa[NV], pb[NV];
 #pragma unroll
   for (int pi = 0; pi < NV; ++pi) {
@@ -294,16 +344,16 @@ dl_step_kernel(const StepParams p) {
   }
   const float a = (VAR == kVarRWKV6) ? 0.f : reduce_rows<NV, LPR>(pa, lane);
   const float b = reduce_rows<NV, LPR>(pb, lane);
-  const int j = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;
+  const int jl = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;  // local row
 
-  // ---- log correction, delta-rule correction and readout for row j
+  // ---- log correction, delta-rule correction and readout for row r0 + jl
   float ck = 0.f, cq = 0.f;
   for (int i = 0; i < f; ++i) {
-    const float uij = to_f(sU[size_t(i) * DV + j]);
+    const float uij = to_f(sU[size_t(i) * ROWS + jl]);
     if (VAR != kVarRWKV6) ck = fmaf(sW[i], uij, ck);
     cq = fmaf(sZ[i], uij, cq);
   }
-  const float vj = sV[j];
+  const float vj = sV[jl];
   const float sdot = sScal[0];
   float u, o;
   if (VAR == kVarGDN) {
@@ -318,11 +368,11 @@ dl_step_kernel(const StepParams p) {
     o = b + cq + sdot * vj;
   }
   if ((lane & 1) == 0) {
-    p.o[head * DV + j] = o;
+    p.o[head * DV + r0 + jl] = o;
     if (merge_now)
-      sU[size_t(f) * DV + j] = Elem<TU>::from_f(u);
+      sU[size_t(f) * ROWS + jl] = Elem<TU>::from_f(u);
     else
-      gU[size_t(f) * DV + j] = Elem<TU>::from_f(u);
+      gU[size_t(f) * DV + r0 + jl] = Elem<TU>::from_f(u);
   }
   if (!merge_now) return;
 
@@ -356,14 +406,14 @@ dl_step_kernel(const StepParams p) {
     }
 #pragma unroll
     for (int pi = 0; pi < NV; ++pi) {
-      const float ui = to_f(sU[size_t(i) * DV + j0 + pi * RPI + rsub]);
+      const float ui = to_f(sU[size_t(i) * ROWS + j0 + pi * RPI + rsub]);
       acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
       acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
       acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
       acc[pi].w = fmaf(ui, k4.w, acc[pi].w);
     }
   }
-  float* gSw = p.base + head * size_t(DV) * DK;
+  float* gSw = p.base + (head * size_t(DV) + r0) * DK;
 #pragma unroll
   for (int pi = 0; pi < NV; ++pi)
     *reinterpret_cast<float4*>(gSw + size_t(j0 + pi * RPI + rsub) * DK + c0) = acc[pi];
@@ -381,7 +431,7 @@ struct MergeLayout {
     offK = offU + align_up(size_t(L) * DV * sizeof(TU), 128);
     offKt = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
     offG = offKt + align_up(size_t(L) * DK * 4, 128);
-    offDec = offG + align_up(size_t(L) * GW * 4, 128);
+    offDec = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
     offBar = offDec + align_up(size_t(DK) * 4, 128);
     total = offBar + 8 * (Tile<DK, DV>::kChunks + 1);
   }
@@ -400,6 +450,7 @@ dl_merge_kernel(const MergeParams p) {
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int L = p.L;
+  const int GS = g_stride(VAR, L, DK);
   const size_t head = blockIdx.x;
   const int f = p.fill[head];
   if (f < 0 || f > L) {
@@ -426,38 +477,31 @@ dl_merge_kernel(const MergeParams p) {
   const float* gS = p.base + head * size_t(DV) * DK;
   const TU* gU = static_cast<const TU*>(p.logU) + head * size_t(L) * DV;
   const TIn* gK = static_cast<const TIn*>(p.logK) + head * size_t(L) * DK;
-  const float* gG = p.logG + head * size_t(L) * GW;
+  const float* gG = p.logG + head * size_t(GS);
 
   if (tid == 0) {
 #pragma unroll
     for (int c = 0; c <= Tl::kChunks; ++c) mbar_init(&bars[c], 1);
     fence_mbar_init();
-    if (f > 0) {
-      const uint32_t bu = uint32_t(f) * DV * sizeof(TU);
-      const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
-      const uint32_t bg = (GW > 1) ? uint32_t(f) * GW * 4 : 0u;
-      mbar_arrive_expect_tx(barLog, bu + bk + bg);
-      tma_load_1d(sU, gU, bu, barLog);
-      tma_load_1d(sK, gK, bk, barLog);
-      if (GW > 1) tma_load_1d(sG, gG, bg, barLog);
-    }
 #pragma unroll
     for (int c = 0; c < Tl::kChunks; ++c) {
       mbar_arrive_expect_tx(&bars[c], Tl::kChunkBytes);
       tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
                          Tl::kChunkBytes, &bars[c]);
     }
+    if (f > 0) {
+      const uint32_t bu = uint32_t(f) * DV * sizeof(TU);
+      const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
+      const uint32_t bg = g_copy_bytes<VAR, DK>(f);
+      mbar_arrive_expect_tx(barLog, bu + bk + bg);
+      tma_load_1d(sU, gU, bu, barLog);
+      tma_load_1d(sK, gK, bk, barLog);
+      tma_load_1d(sG, gG, bg, barLog);
+    }
   }
-  if (GW == 1)
-    for (int i = tid; i < f; i += NT) sG[i] = gG[i];
   __syncthreads();
   bool ok = true;
   if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
-  if (!__syncthreads_and(ok)) {
-    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
-    for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
-    return;
-  }
   // decay of the base and decayed keys k-tilde_i = k_i o e^{g_last - g_i}
   for (int c = tid; c < DK; c += NT) {
     const float gl = (f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f;
@@ -466,7 +510,11 @@ dl_merge_kernel(const MergeParams p) {
       sKt[size_t(i) * DK + c] = to_f(sK[size_t(i) * DK + c]) * expf(gl - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
   }
   if (tid == 0 && p.mode != 2) p.fill[head] = 0;
-  __syncthreads();
+  if (!__syncthreads_and(ok)) {
+    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
+    return;
+  }
 
   const int j0 = warp * Tl::kRowsPerWarp;
   uint64_t* barMine = &bars[j0 / Tl::kChunkRows];

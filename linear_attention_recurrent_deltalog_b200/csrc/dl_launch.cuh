@@ -15,8 +15,13 @@ namespace dl {
 struct Shape {
   int dk;
   int dv;
-  int bf16;  // 1: q/k/v are bf16, 0: fp32
+  int bf16;   // 1: q/k/v are bf16, 0: fp32
+  int split;  // step kernel: CTAs per head (1, 2 or 4; d_v / split >= 32)
 };
+
+inline bool split_ok(int dv, int split) {
+  return (split == 1 || split == 2 || split == 4) && dv % split == 0 && dv / split >= 32;
+}
 
 // Dynamic shared memory each kernel may use; set once per device.
 constexpr int kMaxSmemOptIn = 227 * 1024;
@@ -39,14 +44,14 @@ inline cudaError_t prepare_kernel(Kern kern, std::atomic<unsigned long long>& do
   return cudaSuccess;
 }
 
-template <int VAR, int DK, int DV, typename TIn, bool FUSED>
+template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
 cudaError_t launch_step_t(const StepParams& p, unsigned nheads, cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
-  auto kern = dl_step_kernel<VAR, DK, DV, TIn, FUSED>;
+  auto kern = dl_step_kernel<VAR, DK, DV, ROWS, TIn, FUSED>;
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
-  const size_t smem = StepLayout<VAR, DK, DV, TIn>(p.L).total;
-  kern<<<nheads, Tile<DK, DV>::kThreads, smem, s>>>(p);
+  const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn>(p.L).total;
+  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -120,16 +125,29 @@ DL_DECLARE_VARIANT_LAUNCHERS(kVarRWKV6)
 
 // Functors the shape dispatch calls (namespace scope: local classes cannot
 // have member templates).
+template <int VAR, int DK, int DV, typename T, bool FUSED>
+cudaError_t launch_step_split(int split, const StepParams& p, unsigned n, cudaStream_t s) {
+  if (split == 1) return launch_step_t<VAR, DK, DV, DV, T, FUSED>(p, n, s);
+  if constexpr (DV / 2 >= 32) {
+    if (split == 2) return launch_step_t<VAR, DK, DV, DV / 2, T, FUSED>(p, n, s);
+  }
+  if constexpr (DV / 4 >= 32) {
+    if (split == 4) return launch_step_t<VAR, DK, DV, DV / 4, T, FUSED>(p, n, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int VAR>
 struct StepRun {
   const StepParams& p;
   unsigned n;
   cudaStream_t s;
   bool fused;
+  int split;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    return fused ? launch_step_t<VAR, DK, DV, T, true>(p, n, s)
-                 : launch_step_t<VAR, DK, DV, T, false>(p, n, s);
+    return fused ? launch_step_split<VAR, DK, DV, T, true>(split, p, n, s)
+                 : launch_step_split<VAR, DK, DV, T, false>(split, p, n, s);
   }
 };
 template <int VAR>
@@ -151,11 +169,19 @@ struct EagerRun {
 template <int VAR>
 struct StepSmem {
   int L;
+  int split;
   size_t out;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    out = StepLayout<VAR, DK, DV, T>(L).total;
-    return cudaSuccess;
+    out = 0;
+    if (split == 1) out = StepLayout<VAR, DK, DV, DV, T>(L).total;
+    if constexpr (DV / 2 >= 32) {
+      if (split == 2) out = StepLayout<VAR, DK, DV, DV / 2, T>(L).total;
+    }
+    if constexpr (DV / 4 >= 32) {
+      if (split == 4) out = StepLayout<VAR, DK, DV, DV / 4, T>(L).total;
+    }
+    return out ? cudaSuccess : cudaErrorInvalidValue;
   }
 };
 template <int VAR>
@@ -173,7 +199,7 @@ struct MergeSmem {
   template <>                                                                              \
   cudaError_t launch_step<VAR>(const Shape& sh, bool fused, const StepParams& p,           \
                                unsigned nheads, cudaStream_t s) {                          \
-    StepRun<VAR> f{p, nheads, s, fused};                                                   \
+    StepRun<VAR> f{p, nheads, s, fused, sh.split};                                                   \
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
   template <>                                                                              \
@@ -190,7 +216,7 @@ struct MergeSmem {
   }                                                                                        \
   template <>                                                                              \
   size_t step_smem_bytes<VAR>(const Shape& sh, int L) {                                    \
-    StepSmem<VAR> f{L, 0};                                                                 \
+    StepSmem<VAR> f{L, sh.split, 0};                                                                 \
     return dispatch_shape(sh, f) == cudaSuccess ? f.out : 0;                               \
   }                                                                                        \
   template <>                                                                              \

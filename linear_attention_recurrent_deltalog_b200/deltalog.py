@@ -51,7 +51,7 @@ _lib = _load()
 
 class dl_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("variant", "B", "H", "d_k", "d_v", "L", "in_dtype", "flags")]
+                ("variant", "B", "H", "d_k", "d_v", "L", "in_dtype", "flags", "step_split")]
 
 
 _P = ctypes.c_void_p
@@ -117,10 +117,12 @@ class Config:
     L: int
     in_dtype: str = "bf16"
     fused_merge: bool = False
+    step_split: int = 0
 
     def c(self) -> dl_config:
         return dl_config(VARIANT_IDS[self.variant], self.B, self.H, self.d_k, self.d_v, self.L,
-                         DTYPE_IDS[self.in_dtype], DL_FLAG_FUSED_MERGE if self.fused_merge else 0)
+                         DTYPE_IDS[self.in_dtype], DL_FLAG_FUSED_MERGE if self.fused_merge else 0,
+                         self.step_split)
 
     @property
     def heads(self) -> int:

@@ -51,7 +51,10 @@ def test_state_bytes_layout():
     # u fp32 + k bf16 + scalar g, each array 256-B padded
     pad = lambda x: (x + 255) // 256 * 256
     assert nl == pad(BH * 16 * 128 * 4) + pad(BH * 16 * 128 * 2) + pad(BH * 16 * 4)
-    assert nm == pad(BH * 4) + 256
+    # GDN's scalar log-decay stride is padded to a multiple of 4 entries
+    _, nl5, _ = dlb.dl_state_bytes(cfg(L=5))
+    assert nl5 == pad(BH * 5 * 128 * 4) + pad(BH * 5 * 128 * 2) + pad(BH * 8 * 4)
+    assert nm == 2 * pad(BH * 4) + 256  # two fill arrays (step parity) + error word
     # KDA: vector log-decay; RWKV6: u stored in the input dtype
     _, nl_kda, _ = dlb.dl_state_bytes(cfg(variant="kda"))
     assert nl_kda == pad(BH * 16 * 128 * 4) + pad(BH * 16 * 128 * 2) + pad(BH * 16 * 128 * 4)
@@ -65,6 +68,9 @@ def test_state_bytes_layout():
     (dict(L=65), dlb.DL_ERR_ARG),
     (dict(B=0), dlb.DL_ERR_ARG),
     (dict(H=-1), dlb.DL_ERR_ARG),
+    (dict(step_split=3), dlb.DL_ERR_ARG),
+    (dict(step_split=4, d_v=64), dlb.DL_ERR_ARG),
+    (dict(step_split=8), dlb.DL_ERR_ARG),
 ])
 def test_state_bytes_rejects(bad, code):
     with pytest.raises(dlb.DeltaLogError) as e:

@@ -67,8 +67,19 @@ def test_shapes_and_dtypes(variant, dk, dv, dtype):
     base = {"gdn": "gdn_qwen", "kda": "kda", "rwkv6": "rwkv6"}[variant]
     w = wl.WORKLOADS[base].replace(B=5, H=3, d_k=dk, d_v=dv, in_dtype=dtype, L=6, T=29,
                                    ragged=True)
-    res = run_parity(w, snap_every=7, workers=0)
-    _check(res)
+    for split in (1, dv // 32):
+        _check(run_parity(w, snap_every=7, workers=0, split=split))
+
+
+@pytest.mark.parametrize("split", [1, 2, 4])
+@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
+def test_step_split(name, split):
+    # a head's rows shared by 1, 2 or 4 CTAs: same results
+    w = wl.WORKLOADS[name]
+    if w.d_v // split < 32:
+        pytest.skip("d_v / split < 32 is not built")
+    w = w.replace(B=6, H=5, L=8, T=27, ragged=True)
+    _check(run_parity(w, snap_every=9, workers=0, split=split, arms=("log", "fused")))
 
 
 @pytest.mark.parametrize("L", [1, 2, 64])
@@ -76,8 +87,8 @@ def test_extreme_log_lengths(L):
     # L = 1 merges after every step; L = 64 is the largest log
     for name in ("gdn_qwen", "kda", "rwkv6"):
         w = wl.WORKLOADS[name].replace(B=3, H=4, L=L, T=max(3 * L, 12) + 1, ragged=True)
-        res = run_parity(w, snap_every=max(L, 4), workers=0)
-        _check(res)
+        for split in (1, w.d_v // 32):
+            _check(run_parity(w, snap_every=max(L, 4), workers=0, split=split))
 
 
 def test_forced_merges_mid_log():
