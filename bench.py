@@ -219,6 +219,11 @@ def eager_bytes(cfg) -> tuple:
 
 # ------------------------------------------------------------ our arm
 
+def workload_desc(w, merge: str) -> str:
+    return (f"{w.variant.upper()} decode B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v} fp32 state, "
+            f"{w.in_dtype} q/k/v, {'ragged fills, ' if w.ragged else ''}L={w.L}, merge={merge}")
+
+
 def to_dev(s, device):
     def up(x):
         if x is None:
@@ -236,7 +241,8 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     fused = args.merge == "fused"
-    w = wl.WORKLOADS["gdn_serving"].replace(L=args.L, B=args.B)
+    w = wl.WORKLOADS[args.workload]
+    w = w.replace(L=args.L or w.L, B=args.B or w.B)
     cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=fused,
                      step_split=args.split)
     stream = torch.cuda.current_stream(device)
@@ -249,6 +255,8 @@ def run_ours(args, world, rank, local):
     S0 = (torch.randn(w.heads * w.d_v * w.d_k, generator=gen, device=device) * w.s0_std).contiguous()
     fill0 = wl.fill_offsets(w)
 
+    bonus = (torch.from_numpy(wl.rwkv6_bonus(w)).to(device).reshape(-1)
+             if w.variant == wl.RWKV6 else None)
     st = dlb.DeltaLogState(cfg, device=device)
     st.reset(S0, fill0.tolist())
     o = torch.empty(w.heads * w.d_v, dtype=torch.float32, device=device)
@@ -257,7 +265,7 @@ def run_ours(args, world, rank, local):
         q, k, v, dec, beta = ring[i % RING]
         if ev is not None:
             ev[0].record(stream)
-        st.step(q, k, v, dec, beta, None, o)
+        st.step(q, k, v, dec, beta, bonus, o)
         if ev is not None:
             ev[1].record(stream)
         if not fused:
@@ -299,6 +307,7 @@ def run_ours(args, world, rank, local):
     if code != 0:
         raise RuntimeError(f"device error {code} at head {head}")
     max_elapsed = max_over_ranks(elapsed, world, device)
+    state_mib = w.heads * w.d_v * w.d_k * 4 / 2**20
     tokens = w.B * args.steps
     value = aggregate_value(tokens, world, max_elapsed)
 
@@ -311,7 +320,8 @@ def run_ours(args, world, rank, local):
     if os.path.exists(tfile):
         try:
             t = json.load(open(tfile))
-            if t.get("kernel_hash") == kernel_hash() and t.get("L") == args.L and t.get("merge") == args.merge:
+            if (t.get("kernel_hash") == kernel_hash() and t.get("L") == w.L and t.get("merge") == args.merge
+                    and t.get("workload") == w.name and t.get("B") == w.B):
                 traffic = t.get("bytes_per_launch")
         except Exception:
             traffic = None
@@ -320,7 +330,7 @@ def run_ours(args, world, rank, local):
         st.close()
         return {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "only_step": True,
-                "config": {"B": w.B, "L": args.L, "merge": args.merge, "split": args.split},
+                "config": {"workload": w.name, "B": w.B, "L": w.L, "merge": args.merge, "split": args.split},
                 "roofline": {"achieved": round(achieved, 1), "peak": peak,
                              "frac": round(achieved / peak, 4), "launch_ms": round(step_avg * 1e3, 5)}}
 
@@ -328,23 +338,30 @@ def run_ours(args, world, rank, local):
     S_e = S0.clone()
     for i in range(args.warmup):
         q, k, v, dec, beta = ring[i % RING]
-        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, None, o)
+        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, bonus, o)
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
         q, k, v, dec, beta = ring[i % RING]
-        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, None, o)
+        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, bonus, o)
     e1.record(stream)
     torch.cuda.synchronize(device)
     eager_s = e0.elapsed_time(e1) / 1e3
     erd, ewr = eager_bytes(cfg)
     del S_e
 
-    # end to end: pinned host inputs in, o out, every step
+    # End to end through the public API: every step copies its inputs from
+    # pinned host memory and its output o back to pinned host memory.  The
+    # copies and the kernel run on three streams so step i's compute overlaps
+    # step i+1's upload and step i-1's download (double-buffered device
+    # inputs and outputs; a buffer is reused only after the step that last
+    # used it has finished with it).
     pinned = []
     for s in host_steps:
-        arrs = [s.device_array("q"), s.device_array("k"), s.device_array("v"), s.decay, s.beta]
+        arrs = [s.device_array("q"), s.device_array("k"), s.device_array("v"), s.decay]
+        if s.beta is not None:
+            arrs.append(s.beta)
         ts = []
         for a in arrs:
             if a.dtype == np.uint16:
@@ -352,31 +369,53 @@ def run_ours(args, world, rank, local):
             else:
                 ts.append(torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).reshape(-1).pin_memory())
         pinned.append(ts)
-    dbuf = [torch.empty(t.numel(), dtype=t.dtype, device=device) for t in pinned[0]]
-    o_host = torch.empty(o.numel(), dtype=torch.float32).pin_memory()
+    NB = 2
+    dbufs = [[torch.empty(t.numel(), dtype=t.dtype, device=device) for t in pinned[0]] for _ in range(NB)]
+    obufs = [torch.empty(o.numel(), dtype=torch.float32, device=device) for _ in range(NB)]
+    o_hosts = [torch.empty(o.numel(), dtype=torch.float32).pin_memory() for _ in range(NB)]
     h2d = sum(t.numel() * t.element_size() for t in pinned[0])
-    d2h = o_host.numel() * 4
+    d2h = o_hosts[0].numel() * 4
+    s_cmp = stream
+    s_h2d = torch.cuda.Stream(device)
+    s_d2h = torch.cuda.Stream(device)
+    ev_h2d = [torch.cuda.Event() for _ in range(NB)]
+    ev_cmp = [torch.cuda.Event() for _ in range(NB)]
+    ev_d2h = [torch.cuda.Event() for _ in range(NB)]
 
     def e2e_step(i):
-        for d, h in zip(dbuf, pinned[i % RING]):
-            d.copy_(h, non_blocking=True)
-        q = dbuf[0].view(torch.bfloat16)
-        k = dbuf[1].view(torch.bfloat16)
-        v = dbuf[2].view(torch.bfloat16)
-        st.step(q, k, v, dbuf[3], dbuf[4], None, o)
+        b = i % NB
+        s_h2d.wait_event(ev_cmp[b])          # step i-NB has finished reading dbufs[b]
+        with torch.cuda.stream(s_h2d):
+            for d, h in zip(dbufs[b], pinned[i % RING]):
+                d.copy_(h, non_blocking=True)
+        ev_h2d[b].record(s_h2d)
+        s_cmp.wait_event(ev_h2d[b])
+        s_cmp.wait_event(ev_d2h[b])          # step i-NB's output has left obufs[b]
+        db = dbufs[b]
+        tin = cfg.torch_in_dtype
+        st.step(db[0].view(tin), db[1].view(tin), db[2].view(tin), db[3],
+                db[4] if len(db) > 4 else None, bonus, obufs[b], stream=s_cmp)
         if not fused:
-            st.merge(dlb.DL_MERGE_FULL)
-        o_host.copy_(o, non_blocking=True)
+            st.merge(dlb.DL_MERGE_FULL, stream=s_cmp)
+        ev_cmp[b].record(s_cmp)
+        s_d2h.wait_event(ev_cmp[b])
+        with torch.cuda.stream(s_d2h):
+            o_hosts[b].copy_(obufs[b], non_blocking=True)
+        ev_d2h[b].record(s_d2h)
 
     for i in range(args.warmup):
         e2e_step(i)
     torch.cuda.synchronize(device)
     dist_barrier(world)
     x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    x0.record(stream)
+    x0.record(s_cmp)
+    s_h2d.wait_event(x0)
+    s_d2h.wait_event(x0)
     for i in range(args.steps):
         e2e_step(i)
-    x1.record(stream)
+    for b in range(NB):
+        s_cmp.wait_event(ev_d2h[b])
+    x1.record(s_cmp)
     torch.cuda.synchronize(device)
     dist_barrier(world)
     e2e_s = max_over_ranks(x0.elapsed_time(x1) / 1e3, world, device)
@@ -395,12 +434,12 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"GDN decode B=512 H=32 d_k=d_v=128 fp32 state, bf16 q/k/v, "
-                               f"ragged fills, L={args.L}, merge={args.merge}",
-                   "B": w.B, "H": w.H, "d": w.d_k, "L": args.L, "merge": args.merge,
-                   "step_split": args.split,
-                   "global_batch": w.B * world, "parallelism": f"replicas x{world} (dp, no collective)",
-                   "l2": "state 1 GiB > 126 MB L2 on every step: no flush needed",
+        "config": {"workload": workload_desc(w, args.merge), "name": w.name,
+                   "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "L": w.L, "merge": args.merge,
+                   "step_split": args.split, "global_batch": w.B * world,
+                   "parallelism": f"replicas x{world} (dp, no collective)",
+                   "l2": (f"state {state_mib:.0f} MiB > 126 MB L2 on every step: no flush needed"
+                          if state_mib * 2**20 > L2_BYTES else f"state {state_mib:.0f} MiB fits L2: not a bench line"),
                    "input_ring_steps": RING},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -425,30 +464,33 @@ def run_ours(args, world, rank, local):
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_tokens_per_s(target_s: float, seqs: int = 2, steps_cap: int = 10**6):
-    """The fp64 oracle as it stands on a bounded sample of the workload:
-    the first ``seqs`` sequences (all 32 heads each), successive steps,
-    until ``target_s`` seconds of CPU work have run.  Returns (tokens/s,
-    steps, seconds, threads)."""
+def oracle_tokens_per_s(w, target_s: float = 0.0, seqs: int = 2, steps: int = 0, warmup: int = 0):
+    """The fp64 oracle as it stands on a bounded sample of the workload: the
+    first ``seqs`` sequences (all H heads each), one decode step at a time.
+    After ``warmup`` untimed steps it times either exactly ``steps`` steps or,
+    when ``steps`` is 0, steps until ``target_s`` seconds of oracle time.
+    Drawing the inputs is not timed.  Returns (tokens/s, steps, seconds,
+    threads)."""
+    import types
+
     import oracle
-    from oracle import recurrence as rec  # noqa: F401
-    w = wl.WORKLOADS["gdn_serving"]
+    seqs = min(seqs, w.B)
     heads = np.arange(seqs * w.H)
-    S = np.random.default_rng(w.seed).standard_normal((heads.size, w.d_v, w.d_k)) * w.s0_std
-    steps = 0
-    t0 = time.perf_counter()
-    el = 0.0
-    t = 0
-    while el < target_s and steps < steps_cap:
-        s = wl.step_inputs(w, t)  # drawing is not timed
-        sl = lambda x: x.reshape((w.heads,) + x.shape[2:])[heads][:, None]
-        import types
+    shape = (heads.size, w.d_k, w.d_v) if w.variant == wl.RWKV6 else (heads.size, w.d_v, w.d_k)
+    S = np.random.default_rng(w.seed).standard_normal(shape) * w.s0_std
+    bonus = wl.rwkv6_bonus(w)[heads % w.H] if w.variant == wl.RWKV6 else None
+    done, el, t = 0, 0.0, 0
+    while (done < steps) if steps > 0 else (el < target_s):
+        s = wl.step_inputs(w, t)
+        sl = lambda x: None if x is None else x.reshape((w.heads,) + x.shape[2:])[heads][:, None]
         st = types.SimpleNamespace(q=sl(s.q), k=sl(s.k), v=sl(s.v), decay=sl(s.decay), beta=sl(s.beta))
         a = time.perf_counter()
-        S = oracle.run_eager("gdn", S, [st]).S
-        el += time.perf_counter() - a
-        steps += 1
+        S = oracle.run_eager(w.variant, S, [st], bonus=bonus).S
+        dt = time.perf_counter() - a
         t += 1
+        if t > warmup:
+            el += dt
+            done += 1
     threads = None
     try:
         import threadpoolctl
@@ -456,25 +498,33 @@ def oracle_tokens_per_s(target_s: float, seqs: int = 2, steps_cap: int = 10**6):
         threads = max((i.get("num_threads", 1) for i in info), default=None)
     except Exception:
         threads = os.cpu_count()
-    return seqs * steps / el, steps, el, threads
+    return seqs * done / el, done, el, threads
+
+
+def cpu_sample_desc(w, steps, el, seqs=2):
+    n = min(seqs, w.B)
+    return (f"first {n} of {w.B} sequences ({n * w.H} heads), {steps} steps, "
+            f"{el:.1f} s of fp64 eager oracle time")
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    target = min(20.0, max(2.0, 0.02 * (args.steps + args.warmup)))
-    v, steps, el, threads = oracle_tokens_per_s(target)
+    w = wl.WORKLOADS[args.workload]
+    w = w.replace(L=args.L or w.L, B=args.B or w.B)
+    # each step decodes the first 2 sequences (1 when K is large) of the batch
+    seqs = 2 if args.steps + args.warmup <= 4000 else 1
+    v, steps, el, threads = oracle_tokens_per_s(w, seqs=seqs, steps=args.steps, warmup=args.warmup)
     return {
         "impl": "reference",
         "metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": world,
-        "steps": steps, "warmup": 0, "ms_per_step": round(el * 1e3 / steps, 3),
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"GDN decode B=512 H=32 d_k=d_v=128, L={args.L} (oracle: eager fp64)",
-                   "B": 512, "H": 32, "d": 128, "L": args.L},
+        "config": {"workload": workload_desc(w, args.merge) + " (oracle: eager fp64)",
+                   "name": w.name, "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "L": w.L},
         "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"first 2 of 512 sequences (64 heads), {steps} steps, "
-                                   f"{el:.1f} s of fp64 eager oracle time"},
+                         "sample": cpu_sample_desc(w, steps, el, seqs)},
         "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -484,8 +534,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--L", type=int, default=16)
-    ap.add_argument("--B", type=int, default=512, help="sequences (profiling runs use fewer)")
+    ap.add_argument("--workload", default="gdn_serving", choices=sorted(wl.WORKLOADS),
+                    help="synthetic workload (the headline line is gdn_serving)")
+    ap.add_argument("--L", type=int, default=0, help="log length (0: the workload's)")
+    ap.add_argument("--B", type=int, default=0, help="sequences (0: the workload's)")
     ap.add_argument("--split", type=int, default=0,
                     help="CTAs per head in the step kernel (0 = library default)")
     ap.add_argument("--only-step", action="store_true",
@@ -509,10 +561,11 @@ def main():
             return
         line = run_ours(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.only_step:
-            v, steps, el, threads = oracle_tokens_per_s(args.cpu_seconds)
+            w = wl.WORKLOADS[args.workload]
+            w = w.replace(L=args.L or w.L, B=args.B or w.B)
+            v, steps, el, threads = oracle_tokens_per_s(w, target_s=args.cpu_seconds, warmup=1)
             line["cpu_baseline"] = {"value": round(v, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": f"first 2 of 512 sequences (64 heads), {steps} steps, "
-                                              f"{el:.1f} s of fp64 eager oracle time"}
+                                    "sample": cpu_sample_desc(w, steps, el)}
         if rank == 0:
             print(json.dumps(line), flush=True)
         if args.sweep:

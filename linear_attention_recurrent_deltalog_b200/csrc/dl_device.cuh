@@ -126,6 +126,12 @@ __device__ __forceinline__ void tma_load_1d_stream(void* dst, const void* src, u
       : "memory");
 }
 
+// Bulk prefetch of global memory into L2 (no shared-memory destination).
+// src 16-B aligned; bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // --------------------------------------------------------- row reduction
 //
 // A warp covers rows of a d_v x d_k tile: LPR lanes per row, each lane

@@ -45,6 +45,7 @@ struct StepParams {
   float* o;
   int H;
   int L;
+  int prefetch;  // CTAs ahead whose tile and log this CTA prefetches into L2 (0: off)
 };
 
 struct MergeParams {
@@ -70,6 +71,7 @@ struct EagerParams {
   const float* bonus;
   float* o;
   int H;
+  int prefetch;  // CTAs ahead whose tile this CTA prefetches into L2 (0: off)
 };
 
 template <int VAR, typename TIn>
@@ -189,6 +191,24 @@ dl_step_kernel(const StepParams p) {
       mbar_arrive_expect_tx(&bars[c], Tl::kChunkBytes);
       tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
                          Tl::kChunkBytes, &bars[c]);
+    }
+  }
+  if (tid == 32 && p.prefetch > 0 && blockIdx.x + unsigned(p.prefetch) < gridDim.x) {
+    // Warm L2 for the CTA that starts `prefetch` CTAs later: its tile, then
+    // (once its fill is known) exactly the log entries it will read, so the
+    // DRAM stream does not wait for each CTA's own dependent fill -> log
+    // chain.  Adds no DRAM traffic: that CTA reads these bytes from L2.
+    const unsigned nb = blockIdx.x + unsigned(p.prefetch);
+    const size_t nh = nb / SPLIT;
+    const int nr0 = int(nb % SPLIT) * ROWS;
+    prefetch_l2(p.base + (nh * size_t(DV) + nr0) * DK, uint32_t(Tl::kTileBytes));
+    const int nf = p.fill_in[nh];
+    if (nf > 0 && nf < L) {
+      const TU* nU = static_cast<const TU*>(p.logU) + nh * size_t(L) * DV + nr0;
+      for (int i = 0; i < nf; ++i) prefetch_l2(nU + size_t(i) * DV, uint32_t(ROWS * sizeof(TU)));
+      prefetch_l2(static_cast<const TIn*>(p.logK) + nh * size_t(L) * DK,
+                  uint32_t(nf) * DK * sizeof(TIn));
+      prefetch_l2(p.logG + nh * size_t(GS), g_copy_bytes<VAR, DK>(nf));
     }
   }
   const int f = p.fill_in[head];
@@ -603,6 +623,8 @@ dl_eager_kernel(const EagerParams p) {
       tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
                          Tl::kChunkBytes, &bars[c]);
     }
+    if (p.prefetch > 0 && blockIdx.x + unsigned(p.prefetch) < gridDim.x)
+      prefetch_l2(p.S + (head + size_t(p.prefetch)) * size_t(DV) * DK, uint32_t(Tl::kTileBytes));
   }
   const TIn* gq = static_cast<const TIn*>(p.q) + head * DK;
   const TIn* gk = static_cast<const TIn*>(p.k) + head * DK;
