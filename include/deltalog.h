@@ -74,14 +74,19 @@ enum dl_flags {
   /* The step kernel merges in place: a head whose append would fill its
    * log writes the merged base instead and leaves an empty log, so the log
    * is never full and dl_merge(DL_MERGE_FULL) has nothing to do. */
-  DL_FLAG_FUSED_MERGE = 1
+  DL_FLAG_FUSED_MERGE = 1,
+  /* Use the step kernel that launches one CTA per work item instead of the
+   * persistent warp-specialised one (which is used whenever its ring of
+   * shared-memory stages fits).  A performance choice only. */
+  DL_FLAG_NONPERSISTENT = 2
 };
 
 /* Layer configuration.  d_k, d_v in {64, 128}; 1 <= L <= 64; B, H >= 1 and
  * B*H*d_v*d_k < 2^40.  `flags` is a bitwise OR of dl_flags.  `step_split`
- * is how many CTAs share one head's rows in the step kernel: 0 picks the
- * library's default, otherwise 1, 2 or 4 with d_v / step_split >= 32 (a
- * performance knob only: results do not depend on it). */
+ * is into how many work items (of d_v / step_split rows) the step kernel
+ * cuts one head: 0 picks the library's default, otherwise 1, 2 or 4 with
+ * d_v / step_split >= 32 (a performance knob only: results do not depend
+ * on it). */
 typedef struct dl_config {
   int32_t variant;    /* enum dl_variant */
   int32_t B;          /* sequences in the batch */

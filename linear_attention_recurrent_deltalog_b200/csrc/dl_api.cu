@@ -34,7 +34,7 @@ struct Layout {
   size_t base, u_off, u_bytes, k_off, k_bytes, g_off, g_bytes, log, fill_bytes, err_off, meta;
 };
 
-// Default CTAs per head for the step kernel.
+// Default work items per head for the step kernel: 64-row items.
 int default_split(const dl_config& c) { return c.d_v >= 128 ? 2 : 1; }
 int split_of(const dl_config& c) { return c.step_split == 0 ? default_split(c) : c.step_split; }
 
@@ -69,7 +69,8 @@ int check_config(const dl_config* c, bool need_L) {
   if (c->B < 1 || c->H < 1 || c->d_k < 1 || c->d_v < 1) return DL_ERR_ARG;
   if (c->in_dtype != DL_F32 && c->in_dtype != DL_BF16) return DL_ERR_ARG;
   if (need_L && (c->L < 1 || c->L > 64)) return DL_ERR_ARG;
-  if (need_L && (c->flags & ~int32_t(DL_FLAG_FUSED_MERGE)) != 0) return DL_ERR_ARG;
+  if (need_L && (c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_NONPERSISTENT)) != 0)
+    return DL_ERR_ARG;
   const uint64_t bh = uint64_t(c->B) * uint64_t(c->H);
   if (bh > 0x7fffffffull) return DL_ERR_ARG;  // one CTA per head in a 1-D grid
   if (bh * uint64_t(c->d_v) * uint64_t(c->d_k) >= (1ull << 40)) return DL_ERR_ARG;
@@ -79,7 +80,8 @@ int check_config(const dl_config* c, bool need_L) {
 }
 
 Shape shape_of(const dl_config& c) {
-  return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0, split_of(c)};
+  return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0, split_of(c),
+               (c.flags & DL_FLAG_NONPERSISTENT) ? 0 : 1};
 }
 
 cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, cudaStream_t s) {

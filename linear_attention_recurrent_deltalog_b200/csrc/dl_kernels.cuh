@@ -30,7 +30,7 @@ namespace dl {
 
 struct StepParams {
   float* base;   // [BH, DV, DK]
-  void* logU;    // [BH, L, DV]  fp32 (in_dtype for RWKV6)
+  void* logU;    // [BH, DV/32, L, 32]  fp32 (in_dtype for RWKV6): see u_offset
   void* logK;    // [BH, L, DK]  in_dtype
   float* logG;   // [BH, L, GW]
   const int* fill_in;  // [BH] entries before this step
@@ -45,7 +45,7 @@ struct StepParams {
   float* o;
   int H;
   int L;
-  int prefetch;  // CTAs ahead whose tile and log this CTA prefetches into L2 (0: off)
+  int nitems;    // work items (head rows) of a persistent launch
 };
 
 struct MergeParams {
@@ -71,7 +71,6 @@ struct EagerParams {
   const float* bonus;
   float* o;
   int H;
-  int prefetch;  // CTAs ahead whose tile this CTA prefetches into L2 (0: off)
 };
 
 template <int VAR, typename TIn>
@@ -80,6 +79,20 @@ template <typename TIn>
 struct LogU<kVarRWKV6, TIn> { using type = TIn; };  // RWKV6 logs v itself
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// The log's u vectors are stored in blocks of 32 value rows: [head][row
+// block][entry][32].  The f entries of one row block are contiguous, so a
+// work item of ROWS rows fetches its u rows with ROWS/32 bulk copies
+// whatever f is, and an append writes 32 consecutive values per block.
+constexpr int kURows = 32;
+__host__ __device__ constexpr size_t u_offset(size_t head, int row, int entry, int L, int DV) {
+  return ((head * size_t(DV / kURows) + size_t(row / kURows)) * size_t(L) + size_t(entry)) * kURows +
+         size_t(row % kURows);
+}
+// Same, inside a staged copy that starts at row block `row0 / 32` of a head.
+__host__ __device__ constexpr int su_offset(int local_row, int entry, int L) {
+  return ((local_row / kURows) * L + entry) * kURows + local_row % kURows;
+}
 
 // Per-head stride of the log-decay array: GDN keeps one scalar per entry,
 // padded to a multiple of 4 entries so a head's block starts 16-B aligned and
@@ -178,7 +191,7 @@ dl_step_kernel(const StepParams p) {
   const int h = static_cast<int>(head % static_cast<size_t>(p.H));
 
   const float* gS = p.base + (head * size_t(DV) + r0) * DK;
-  TU* gU = static_cast<TU*>(p.logU) + head * size_t(L) * DV;
+  TU* gU = static_cast<TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
   TIn* gK = static_cast<TIn*>(p.logK) + head * size_t(L) * DK;
   float* gG = p.logG + head * size_t(GS);
 
@@ -193,24 +206,6 @@ dl_step_kernel(const StepParams p) {
                          Tl::kChunkBytes, &bars[c]);
     }
   }
-  if (tid == 32 && p.prefetch > 0 && blockIdx.x + unsigned(p.prefetch) < gridDim.x) {
-    // Warm L2 for the CTA that starts `prefetch` CTAs later: its tile, then
-    // (once its fill is known) exactly the log entries it will read, so the
-    // DRAM stream does not wait for each CTA's own dependent fill -> log
-    // chain.  Adds no DRAM traffic: that CTA reads these bytes from L2.
-    const unsigned nb = blockIdx.x + unsigned(p.prefetch);
-    const size_t nh = nb / SPLIT;
-    const int nr0 = int(nb % SPLIT) * ROWS;
-    prefetch_l2(p.base + (nh * size_t(DV) + nr0) * DK, uint32_t(Tl::kTileBytes));
-    const int nf = p.fill_in[nh];
-    if (nf > 0 && nf < L) {
-      const TU* nU = static_cast<const TU*>(p.logU) + nh * size_t(L) * DV + nr0;
-      for (int i = 0; i < nf; ++i) prefetch_l2(nU + size_t(i) * DV, uint32_t(ROWS * sizeof(TU)));
-      prefetch_l2(static_cast<const TIn*>(p.logK) + nh * size_t(L) * DK,
-                  uint32_t(nf) * DK * sizeof(TIn));
-      prefetch_l2(p.logG + nh * size_t(GS), g_copy_bytes<VAR, DK>(nf));
-    }
-  }
   const int f = p.fill_in[head];
   if (f < 0 || f >= L) {  // the host never launches a step on a full log
     if (tid == 0) {
@@ -222,14 +217,15 @@ dl_step_kernel(const StepParams p) {
   const bool merge_now = FUSED && (f + 1 == L);
   const bool appender = (part == 0) && !merge_now;
   if (tid == 0 && f > 0) {
-    const uint32_t bu = uint32_t(ROWS) * sizeof(TU);
+    const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one row block
     const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
     const uint32_t bg = g_copy_bytes<VAR, DK>(f);
-    mbar_arrive_expect_tx(barLog, bu * uint32_t(f) + bk + bg);
+    mbar_arrive_expect_tx(barLog, bu * uint32_t(ROWS / kURows) + bk + bg);
     tma_load_1d(sK, gK, bk, barLog);
     tma_load_1d(sG, gG, bg, barLog);
-    for (int i = 0; i < f; ++i)
-      tma_load_1d(sU + size_t(i) * ROWS, gU + size_t(i) * DV + r0, bu, barLog);
+    for (int rb = 0; rb < ROWS / kURows; ++rb)
+      tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, r0 + rb * kURows, 0, L, DV), bu,
+                  barLog);
   }
 
   // ---- per-head vectors while the tile and the log stream in
@@ -369,7 +365,7 @@ dl_step_kernel(const StepParams p) {
   // ---- log correction, delta-rule correction and readout for row r0 + jl
   float ck = 0.f, cq = 0.f;
   for (int i = 0; i < f; ++i) {
-    const float uij = to_f(sU[size_t(i) * ROWS + jl]);
+    const float uij = to_f(sU[su_offset(jl, i, L)]);
     if (VAR != kVarRWKV6) ck = fmaf(sW[i], uij, ck);
     cq = fmaf(sZ[i], uij, cq);
   }
@@ -390,9 +386,9 @@ dl_step_kernel(const StepParams p) {
   if ((lane & 1) == 0) {
     p.o[head * DV + r0 + jl] = o;
     if (merge_now)
-      sU[size_t(f) * ROWS + jl] = Elem<TU>::from_f(u);
+      sU[su_offset(jl, f, L)] = Elem<TU>::from_f(u);
     else
-      gU[size_t(f) * DV + r0 + jl] = Elem<TU>::from_f(u);
+      gU[u_offset(0, r0 + jl, f, L, DV)] = Elem<TU>::from_f(u);
   }
   if (!merge_now) return;
 
@@ -426,7 +422,7 @@ dl_step_kernel(const StepParams p) {
     }
 #pragma unroll
     for (int pi = 0; pi < NV; ++pi) {
-      const float ui = to_f(sU[size_t(i) * ROWS + j0 + pi * RPI + rsub]);
+      const float ui = to_f(sU[su_offset(j0 + pi * RPI + rsub, i, L)]);
       acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
       acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
       acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
@@ -495,7 +491,7 @@ dl_merge_kernel(const MergeParams p) {
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const float* gS = p.base + head * size_t(DV) * DK;
-  const TU* gU = static_cast<const TU*>(p.logU) + head * size_t(L) * DV;
+  const TU* gU = static_cast<const TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
   const TIn* gK = static_cast<const TIn*>(p.logK) + head * size_t(L) * DK;
   const float* gG = p.logG + head * size_t(GS);
 
@@ -510,11 +506,12 @@ dl_merge_kernel(const MergeParams p) {
                          Tl::kChunkBytes, &bars[c]);
     }
     if (f > 0) {
-      const uint32_t bu = uint32_t(f) * DV * sizeof(TU);
+      const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one row block
       const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
       const uint32_t bg = g_copy_bytes<VAR, DK>(f);
-      mbar_arrive_expect_tx(barLog, bu + bk + bg);
-      tma_load_1d(sU, gU, bu, barLog);
+      mbar_arrive_expect_tx(barLog, bu * uint32_t(DV / kURows) + bk + bg);
+      for (int rb = 0; rb < DV / kURows; ++rb)
+        tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, rb * kURows, 0, L, DV), bu, barLog);
       tma_load_1d(sK, gK, bk, barLog);
       tma_load_1d(sG, gG, bg, barLog);
     }
@@ -555,7 +552,7 @@ dl_merge_kernel(const MergeParams p) {
     const float4 k4 = *reinterpret_cast<const float4*>(sKt + size_t(i) * DK + c0);
 #pragma unroll
     for (int pi = 0; pi < NV; ++pi) {
-      const float ui = to_f(sU[size_t(i) * DV + j0 + pi * RPI + rsub]);
+      const float ui = to_f(sU[su_offset(j0 + pi * RPI + rsub, i, L)]);
       acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
       acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
       acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
@@ -623,8 +620,6 @@ dl_eager_kernel(const EagerParams p) {
       tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
                          Tl::kChunkBytes, &bars[c]);
     }
-    if (p.prefetch > 0 && blockIdx.x + unsigned(p.prefetch) < gridDim.x)
-      prefetch_l2(p.S + (head + size_t(p.prefetch)) * size_t(DV) * DK, uint32_t(Tl::kTileBytes));
   }
   const TIn* gq = static_cast<const TIn*>(p.q) + head * DK;
   const TIn* gk = static_cast<const TIn*>(p.k) + head * DK;

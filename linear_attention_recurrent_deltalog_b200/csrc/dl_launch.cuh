@@ -9,6 +9,7 @@
 #include <cstdlib>
 
 #include "dl_kernels.cuh"
+#include "dl_step_persistent.cuh"
 
 namespace dl {
 
@@ -16,8 +17,9 @@ namespace dl {
 struct Shape {
   int dk;
   int dv;
-  int bf16;   // 1: q/k/v are bf16, 0: fp32
-  int split;  // step kernel: CTAs per head (1, 2 or 4; d_v / split >= 32)
+  int bf16;        // 1: q/k/v are bf16, 0: fp32
+  int split;       // step kernel: work items per head (1, 2 or 4; d_v / split >= 32)
+  int persistent;  // 1: persistent warp-specialised step kernel when its ring fits
 };
 
 inline bool split_ok(int dv, int split) {
@@ -45,43 +47,6 @@ inline cudaError_t prepare_kernel(Kern kern, std::atomic<unsigned long long>& do
   return cudaSuccess;
 }
 
-// How far ahead (in CTAs) a CTA warms L2 for a later CTA, as a multiple of
-// the number of CTAs resident on the whole GPU at once (1.0 = the CTA that
-// will take this CTA's place).  Off by default: on B200 it measured neutral
-// for the step kernel and slightly negative for the eager kernel.
-// DELTALOG_PREFETCH_SCALE (read once) sets it.
-inline float prefetch_scale() {
-  static const float scale = [] {
-    const char* e = std::getenv("DELTALOG_PREFETCH_SCALE");
-    if (e == nullptr || *e == 0) return 0.0f;
-    const float v = static_cast<float>(std::atof(e));
-    return v < 0.f ? 0.f : (v > 8.f ? 8.f : v);
-  }();
-  return scale;
-}
-
-// Resident CTAs of `kern` on the current device for this launch shape,
-// cached per device and shared-memory size.
-template <typename Kern>
-int resident_ctas(Kern kern, int threads, size_t smem) {
-  struct Entry {
-    std::atomic<long long> smem{-1};
-    std::atomic<int> ctas{0};
-  };
-  static Entry cache[kMaxDevices];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-  if (cache[dev].smem.load(std::memory_order_acquire) == static_cast<long long>(smem))
-    return cache[dev].ctas.load(std::memory_order_relaxed);
-  int sms = 0, per = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, threads, smem) != cudaSuccess)
-    return 0;
-  cache[dev].ctas.store(sms * per, std::memory_order_relaxed);
-  cache[dev].smem.store(static_cast<long long>(smem), std::memory_order_release);
-  return sms * per;
-}
-
 template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
 cudaError_t launch_step_t(const StepParams& p, unsigned nheads, cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
@@ -89,10 +54,7 @@ cudaError_t launch_step_t(const StepParams& p, unsigned nheads, cudaStream_t s) 
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
   const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn>(p.L).total;
-  StepParams q = p;
-  q.prefetch = static_cast<int>(prefetch_scale() *
-                                resident_ctas(kern, Tile<DK, ROWS>::kThreads, smem));
-  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(q);
+  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -114,10 +76,7 @@ cudaError_t launch_eager_t(const EagerParams& p, unsigned nheads, cudaStream_t s
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
   const size_t smem = EagerLayout<DK, DV>().total;
-  EagerParams q = p;
-  q.prefetch = static_cast<int>(prefetch_scale() *
-                                resident_ctas(kern, Tile<DK, DV>::kThreads, smem));
-  kern<<<nheads, Tile<DK, DV>::kThreads, smem, s>>>(q);
+  kern<<<nheads, Tile<DK, DV>::kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -169,14 +128,74 @@ DL_DECLARE_VARIANT_LAUNCHERS(kVarRWKV6)
 
 // Functors the shape dispatch calls (namespace scope: local classes cannot
 // have member templates).
+// Ring stages of the persistent step kernel that fit in shared memory
+// (capped by DELTALOG_MAX_STAGES, default 8).
+inline int max_stages() {
+  static const int m = [] {
+    const char* e = std::getenv("DELTALOG_MAX_STAGES");
+    const int v = (e && *e) ? std::atoi(e) : 8;
+    return v < 2 ? 2 : (v > 8 ? 8 : v);
+  }();
+  return m;
+}
+
+inline int sm_count() {
+  static std::atomic<int> cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+template <int VAR, int DK, int DV, int ROWS, typename TIn>
+int persistent_stages(int L) {
+  const size_t stage = PStage<VAR, DK, DV, ROWS, TIn>(L).bytes + 16;
+  const int n = int((size_t(kMaxSmemOptIn) - 256) / stage);
+  return n < max_stages() ? n : max_stages();
+}
+
+// Persistent launch: one CTA per SM (or per item when there are fewer).
+// Returns cudaErrorNotSupported when its ring would have fewer than 2 stages.
+template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
+cudaError_t launch_step_persistent_t(const StepParams& p, unsigned nheads, cudaStream_t s) {
+  const int nst = persistent_stages<VAR, DK, DV, ROWS, TIn>(p.L);
+  if (nst < 2) return cudaErrorNotSupported;
+  static std::atomic<unsigned long long> done{0};
+  auto kern = dl_step_persistent_kernel<VAR, DK, DV, ROWS, TIn, FUSED>;
+  cudaError_t e = prepare_kernel(kern, done);
+  if (e != cudaSuccess) return e;
+  const size_t smem = size_t(nst) * PStage<VAR, DK, DV, ROWS, TIn>(p.L).bytes + 16 * size_t(nst);
+  const unsigned nitems = nheads * unsigned(DV / ROWS);
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const unsigned grid = nitems < unsigned(sms) ? nitems : unsigned(sms);
+  StepParams q = p;
+  q.nitems = int(nitems);
+  kern<<<grid, PGeom<ROWS>::kThreads, smem, s>>>(q, nst);
+  return cudaGetLastError();
+}
+
+template <int VAR, int DK, int DV, int ROWS, typename T, bool FUSED>
+cudaError_t launch_step_rows(bool persistent, const StepParams& p, unsigned n, cudaStream_t s) {
+  if (persistent) {
+    const cudaError_t e = launch_step_persistent_t<VAR, DK, DV, ROWS, T, FUSED>(p, n, s);
+    if (e != cudaErrorNotSupported) return e;
+  }
+  return launch_step_t<VAR, DK, DV, ROWS, T, FUSED>(p, n, s);
+}
+
 template <int VAR, int DK, int DV, typename T, bool FUSED>
-cudaError_t launch_step_split(int split, const StepParams& p, unsigned n, cudaStream_t s) {
-  if (split == 1) return launch_step_t<VAR, DK, DV, DV, T, FUSED>(p, n, s);
+cudaError_t launch_step_split(int split, bool persistent, const StepParams& p, unsigned n,
+                              cudaStream_t s) {
+  if (split == 1) return launch_step_rows<VAR, DK, DV, DV, T, FUSED>(persistent, p, n, s);
   if constexpr (DV / 2 >= 32) {
-    if (split == 2) return launch_step_t<VAR, DK, DV, DV / 2, T, FUSED>(p, n, s);
+    if (split == 2) return launch_step_rows<VAR, DK, DV, DV / 2, T, FUSED>(persistent, p, n, s);
   }
   if constexpr (DV / 4 >= 32) {
-    if (split == 4) return launch_step_t<VAR, DK, DV, DV / 4, T, FUSED>(p, n, s);
+    if (split == 4) return launch_step_rows<VAR, DK, DV, DV / 4, T, FUSED>(persistent, p, n, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -188,10 +207,11 @@ struct StepRun {
   cudaStream_t s;
   bool fused;
   int split;
+  bool persistent;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    return fused ? launch_step_split<VAR, DK, DV, T, true>(split, p, n, s)
-                 : launch_step_split<VAR, DK, DV, T, false>(split, p, n, s);
+    return fused ? launch_step_split<VAR, DK, DV, T, true>(split, persistent, p, n, s)
+                 : launch_step_split<VAR, DK, DV, T, false>(split, persistent, p, n, s);
   }
 };
 template <int VAR>
@@ -243,7 +263,7 @@ struct MergeSmem {
   template <>                                                                              \
   cudaError_t launch_step<VAR>(const Shape& sh, bool fused, const StepParams& p,           \
                                unsigned nheads, cudaStream_t s) {                          \
-    StepRun<VAR> f{p, nheads, s, fused, sh.split};                                                   \
+    StepRun<VAR> f{p, nheads, s, fused, sh.split, sh.persistent != 0};                                                   \
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
   template <>                                                                              \

@@ -68,18 +68,28 @@ def test_shapes_and_dtypes(variant, dk, dv, dtype):
     w = wl.WORKLOADS[base].replace(B=5, H=3, d_k=dk, d_v=dv, in_dtype=dtype, L=6, T=29,
                                    ragged=True)
     for split in (1, dv // 32):
-        _check(run_parity(w, snap_every=7, workers=0, split=split))
+        for persistent in (True, False):
+            _check(run_parity(w, snap_every=7, workers=0, split=split, persistent=persistent))
 
 
+@pytest.mark.parametrize("persistent", [True, False])
 @pytest.mark.parametrize("split", [1, 2, 4])
 @pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
-def test_step_split(name, split):
-    # a head's rows shared by 1, 2 or 4 CTAs: same results
+def test_step_split(name, split, persistent):
+    # a head cut into 1, 2 or 4 work items, persistent or one CTA per item
     w = wl.WORKLOADS[name]
     if w.d_v // split < 32:
         pytest.skip("d_v / split < 32 is not built")
     w = w.replace(B=6, H=5, L=8, T=27, ragged=True)
-    _check(run_parity(w, snap_every=9, workers=0, split=split, arms=("log", "fused")))
+    _check(run_parity(w, snap_every=9, workers=0, split=split, persistent=persistent,
+                      arms=("log", "fused")))
+
+
+@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
+def test_nonpersistent_full_workload(name):
+    w = wl.WORKLOADS[name]
+    res = run_parity(w, T=64, heads=wl.sample_heads(w, 24), persistent=False, arms=("fused",))
+    _check(res)
 
 
 @pytest.mark.parametrize("L", [1, 2, 64])
