@@ -84,13 +84,14 @@ Shape shape_of(const dl_config& c) {
                (c.flags & DL_FLAG_NONPERSISTENT) ? 0 : 1};
 }
 
-cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, cudaStream_t s) {
+cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, const dl::FillParam& fp,
+                        cudaStream_t s) {
   const unsigned n = unsigned(size_t(c.B) * c.H);
   const bool fused = (c.flags & DL_FLAG_FUSED_MERGE) != 0;
   switch (c.variant) {
-    case DL_GDN: return dl::launch_step<dl::kVarGDN>(shape_of(c), fused, p, n, s);
-    case DL_KDA: return dl::launch_step<dl::kVarKDA>(shape_of(c), fused, p, n, s);
-    default: return dl::launch_step<dl::kVarRWKV6>(shape_of(c), fused, p, n, s);
+    case DL_GDN: return dl::launch_step<dl::kVarGDN>(shape_of(c), fused, p, fp, n, s);
+    case DL_KDA: return dl::launch_step<dl::kVarKDA>(shape_of(c), fused, p, fp, n, s);
+    default: return dl::launch_step<dl::kVarRWKV6>(shape_of(c), fused, p, fp, n, s);
   }
 }
 
@@ -150,6 +151,7 @@ struct dl_state {
   int n_full;                       // sequences whose log holds L entries
   int n_nonempty;                   // sequences whose log holds >= 1 entry
   int parity;                       // which fill array holds the current counts
+  dl::FillParam fill_param;         // the mirror as a launch argument (B <= kParamFills)
 
   int* dev_fill(int which) const {
     return reinterpret_cast<int*>(meta + size_t(which) * lay.fill_bytes);
@@ -277,7 +279,11 @@ int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v, co
   p.o = o;
   p.H = c.H;
   p.L = c.L;
-  if (launch_step(c, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
+  p.fills_in_param = (c.B <= dl::kParamFills) ? 1 : 0;
+  if (p.fills_in_param)
+    for (int b = 0; b < c.B; ++b) st->fill_param.f[b] = static_cast<uint8_t>(st->fill[b]);
+  if (launch_step(c, p, st->fill_param, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DL_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   st->parity ^= 1;
   for (int32_t& f : st->fill) {

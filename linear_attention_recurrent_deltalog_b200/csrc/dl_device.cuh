@@ -50,6 +50,35 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
   return f;
 }
 
+// N consecutive elements (N a multiple of 4 for fp32, of 8 for bf16; p
+// aligned to 16 bytes) as fp32, with 16-byte shared/global vector loads.
+template <int N>
+__device__ __forceinline__ void load_f(const float* p, float (&out)[N]) {
+  static_assert(N % 4 == 0, "whole float4s");
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i) {
+    const float4 v = reinterpret_cast<const float4*>(p)[i];
+    out[4 * i] = v.x;
+    out[4 * i + 1] = v.y;
+    out[4 * i + 2] = v.z;
+    out[4 * i + 3] = v.w;
+  }
+}
+template <int N>
+__device__ __forceinline__ void load_f(const __nv_bfloat16* p, float (&out)[N]) {
+  static_assert(N % 8 == 0, "whole 16-byte groups");
+#pragma unroll
+  for (int i = 0; i < N / 8; ++i) {
+    const uint4 r = reinterpret_cast<const uint4*>(p)[i];
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      out[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+      out[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+}
+
 __device__ __forceinline__ float dot4(float4 a, float4 b) {
   return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
@@ -212,7 +241,10 @@ struct Tile {
   static constexpr int kLPR = DK / 4;              // lanes per row (float4 each)
   static constexpr int kRPI = 32 / kLPR;           // rows per warp instruction
   static constexpr int kNV = kRowsPerWarp / kRPI;  // partials per lane
-  static constexpr int kChunkRows = 32;            // rows per bulk copy
+  // Rows per bulk copy: one copy per warp's 16 rows (8 KiB at d_k = 128).
+  // B200 streams a single bulk copy far slower than HBM can deliver, so a
+  // tile goes out as several concurrent copies.
+  static constexpr int kChunkRows = 16;
   static constexpr int kChunks = ROWS / kChunkRows;
   static constexpr uint32_t kChunkBytes = kChunkRows * DK * 4;
   static constexpr size_t kTileBytes = size_t(ROWS) * DK * 4;

@@ -28,6 +28,15 @@
 
 namespace dl {
 
+// Per-sequence fills passed by value with the launch (the host keeps an
+// exact mirror of them), so a step CTA knows how many log entries to fetch
+// without first reading a device counter.  Batches of more than
+// kParamFills sequences read the device fill array instead.
+constexpr int kParamFills = 16384;
+struct FillParam {
+  uint8_t f[kParamFills];
+};
+
 struct StepParams {
   float* base;   // [BH, DV, DK]
   void* logU;    // [BH, DV/32, L, 32]  fp32 (in_dtype for RWKV6): see u_offset
@@ -46,7 +55,13 @@ struct StepParams {
   int H;
   int L;
   int nitems;    // work items (head rows) of a persistent launch
+  int fills_in_param;  // 1: read fills from the FillParam argument
 };
+
+// Entries in the log of `head` before this step.
+__device__ __forceinline__ int step_fill(const StepParams& p, const FillParam& fp, size_t head) {
+  return p.fills_in_param ? int(fp.f[head / size_t(p.H)]) : p.fill_in[head];
+}
 
 struct MergeParams {
   float* base;
@@ -108,6 +123,76 @@ __device__ __forceinline__ uint32_t g_copy_bytes(int f) {
   return VAR == kVarGDN ? uint32_t((f + 3) / 4) * 16u : uint32_t(f) * DK * 4u;
 }
 
+// Per-entry weights of the log correction for the f entries of one head,
+// computed entry-parallel: eight lanes share an entry (d_k/8 key channels
+// each), so a warp covers four entries per pass and each sum needs a 3-level
+// shuffle reduction rather than a full 5-level one per entry.
+//   GDN  : W_i = e^{g_t - g_i} (k_i . k_t),  Z_i = e^{g_t - g_i} (k_i . q_t)
+//   KDA  : W_i = sum_c k_i[c] k_t[c] e^{g_t[c] - g_i[c]},  Z_i the same with q_t
+//   RWKV6: Z_i = sum_c k_i[c] r_t[c] e^{g_{t-1}[c] - g_i[c]}
+// kin, qin: k_t and q_t (r_t) in shared memory (fp32 or the input type);
+// sK: the staged log keys [f][DK]; sG: the staged log-decay; dec: the
+// step's decay (one scalar for GDN, d_k values otherwise).  Requires f > 0.
+template <int VAR, int DK, typename TK, typename TIn>
+__device__ __forceinline__ void entry_weights(int f, int warp, int nwarps, int lane, const TK* kin,
+                                              const TK* qin, const TIn* sK, const float* sG,
+                                              const float* dec, float* sW, float* sZ) {
+  constexpr int CPE = DK / 8;  // channels per lane
+  const int slot = lane >> 3;
+  const int c0 = (lane & 7) * CPE;
+  float kl[CPE], ql[CPE], gl[CPE];
+  load_f<CPE>(kin + c0, kl);
+  load_f<CPE>(qin + c0, ql);
+  float gt0 = 0.f;
+  if (VAR == kVarGDN) {
+    gt0 = sG[f - 1] + logf(dec[0]);
+  } else {
+    load_f<CPE>(sG + size_t(f - 1) * DK + c0, gl);
+    if (VAR == kVarKDA) {
+      float dl[CPE];
+      load_f<CPE>(dec + c0, dl);
+#pragma unroll
+      for (int c = 0; c < CPE; ++c) gl[c] += logf(dl[c]);
+    }
+  }
+  for (int base = warp * 4; base < f; base += nwarps * 4) {
+    const int i = base + slot;
+    float x = 0.f, y = 0.f;
+    if (i < f) {
+      float ki[CPE];
+      load_f<CPE>(sK + size_t(i) * DK + c0, ki);
+      if (VAR != kVarGDN) {
+        float gi[CPE];
+        load_f<CPE>(sG + size_t(i) * DK + c0, gi);
+#pragma unroll
+        for (int c = 0; c < CPE; ++c) ki[c] *= expf(gl[c] - gi[c]);
+      }
+#pragma unroll
+      for (int c = 0; c < CPE; ++c) {
+        if (VAR != kVarRWKV6) x = fmaf(ki[c], kl[c], x);
+        y = fmaf(ki[c], ql[c], y);
+      }
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+      if (VAR != kVarRWKV6) x += __shfl_xor_sync(0xffffffffu, x, o);
+      y += __shfl_xor_sync(0xffffffffu, y, o);
+    }
+    if (i < f && (lane & 7) == 0) {
+      float e = 1.f;
+      if (VAR == kVarGDN) e = expf(gt0 - sG[i]);
+      sW[i] = x * e;
+      sZ[i] = y * e;
+    }
+  }
+}
+
+// The 16 staged u values of rows j0 .. j0+15 (one 32-row block) of entry i.
+template <typename TU>
+__device__ __forceinline__ void load_u16(const TU* sU, int j0, int i, int L, float (&u)[16]) {
+  load_f<16>(sU + su_offset(j0, i, L), u);
+}
+
 // ------------------------------------------------------------------ step
 //
 // A head's rows may be split over SPLIT = DV / ROWS CTAs (blockIdx.x =
@@ -147,7 +232,7 @@ struct StepLayout {
 
 template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
 __global__ void __launch_bounds__(Tile<DK, ROWS>::kThreads)
-dl_step_kernel(const StepParams p) {
+dl_step_kernel(const StepParams p, const FillParam fp) {
   using Tl = Tile<DK, ROWS>;
   using TU = typename LogU<VAR, TIn>::type;
   constexpr int SPLIT = DV / ROWS;
@@ -206,7 +291,7 @@ dl_step_kernel(const StepParams p) {
                          Tl::kChunkBytes, &bars[c]);
     }
   }
-  const int f = p.fill_in[head];
+  const int f = step_fill(p, fp, head);
   if (f < 0 || f >= L) {  // the host never launches a step on a full log
     if (tid == 0) {
       if (p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
@@ -278,47 +363,8 @@ dl_step_kernel(const StepParams p) {
       if (appender) gG[size_t(f) * DK + c] = gt;
     }
   }
-  if (f > 0) {
-    // g_t (KDA) or g_{t-1} (RWKV6) for this lane's key columns, and g_t for GDN
-    float gl[CPL];
-    float gt0 = 0.f;
-    if (VAR == kVarGDN) {
-      gt0 = sG[f - 1] + logf(sDec[0]);
-    } else {
-#pragma unroll
-      for (int cc = 0; cc < CPL; ++cc) {
-        const int c = lane * CPL + cc;
-        gl[cc] = sG[size_t(f - 1) * DK + c] + (VAR == kVarKDA ? logf(sDec[c]) : 0.f);
-      }
-    }
-    for (int i = warp; i < f; i += NW) {
-      float x = 0.f, y = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < CPL; ++cc) {
-        const int c = lane * CPL + cc;
-        const float ki = to_f(sK[size_t(i) * DK + c]);
-        if (VAR == kVarGDN) {
-          x = fmaf(ki, sk[c], x);
-          y = fmaf(ki, sq[c], y);
-        } else {
-          const float kie = ki * expf(gl[cc] - sG[size_t(i) * DK + c]);
-          if (VAR == kVarKDA) x = fmaf(kie, sk[c], x);
-          y = fmaf(kie, sq[c], y);
-        }
-      }
-      if (VAR != kVarRWKV6) x = warp_sum(x);
-      y = warp_sum(y);
-      if (VAR == kVarGDN) {
-        const float e = expf(gt0 - sG[i]);
-        x *= e;
-        y *= e;
-      }
-      if (lane == 0) {
-        sW[i] = x;
-        sZ[i] = y;
-      }
-    }
-  }
+  if (f > 0)
+    entry_weights<VAR, DK, float, TIn>(f, warp, NW, lane, sk, sq, sK, sG, sDec, sW, sZ);
   if (warp == NW - 1) {
     // GDN/KDA: k_t . q_t (the current entry's own weight on q);
     // RWKV6: the bonus sum_c r_c u_c k_c.
@@ -420,9 +466,11 @@ dl_step_kernel(const StepParams p) {
         k4.w *= expf(sGt[c0 + 3] - gi[3]);
       }
     }
+    float u16[16];
+    load_u16(sU, j0, i, L, u16);
 #pragma unroll
     for (int pi = 0; pi < NV; ++pi) {
-      const float ui = to_f(sU[su_offset(j0 + pi * RPI + rsub, i, L)]);
+      const float ui = (RPI == 1) ? u16[pi] : (rsub ? u16[pi * RPI + 1] : u16[pi * RPI]);
       acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
       acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
       acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
@@ -550,9 +598,11 @@ dl_merge_kernel(const MergeParams p) {
   }
   for (int i = 0; i < f; ++i) {
     const float4 k4 = *reinterpret_cast<const float4*>(sKt + size_t(i) * DK + c0);
+    float u16[16];
+    load_u16(sU, j0, i, L, u16);
 #pragma unroll
     for (int pi = 0; pi < NV; ++pi) {
-      const float ui = to_f(sU[su_offset(j0 + pi * RPI + rsub, i, L)]);
+      const float ui = (RPI == 1) ? u16[pi] : (rsub ? u16[pi * RPI + 1] : u16[pi * RPI]);
       acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
       acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
       acc[pi].z = fmaf(ui, k4.z, acc[pi].z);

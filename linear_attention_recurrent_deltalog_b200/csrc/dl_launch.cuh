@@ -48,13 +48,14 @@ inline cudaError_t prepare_kernel(Kern kern, std::atomic<unsigned long long>& do
 }
 
 template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
-cudaError_t launch_step_t(const StepParams& p, unsigned nheads, cudaStream_t s) {
+cudaError_t launch_step_t(const StepParams& p, const FillParam& fp, unsigned nheads,
+                          cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
   auto kern = dl_step_kernel<VAR, DK, DV, ROWS, TIn, FUSED>;
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
   const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn>(p.L).total;
-  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p);
+  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p, fp);
   return cudaGetLastError();
 }
 
@@ -97,8 +98,8 @@ inline cudaError_t dispatch_shape(const Shape& sh, F&& f) {
 
 // Per-variant entry points (defined in dl_kernels_<variant>.cu).
 template <int VAR>
-cudaError_t launch_step(const Shape& sh, bool fused, const StepParams& p, unsigned nheads,
-                        cudaStream_t s);
+cudaError_t launch_step(const Shape& sh, bool fused, const StepParams& p, const FillParam& fp,
+                        unsigned nheads, cudaStream_t s);
 template <int VAR>
 cudaError_t launch_merge(const Shape& sh, const MergeParams& p, unsigned nheads, cudaStream_t s);
 template <int VAR>
@@ -112,7 +113,8 @@ size_t merge_smem_bytes(const Shape& sh, int L);
 
 #define DL_DECLARE_VARIANT_LAUNCHERS(VAR)                                                     \
   template <>                                                                                 \
-  cudaError_t launch_step<VAR>(const Shape&, bool, const StepParams&, unsigned, cudaStream_t); \
+  cudaError_t launch_step<VAR>(const Shape&, bool, const StepParams&, const FillParam&, unsigned, \
+                               cudaStream_t);                                                   \
   template <>                                                                                 \
   cudaError_t launch_merge<VAR>(const Shape&, const MergeParams&, unsigned, cudaStream_t);    \
   template <>                                                                                 \
@@ -160,7 +162,8 @@ int persistent_stages(int L) {
 // Persistent launch: one CTA per SM (or per item when there are fewer).
 // Returns cudaErrorNotSupported when its ring would have fewer than 2 stages.
 template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
-cudaError_t launch_step_persistent_t(const StepParams& p, unsigned nheads, cudaStream_t s) {
+cudaError_t launch_step_persistent_t(const StepParams& p, const FillParam& fp, unsigned nheads,
+                                     cudaStream_t s) {
   const int nst = persistent_stages<VAR, DK, DV, ROWS, TIn>(p.L);
   if (nst < 2) return cudaErrorNotSupported;
   static std::atomic<unsigned long long> done{0};
@@ -174,28 +177,29 @@ cudaError_t launch_step_persistent_t(const StepParams& p, unsigned nheads, cudaS
   const unsigned grid = nitems < unsigned(sms) ? nitems : unsigned(sms);
   StepParams q = p;
   q.nitems = int(nitems);
-  kern<<<grid, PGeom<ROWS>::kThreads, smem, s>>>(q, nst);
+  kern<<<grid, PGeom<ROWS>::kThreads, smem, s>>>(q, nst, fp);
   return cudaGetLastError();
 }
 
 template <int VAR, int DK, int DV, int ROWS, typename T, bool FUSED>
-cudaError_t launch_step_rows(bool persistent, const StepParams& p, unsigned n, cudaStream_t s) {
+cudaError_t launch_step_rows(bool persistent, const StepParams& p, const FillParam& fp, unsigned n,
+                             cudaStream_t s) {
   if (persistent) {
-    const cudaError_t e = launch_step_persistent_t<VAR, DK, DV, ROWS, T, FUSED>(p, n, s);
+    const cudaError_t e = launch_step_persistent_t<VAR, DK, DV, ROWS, T, FUSED>(p, fp, n, s);
     if (e != cudaErrorNotSupported) return e;
   }
-  return launch_step_t<VAR, DK, DV, ROWS, T, FUSED>(p, n, s);
+  return launch_step_t<VAR, DK, DV, ROWS, T, FUSED>(p, fp, n, s);
 }
 
 template <int VAR, int DK, int DV, typename T, bool FUSED>
-cudaError_t launch_step_split(int split, bool persistent, const StepParams& p, unsigned n,
-                              cudaStream_t s) {
-  if (split == 1) return launch_step_rows<VAR, DK, DV, DV, T, FUSED>(persistent, p, n, s);
+cudaError_t launch_step_split(int split, bool persistent, const StepParams& p, const FillParam& fp,
+                              unsigned n, cudaStream_t s) {
+  if (split == 1) return launch_step_rows<VAR, DK, DV, DV, T, FUSED>(persistent, p, fp, n, s);
   if constexpr (DV / 2 >= 32) {
-    if (split == 2) return launch_step_rows<VAR, DK, DV, DV / 2, T, FUSED>(persistent, p, n, s);
+    if (split == 2) return launch_step_rows<VAR, DK, DV, DV / 2, T, FUSED>(persistent, p, fp, n, s);
   }
   if constexpr (DV / 4 >= 32) {
-    if (split == 4) return launch_step_rows<VAR, DK, DV, DV / 4, T, FUSED>(persistent, p, n, s);
+    if (split == 4) return launch_step_rows<VAR, DK, DV, DV / 4, T, FUSED>(persistent, p, fp, n, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -203,6 +207,7 @@ cudaError_t launch_step_split(int split, bool persistent, const StepParams& p, u
 template <int VAR>
 struct StepRun {
   const StepParams& p;
+  const FillParam& fp;
   unsigned n;
   cudaStream_t s;
   bool fused;
@@ -210,8 +215,8 @@ struct StepRun {
   bool persistent;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    return fused ? launch_step_split<VAR, DK, DV, T, true>(split, persistent, p, n, s)
-                 : launch_step_split<VAR, DK, DV, T, false>(split, persistent, p, n, s);
+    return fused ? launch_step_split<VAR, DK, DV, T, true>(split, persistent, p, fp, n, s)
+                 : launch_step_split<VAR, DK, DV, T, false>(split, persistent, p, fp, n, s);
   }
 };
 template <int VAR>
@@ -262,8 +267,8 @@ struct MergeSmem {
 #define DL_DEFINE_VARIANT_LAUNCHERS(VAR)                                                   \
   template <>                                                                              \
   cudaError_t launch_step<VAR>(const Shape& sh, bool fused, const StepParams& p,           \
-                               unsigned nheads, cudaStream_t s) {                          \
-    StepRun<VAR> f{p, nheads, s, fused, sh.split, sh.persistent != 0};                                                   \
+                               const FillParam& fp, unsigned nheads, cudaStream_t s) {     \
+    StepRun<VAR> f{p, fp, nheads, s, fused, sh.split, sh.persistent != 0};                                                   \
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
   template <>                                                                              \

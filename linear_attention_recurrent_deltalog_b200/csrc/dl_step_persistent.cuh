@@ -77,7 +77,7 @@ struct PGeom {
 
 template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
 __global__ void __launch_bounds__(PGeom<ROWS>::kThreads, 1)
-dl_step_persistent_kernel(const StepParams p, const int nstage) {
+dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam fp) {
   using Tl = Tile<DK, ROWS>;
   using G = PGeom<ROWS>;
   using TU = typename LogU<VAR, TIn>::type;
@@ -121,7 +121,7 @@ dl_step_persistent_kernel(const StepParams p, const int nstage) {
     float dec_nx = 0.f, beta_nx = 0.f;
     if (w < nitems) {
       const size_t hh = w / SPLIT;
-      f_nx = p.fill_in[hh];
+      f_nx = step_fill(p, fp, hh);
       if (GW == 1) dec_nx = p.decay[hh];
       if (VAR != kVarRWKV6) beta_nx = p.beta[hh];
     }
@@ -149,7 +149,10 @@ dl_step_persistent_kernel(const StepParams p, const int nstage) {
       const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
       mbar_expect_tx(&full[s], tile_b + vec_b + bu * uint32_t(ROWS / kURows) + bk + bg);
       const float* gS = p.base + (head * size_t(DV) + r0) * DK;
-      tma_load_1d_stream(st, gS, tile_b, &full[s]);
+#pragma unroll
+      for (int c = 0; c < Tl::kChunks; ++c)
+        tma_load_1d_stream(st + size_t(c) * Tl::kChunkBytes, gS + size_t(c) * Tl::kChunkRows * DK,
+                           Tl::kChunkBytes, &full[s]);
       tma_load_1d(st + lay.offQ, static_cast<const TIn*>(p.q) + head * DK, DK * sizeof(TIn), &full[s]);
       tma_load_1d(st + lay.offKt, static_cast<const TIn*>(p.k) + head * DK, DK * sizeof(TIn), &full[s]);
       tma_load_1d(st + lay.offV, static_cast<const TIn*>(p.v) + head * DV + r0, ROWS * sizeof(TIn),
@@ -171,7 +174,7 @@ dl_step_persistent_kernel(const StepParams p, const int nstage) {
       const unsigned wn = w + gridDim.x;
       if (wn < nitems) {
         const size_t hn = wn / SPLIT;
-        f_nx = p.fill_in[hn];
+        f_nx = step_fill(p, fp, hn);
         if (GW == 1) dec_nx = p.decay[hn];
         if (VAR != kVarRWKV6) beta_nx = p.beta[hn];
       }
@@ -263,45 +266,8 @@ dl_step_persistent_kernel(const StepParams p, const int nstage) {
       if (part == 0) p.fill_out[head] = merge_now ? 0 : f + 1;
     }
     if (f > 0) {
-      float gl[CPL];
-      float gt0 = 0.f;
-      float kl[CPL], ql[CPL];
-#pragma unroll
-      for (int cc = 0; cc < CPL; ++cc) {
-        const int c = lane * CPL + cc;
-        kl[cc] = to_f(sKr[c]);
-        ql[cc] = to_f(sQr[c]);
-        if (VAR != kVarGDN)
-          gl[cc] = sG[size_t(f - 1) * DK + c] + (VAR == kVarKDA ? logf(sDec[c]) : 0.f);
-      }
-      if (VAR == kVarGDN) gt0 = sG[f - 1] + logf(hdr.decay);
-      for (int i = cw; i < f; i += NCW) {
-        float x = 0.f, y = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < CPL; ++cc) {
-          const int c = lane * CPL + cc;
-          const float ki = to_f(sK[size_t(i) * DK + c]);
-          if (VAR == kVarGDN) {
-            x = fmaf(ki, kl[cc], x);
-            y = fmaf(ki, ql[cc], y);
-          } else {
-            const float kie = ki * expf(gl[cc] - sG[size_t(i) * DK + c]);
-            if (VAR == kVarKDA) x = fmaf(kie, kl[cc], x);
-            y = fmaf(kie, ql[cc], y);
-          }
-        }
-        if (VAR != kVarRWKV6) x = warp_sum(x);
-        y = warp_sum(y);
-        if (VAR == kVarGDN) {
-          const float e = expf(gt0 - sG[i]);
-          x *= e;
-          y *= e;
-        }
-        if (lane == 0) {
-          sW[i] = x;
-          sZ[i] = y;
-        }
-      }
+      const float* dec = (GW == 1) ? &reinterpret_cast<const PHdr*>(st + lay.offHdr)->decay : sDec;
+      entry_weights<VAR, DK, TIn, TIn>(f, cw, NCW, lane, sKr, sQr, sK, sG, dec, sW, sZ);
     }
     if (cw == NCW - 1) {
       float x = 0.f;
@@ -390,9 +356,11 @@ dl_step_persistent_kernel(const StepParams p, const int nstage) {
             k4.w *= expf(sGt[c0 + 3] - gi[3]);
           }
         }
+        float u16[16];
+        load_u16(sU, j0, i, L, u16);
 #pragma unroll
         for (int pi = 0; pi < NV; ++pi) {
-          const float ui = to_f(sU[su_offset(j0 + pi * RPI + rsub, i, L)]);
+          const float ui = (RPI == 1) ? u16[pi] : (rsub ? u16[pi * RPI + 1] : u16[pi * RPI]);
           acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
           acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
           acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
