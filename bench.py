@@ -244,7 +244,7 @@ def run_ours(args, world, rank, local):
     w = wl.WORKLOADS[args.workload]
     w = w.replace(L=args.L or w.L, B=args.B or w.B)
     cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=fused,
-                     step_split=args.split, persistent=not args.nonpersistent)
+                     step_split=args.split, persistent=args.persistent)
     stream = torch.cuda.current_stream(device)
 
     # inputs: a device ring of RING pre-drawn steps (the generator's recipe)
@@ -436,7 +436,7 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": workload_desc(w, args.merge), "name": w.name,
                    "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "L": w.L, "merge": args.merge,
-                   "step_split": args.split, "persistent": not args.nonpersistent,
+                   "step_split": args.split, "persistent": args.persistent,
                    "global_batch": w.B * world,
                    "parallelism": f"replicas x{world} (dp, no collective)",
                    "l2": (f"state {state_mib:.0f} MiB > 126 MB L2 on every step: no flush needed"
@@ -539,8 +539,8 @@ def main():
                     help="synthetic workload (the headline line is gdn_serving)")
     ap.add_argument("--L", type=int, default=0, help="log length (0: the workload's)")
     ap.add_argument("--B", type=int, default=0, help="sequences (0: the workload's)")
-    ap.add_argument("--nonpersistent", action="store_true",
-                    help="use the one-CTA-per-item step kernel instead of the persistent one")
+    ap.add_argument("--persistent", action="store_true",
+                    help="use the persistent warp-specialised step kernel (opt-in)")
     ap.add_argument("--split", type=int, default=0,
                     help="CTAs per head in the step kernel (0 = library default)")
     ap.add_argument("--only-step", action="store_true",

@@ -75,10 +75,11 @@ enum dl_flags {
    * log writes the merged base instead and leaves an empty log, so the log
    * is never full and dl_merge(DL_MERGE_FULL) has nothing to do. */
   DL_FLAG_FUSED_MERGE = 1,
-  /* Use the step kernel that launches one CTA per work item instead of the
-   * persistent warp-specialised one (which is used whenever its ring of
-   * shared-memory stages fits).  A performance choice only. */
-  DL_FLAG_NONPERSISTENT = 2
+  /* Run the step as a persistent warp-specialised kernel (one CTA per SM, a
+   * producer lane streaming work items through a ring of shared-memory
+   * stages) when its ring fits, instead of one CTA per work item.  A
+   * performance choice only; on B200 the default measured faster. */
+  DL_FLAG_PERSISTENT = 2
 };
 
 /* Layer configuration.  d_k, d_v in {64, 128}; 1 <= L <= 64; B, H >= 1 and

@@ -69,7 +69,7 @@ int check_config(const dl_config* c, bool need_L) {
   if (c->B < 1 || c->H < 1 || c->d_k < 1 || c->d_v < 1) return DL_ERR_ARG;
   if (c->in_dtype != DL_F32 && c->in_dtype != DL_BF16) return DL_ERR_ARG;
   if (need_L && (c->L < 1 || c->L > 64)) return DL_ERR_ARG;
-  if (need_L && (c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_NONPERSISTENT)) != 0)
+  if (need_L && (c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_PERSISTENT)) != 0)
     return DL_ERR_ARG;
   const uint64_t bh = uint64_t(c->B) * uint64_t(c->H);
   if (bh > 0x7fffffffull) return DL_ERR_ARG;  // one CTA per head in a 1-D grid
@@ -81,7 +81,7 @@ int check_config(const dl_config* c, bool need_L) {
 
 Shape shape_of(const dl_config& c) {
   return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0, split_of(c),
-               (c.flags & DL_FLAG_NONPERSISTENT) ? 0 : 1};
+               (c.flags & DL_FLAG_PERSISTENT) ? 1 : 0};
 }
 
 cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, const dl::FillParam& fp,

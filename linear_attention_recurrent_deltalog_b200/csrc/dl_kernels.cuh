@@ -215,14 +215,18 @@ template <int VAR, int DK, int DV, int ROWS, typename TIn>
 struct StepLayout {
   using TU = typename LogU<VAR, TIn>::type;
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
-  size_t offU, offK, offG, offVec, offW, offZ, offScal, offBar, total;
+  size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offBar, total;
   __host__ __device__ explicit StepLayout(int L) {
     offU = Tile<DK, ROWS>::kTileBytes;
     offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
     offG = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
-    offVec = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
-    // k, q (raw), k-hat, q-hat, decay [DK] each; v [ROWS]; g_t, g_{t-1} [GW]
-    offW = offVec + align_up(size_t(5 * DK + ROWS + 2 * GW) * 4, 128);
+    offQr = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
+    offKr = offQr + align_up(size_t(DK) * sizeof(TIn), 128);
+    offVr = offKr + align_up(size_t(DK) * sizeof(TIn), 128);
+    offDecV = offVr + align_up(size_t(ROWS) * sizeof(TIn), 128);
+    offVec = offDecV + align_up(size_t(GW) * 4, 128);
+    // fp32 k, q, k-hat, q-hat [DK] each; g_t, g_{t-1} [GW]
+    offW = offVec + align_up(size_t(4 * DK + 2 * GW) * 4, 128);
     offZ = offW + align_up(size_t(L) * 4, 16);
     offScal = offZ + align_up(size_t(L) * 4, 16);
     offBar = offScal + 64;
@@ -244,26 +248,30 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   constexpr int RPI = Tl::kRPI;
   constexpr int CPL = Tl::kCPL;
   static_assert(DV % ROWS == 0, "rows split evenly");
+  static_assert(NW >= 2, "one warp issues the tile copies, another the small ones");
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int L = p.L;
   const int GS = g_stride(VAR, L, DK);
   const StepLayout<VAR, DK, DV, ROWS, TIn> lay(L);
   float* sS = reinterpret_cast<float*>(smem);                 // [ROWS][DK]
-  TU* sU = reinterpret_cast<TU*>(smem + lay.offU);            // [L][ROWS]
+  TU* sU = reinterpret_cast<TU*>(smem + lay.offU);            // [ROWS/32][L][32]
   TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);          // [L][DK]
   float* sG = reinterpret_cast<float*>(smem + lay.offG);      // [L][GW]
-  float* sk = reinterpret_cast<float*>(smem + lay.offVec);    // raw k_t
-  float* sq = sk + DK;                                        // raw q_t / r_t
+  TIn* sQr = reinterpret_cast<TIn*>(smem + lay.offQr);        // q_t (r_t) as given
+  TIn* sKr = reinterpret_cast<TIn*>(smem + lay.offKr);        // k_t as given
+  TIn* sVr = reinterpret_cast<TIn*>(smem + lay.offVr);        // this part's rows of v_t
+  float* sDecV = reinterpret_cast<float*>(smem + lay.offDecV);  // decay_t (vector variants)
+  float* sk = reinterpret_cast<float*>(smem + lay.offVec);    // k_t (fp32)
+  float* sq = sk + DK;                                        // q_t / r_t (fp32)
   float* sKh = sq + DK;                                       // GEMV vector for a
   float* sQh = sKh + DK;                                      // GEMV vector for b
-  float* sDec = sQh + DK;                                     // decay_t
-  float* sV = sDec + DK;                                      // v_t (this part's rows)
-  float* sGt = sV + ROWS;                                     // g_t
+  float* sGt = sQh + DK;                                      // g_t
   float* sGp = sGt + GW;                                      // g_{t-1}
   float* sW = reinterpret_cast<float*>(smem + lay.offW);      // per-entry weights on k
   float* sZ = reinterpret_cast<float*>(smem + lay.offZ);      // per-entry weights on q / r
-  float* sScal = reinterpret_cast<float*>(smem + lay.offScal);
+  float* sScal = reinterpret_cast<float*>(smem + lay.offScal);  // [0] k.q / bonus [1] beta
+                                                                // [2] e^{g_t} [3] decay (GDN)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
   uint64_t* barLog = &bars[Tl::kChunks];
 
@@ -274,15 +282,25 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   const int part = static_cast<int>(blockIdx.x % SPLIT);
   const int r0 = part * ROWS;  // first value row of this CTA
   const int h = static_cast<int>(head % static_cast<size_t>(p.H));
+  const int f = step_fill(p, fp, head);
+  if (f < 0 || f >= L) {  // the host never launches a step on a full log
+    if (tid == 0 && p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
+    return;
+  }
+  const bool merge_now = FUSED && (f + 1 == L);
+  const bool appender = (part == 0) && !merge_now;
 
   const float* gS = p.base + (head * size_t(DV) + r0) * DK;
   TU* gU = static_cast<TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
   TIn* gK = static_cast<TIn*>(p.logK) + head * size_t(L) * DK;
   float* gG = p.logG + head * size_t(GS);
 
-  if (tid == 0) {
+  // Warp 0 streams the tile; warp 1 fetches everything small (the step's
+  // vectors and the f log entries) and the two scalars no bulk copy can
+  // carry.  No other thread touches global memory before the data is in.
+  if (warp == 0 && lane == 0) {
 #pragma unroll
-    for (int c = 0; c <= Tl::kChunks; ++c) mbar_init(&bars[c], 1);
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_init(&bars[c], 1);
     fence_mbar_init();
 #pragma unroll
     for (int c = 0; c < Tl::kChunks; ++c) {
@@ -290,81 +308,73 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
                          Tl::kChunkBytes, &bars[c]);
     }
-  }
-  const int f = step_fill(p, fp, head);
-  if (f < 0 || f >= L) {  // the host never launches a step on a full log
-    if (tid == 0) {
-      if (p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
-      for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
-    }
-    return;
-  }
-  const bool merge_now = FUSED && (f + 1 == L);
-  const bool appender = (part == 0) && !merge_now;
-  if (tid == 0 && f > 0) {
+  } else if (warp == 1 && lane == 0) {
+    const float dec_s = (GW == 1) ? p.decay[head] : 0.f;      // loads in flight while
+    const float beta_s = (VAR == kVarRWKV6) ? 0.f : p.beta[head];  // the copies go out
+    mbar_init(barLog, 1);
+    fence_mbar_init();
+    const uint32_t bq = DK * sizeof(TIn);
+    const uint32_t bv = ROWS * sizeof(TIn);
+    const uint32_t bd = (GW > 1) ? DK * 4u : 0u;
     const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one row block
     const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
-    const uint32_t bg = g_copy_bytes<VAR, DK>(f);
-    mbar_arrive_expect_tx(barLog, bu * uint32_t(ROWS / kURows) + bk + bg);
-    tma_load_1d(sK, gK, bk, barLog);
-    tma_load_1d(sG, gG, bg, barLog);
-    for (int rb = 0; rb < ROWS / kURows; ++rb)
-      tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, r0 + rb * kURows, 0, L, DV), bu,
-                  barLog);
+    const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
+    mbar_arrive_expect_tx(barLog, 2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg);
+    tma_load_1d(sQr, static_cast<const TIn*>(p.q) + head * DK, bq, barLog);
+    tma_load_1d(sKr, static_cast<const TIn*>(p.k) + head * DK, bq, barLog);
+    tma_load_1d(sVr, static_cast<const TIn*>(p.v) + head * DV + r0, bv, barLog);
+    if (GW > 1) tma_load_1d(sDecV, p.decay + head * DK, bd, barLog);
+    if (f > 0) {
+      tma_load_1d(sK, gK, bk, barLog);
+      tma_load_1d(sG, gG, bg, barLog);
+      for (int rb = 0; rb < ROWS / kURows; ++rb)
+        tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, r0 + rb * kURows, 0, L, DV), bu,
+                    barLog);
+    }
+    sScal[1] = beta_s;
+    sScal[3] = dec_s;
+    if (part == 0) p.fill_out[head] = merge_now ? 0 : f + 1;
   }
+  __syncthreads();
 
-  // ---- per-head vectors while the tile and the log stream in
-  const TIn* gq = static_cast<const TIn*>(p.q) + head * DK;
-  const TIn* gk = static_cast<const TIn*>(p.k) + head * DK;
-  const TIn* gv = static_cast<const TIn*>(p.v) + head * DV + r0;
+  // ---- decay bookkeeping, appends of k and g, per-entry weights
+  const bool ok = mbar_wait(barLog, 0, p.err, int(head));
   for (int c = tid; c < DK; c += NT) {
-    const TIn kraw = gk[c];
-    sk[c] = to_f(kraw);
-    sq[c] = to_f(gq[c]);
-    sDec[c] = (GW > 1) ? p.decay[head * DK + c] : 0.f;
+    const TIn kraw = sKr[c];
+    const float kc = to_f(kraw);
+    const float qc = to_f(sQr[c]);
+    sk[c] = kc;
+    sq[c] = qc;
+    if (GW > 1) {
+      const float gp = (f > 0) ? sG[size_t(f - 1) * DK + c] : 0.f;
+      const float gt = gp + logf(sDecV[c]);
+      sGp[c] = gp;
+      sGt[c] = gt;
+      if (VAR == kVarKDA) {
+        const float e = expf(gt);
+        sKh[c] = e * kc;
+        sQh[c] = e * qc;
+      } else {  // RWKV6 reads S_{t-1}: decay up to the previous step
+        sQh[c] = expf(gp) * qc;
+      }
+      if (appender) gG[size_t(f) * DK + c] = gt;
+    }
     if (merge_now)
       sK[size_t(f) * DK + c] = kraw;
     else if (appender)
       gK[size_t(f) * DK + c] = kraw;
   }
-  for (int j = tid; j < ROWS; j += NT) sV[j] = to_f(gv[j]);
-  if (tid == 0) {
-    if (GW == 1) sDec[0] = p.decay[head];
-    sScal[1] = (VAR == kVarRWKV6) ? 0.f : p.beta[head];
-    if (part == 0) p.fill_out[head] = merge_now ? 0 : f + 1;
-  }
-  __syncthreads();
-
-  // ---- log-decay bookkeeping and per-entry weights (needs the log)
-  bool ok = true;
-  if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
-  if (GW == 1) {
-    if (tid == 0) {
-      const float gp = (f > 0) ? sG[f - 1] : 0.f;
-      const float gt = gp + logf(sDec[0]);
-      sGp[0] = gp;
-      sGt[0] = gt;
-      sScal[2] = expf(gt);
-      if (appender) gG[f] = gt;
-    }
-  } else {
-    for (int c = tid; c < DK; c += NT) {
-      const float gp = (f > 0) ? sG[size_t(f - 1) * DK + c] : 0.f;
-      const float gt = gp + logf(sDec[c]);
-      sGp[c] = gp;
-      sGt[c] = gt;
-      if (VAR == kVarKDA) {
-        const float e = expf(gt);
-        sKh[c] = e * sk[c];
-        sQh[c] = e * sq[c];
-      } else {  // RWKV6 reads S_{t-1}: decay up to the previous step
-        sQh[c] = expf(gp) * sq[c];
-      }
-      if (appender) gG[size_t(f) * DK + c] = gt;
-    }
+  if (GW == 1 && tid == NT - 1) {
+    const float gp = (f > 0) ? sG[f - 1] : 0.f;
+    const float gt = gp + logf(sScal[3]);
+    sGp[0] = gp;
+    sGt[0] = gt;
+    sScal[2] = expf(gt);
+    if (appender) gG[f] = gt;
   }
   if (f > 0)
-    entry_weights<VAR, DK, float, TIn>(f, warp, NW, lane, sk, sq, sK, sG, sDec, sW, sZ);
+    entry_weights<VAR, DK, TIn, TIn>(f, warp, NW, lane, sKr, sQr, sK, sG,
+                                     (GW == 1) ? &sScal[3] : sDecV, sW, sZ);
   if (warp == NW - 1) {
     // GDN/KDA: k_t . q_t (the current entry's own weight on q);
     // RWKV6: the bonus sum_c r_c u_c k_c.
@@ -372,14 +382,15 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
 #pragma unroll
     for (int cc = 0; cc < CPL; ++cc) {
       const int c = lane * CPL + cc;
-      x = (VAR == kVarRWKV6) ? fmaf(sq[c] * p.bonus[size_t(h) * DK + c], sk[c], x)
-                             : fmaf(sk[c], sq[c], x);
+      const float kc = to_f(sKr[c]);
+      const float qc = to_f(sQr[c]);
+      x = (VAR == kVarRWKV6) ? fmaf(qc * p.bonus[size_t(h) * DK + c], kc, x) : fmaf(kc, qc, x);
     }
     x = warp_sum(x);
     if (lane == 0) sScal[0] = x;
   }
   if (!__syncthreads_and(ok)) {
-    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
+    mbar_wait(barLog, 0, nullptr, 0);
     for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
     return;
   }
@@ -409,13 +420,27 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   const int jl = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;  // local row
 
   // ---- log correction, delta-rule correction and readout for row r0 + jl
-  float ck = 0.f, cq = 0.f;
-  for (int i = 0; i < f; ++i) {
-    const float uij = to_f(sU[su_offset(jl, i, L)]);
-    if (VAR != kVarRWKV6) ck = fmaf(sW[i], uij, ck);
-    cq = fmaf(sZ[i], uij, cq);
+  // (two partial sums per weight vector for instruction-level parallelism)
+  float ck0 = 0.f, ck1 = 0.f, cq0 = 0.f, cq1 = 0.f;
+  int i = 0;
+  for (; i + 1 < f; i += 2) {
+    const float u0 = to_f(sU[su_offset(jl, i, L)]);
+    const float u1 = to_f(sU[su_offset(jl, i + 1, L)]);
+    if (VAR != kVarRWKV6) {
+      ck0 = fmaf(sW[i], u0, ck0);
+      ck1 = fmaf(sW[i + 1], u1, ck1);
+    }
+    cq0 = fmaf(sZ[i], u0, cq0);
+    cq1 = fmaf(sZ[i + 1], u1, cq1);
   }
-  const float vj = sV[jl];
+  if (i < f) {
+    const float u0 = to_f(sU[su_offset(jl, i, L)]);
+    if (VAR != kVarRWKV6) ck0 = fmaf(sW[i], u0, ck0);
+    cq0 = fmaf(sZ[i], u0, cq0);
+  }
+  const float ck = ck0 + ck1;
+  const float cq = cq0 + cq1;
+  const float vj = to_f(sVr[jl]);
   const float sdot = sScal[0];
   float u, o;
   if (VAR == kVarGDN) {
@@ -452,22 +477,22 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
     acc[pi] = make_float4(s4.x * dec.x, s4.y * dec.y, s4.z * dec.z, s4.w * dec.w);
   }
-  for (int i = 0; i <= f; ++i) {
-    float4 k4 = load4(sK + size_t(i) * DK + c0);
-    if (i < f) {
+  for (int e = 0; e <= f; ++e) {
+    float4 k4 = load4(sK + size_t(e) * DK + c0);
+    if (e < f) {
       if (VAR == kVarGDN) {
-        const float e = expf(sGt[0] - sG[i]);
-        k4.x *= e; k4.y *= e; k4.z *= e; k4.w *= e;
+        const float x = expf(sGt[0] - sG[e]);
+        k4.x *= x; k4.y *= x; k4.z *= x; k4.w *= x;
       } else {
-        const float* gi = sG + size_t(i) * DK + c0;
-        k4.x *= expf(sGt[c0] - gi[0]);
-        k4.y *= expf(sGt[c0 + 1] - gi[1]);
-        k4.z *= expf(sGt[c0 + 2] - gi[2]);
-        k4.w *= expf(sGt[c0 + 3] - gi[3]);
+        const float* ge = sG + size_t(e) * DK + c0;
+        k4.x *= expf(sGt[c0] - ge[0]);
+        k4.y *= expf(sGt[c0 + 1] - ge[1]);
+        k4.z *= expf(sGt[c0 + 2] - ge[2]);
+        k4.w *= expf(sGt[c0 + 3] - ge[3]);
       }
     }
     float u16[16];
-    load_u16(sU, j0, i, L, u16);
+    load_u16(sU, j0, e, L, u16);
 #pragma unroll
     for (int pi = 0; pi < NV; ++pi) {
       const float ui = (RPI == 1) ? u16[pi] : (rsub ? u16[pi * RPI + 1] : u16[pi * RPI]);

@@ -32,7 +32,7 @@ DL_ERR_ARG, DL_ERR_ALIGN, DL_ERR_LOG_FULL = -1, -2, -3
 DL_ERR_CUDA, DL_ERR_UNSUPPORTED, DL_ERR_DEVICE = -4, -5, -6
 DL_MERGE_FULL, DL_MERGE_ALL = 0, 1
 DL_FLAG_FUSED_MERGE = 1
-DL_FLAG_NONPERSISTENT = 2
+DL_FLAG_PERSISTENT = 2
 
 VARIANT_IDS = {"gdn": DL_GDN, "kda": DL_KDA, "rwkv6": DL_RWKV6}
 DTYPE_IDS = {"f32": DL_F32, "bf16": DL_BF16}
@@ -119,11 +119,11 @@ class Config:
     in_dtype: str = "bf16"
     fused_merge: bool = False
     step_split: int = 0
-    persistent: bool = True
+    persistent: bool = False
 
     def c(self) -> dl_config:
         flags = (DL_FLAG_FUSED_MERGE if self.fused_merge else 0) | \
-            (0 if self.persistent else DL_FLAG_NONPERSISTENT)
+            (DL_FLAG_PERSISTENT if self.persistent else 0)
         return dl_config(VARIANT_IDS[self.variant], self.B, self.H, self.d_k, self.d_v, self.L,
                          DTYPE_IDS[self.in_dtype], flags, self.step_split)
 

@@ -79,7 +79,7 @@ def _rel(a: np.ndarray, ref: np.ndarray) -> float:
 def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence[int]] = None,
                arms=("log", "fused", "eager"), snap_every: int = 64, L: Optional[int] = None,
                merge_all_at: Sequence[int] = (), workers: Optional[int] = None,
-               split: int = 0, persistent: bool = True, device="cuda") -> Dict[str, ArmResult]:
+               split: int = 0, persistent: bool = False, device="cuda") -> Dict[str, ArmResult]:
     """Runs the given arms and the oracle; returns per-arm errors."""
     if L is not None:
         w = w.replace(L=L)

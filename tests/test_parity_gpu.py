@@ -86,9 +86,9 @@ def test_step_split(name, split, persistent):
 
 
 @pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
-def test_nonpersistent_full_workload(name):
+def test_persistent_full_workload(name):
     w = wl.WORKLOADS[name]
-    res = run_parity(w, T=64, heads=wl.sample_heads(w, 24), persistent=False, arms=("fused",))
+    res = run_parity(w, T=64, heads=wl.sample_heads(w, 24), persistent=True, arms=("fused",))
     _check(res)
 
 
