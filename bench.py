@@ -219,6 +219,69 @@ def eager_bytes(cfg) -> tuple:
 
 # ------------------------------------------------------------ our arm
 
+def log_entry_bytes(cfg) -> int:
+    ein = 2 if cfg.in_dtype == "bf16" else 4
+    uin = ein if cfg.variant == "rwkv6" else 4
+    gw = 1 if cfg.variant == "gdn" else cfg.d_k
+    return cfg.d_v * uin + cfg.d_k * ein + gw * 4
+
+
+def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, reps: int = 3):
+    """Times dl_merge (every log full, all heads) and dl_materialize (logs
+    half full) with CUDA events; algorithmic bytes per head: merge reads the
+    tile and L entries and writes the tile; materialize reads the tile and f
+    entries and writes the dense state to a separate buffer."""
+    import dataclasses as dc
+
+    from linear_attention_recurrent_deltalog_b200 import deltalog as dlb
+    cm = dc.replace(cfg, fused_merge=False)
+    st = dlb.DeltaLogState(cm, device=device)
+    o = torch.empty(w.heads * w.d_v, dtype=torch.float32, device=device)
+    tile = w.d_v * w.d_k * 4
+    entry = log_entry_bytes(cm)
+    ms_merge = []
+    for r in range(reps):
+        st.reset(S0, [0] * w.B)
+        for i in range(w.L):
+            q, k, v, dec, beta = ring[i % len(ring)]
+            st.step(q, k, v, dec, beta, bonus, o)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        st.merge(dlb.DL_MERGE_FULL)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ms_merge.append(a.elapsed_time(b))
+    mb = w.heads * (2 * tile + w.L * entry + 8)
+    t_merge = sorted(ms_merge)[len(ms_merge) // 2] / 1e3
+    st.reset(S0, [0] * w.B)
+    half = w.L // 2
+    for i in range(half):
+        q, k, v, dec, beta = ring[i % len(ring)]
+        st.step(q, k, v, dec, beta, bonus, o)
+    out = torch.empty(w.heads * w.d_v * w.d_k, dtype=torch.float32, device=device)
+    st.materialize(out)
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        st.materialize(out)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    t_mat = a.elapsed_time(b) / reps / 1e3
+    mtb = w.heads * (2 * tile + half * entry + 4)
+    code, head = st.device_error()
+    st.close()
+    del out
+    if code != 0:
+        raise RuntimeError(f"device error {code} at head {head}")
+    return ({"launch_ms": round(t_merge * 1e3, 4), "achieved_gbs": round(mb / t_merge / 1e9, 1),
+             "frac": round(mb / t_merge / 1e9 / peak, 4), "heads": w.heads, "entries": w.L,
+             "algorithmic_bytes": int(mb)},
+            {"launch_ms": round(t_mat * 1e3, 4), "achieved_gbs": round(mtb / t_mat / 1e9, 1),
+             "frac": round(mtb / t_mat / 1e9 / peak, 4), "heads": w.heads, "entries": half,
+             "algorithmic_bytes": int(mtb)})
+
+
 def workload_desc(w, merge: str) -> str:
     return (f"{w.variant.upper()} decode B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v} fp32 state, "
             f"{w.in_dtype} q/k/v, {'ragged fills, ' if w.ragged else ''}L={w.L}, merge={merge}")
@@ -351,6 +414,10 @@ def run_ours(args, world, rank, local):
     erd, ewr = eager_bytes(cfg)
     del S_e
 
+    # The merge and materialize kernels on their own: a state whose sequences
+    # all sit at the same phase, so that after L steps every log is full.
+    merge_k, mat_k = measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak)
+
     # End to end through the public API: every step copies its inputs from
     # pinned host memory and its output o back to pinned host memory.  The
     # copies and the kernel run on three streams so step i's compute overlaps
@@ -455,6 +522,8 @@ def run_ours(args, world, rank, local):
         "write_bytes_per_token": {"deltalog": round((wr + mwr) / args.steps / w.B, 1),
                                   "eager": round(ewr / w.B, 1),
                                   "reduction": round(ewr / ((wr + mwr) / args.steps), 3)},
+        "merge_kernel": merge_k,
+        "materialize_kernel": mat_k,
         "eager": {"value": round(aggregate_value(tokens, 1, eager_s), 1), "unit": UNIT,
                   "achieved_gbs": round((erd + ewr) / (eager_s / args.steps) / 1e9, 1),
                   "frac": round((erd + ewr) / (eager_s / args.steps) / 1e9 / peak, 4),

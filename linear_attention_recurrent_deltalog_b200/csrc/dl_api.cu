@@ -95,12 +95,13 @@ cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, const dl::F
   }
 }
 
-cudaError_t launch_merge(const dl_config& c, const dl::MergeParams& p, cudaStream_t s) {
-  const unsigned n = unsigned(size_t(c.B) * c.H);
+// `nctas`: B*H, or (with p.use_list) the listed sequences times H.
+cudaError_t launch_merge(const dl_config& c, const dl::MergeParams& p, const dl::SeqList& list,
+                         unsigned nctas, cudaStream_t s) {
   switch (c.variant) {
-    case DL_GDN: return dl::launch_merge<dl::kVarGDN>(shape_of(c), p, n, s);
-    case DL_KDA: return dl::launch_merge<dl::kVarKDA>(shape_of(c), p, n, s);
-    default: return dl::launch_merge<dl::kVarRWKV6>(shape_of(c), p, n, s);
+    case DL_GDN: return dl::launch_merge<dl::kVarGDN>(shape_of(c), p, list, nctas, s);
+    case DL_KDA: return dl::launch_merge<dl::kVarKDA>(shape_of(c), p, list, nctas, s);
+    default: return dl::launch_merge<dl::kVarRWKV6>(shape_of(c), p, list, nctas, s);
   }
 }
 
@@ -152,6 +153,7 @@ struct dl_state {
   int n_nonempty;                   // sequences whose log holds >= 1 entry
   int parity;                       // which fill array holds the current counts
   dl::FillParam fill_param;         // the mirror as a launch argument (B <= kParamFills)
+  dl::SeqList merge_list;           // sequences a merge launch covers
 
   int* dev_fill(int which) const {
     return reinterpret_cast<int*>(meta + size_t(which) * lay.fill_bytes);
@@ -309,7 +311,22 @@ int dl_merge(dl_state* st, int mode, void* stream) {
   p.out = st->base;
   p.L = c.L;
   p.mode = mode;
-  if (launch_merge(c, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
+  p.H = c.H;
+  // The qualifying sequences, from the host mirror.
+  const int nlist = (mode == DL_MERGE_FULL) ? st->n_full : st->n_nonempty;
+  unsigned nctas = unsigned(size_t(c.B) * c.H);
+  p.use_list = (nlist <= dl::kListSeqs && c.B <= 65536) ? 1 : 0;
+  if (p.use_list) {
+    int n = 0;
+    for (int b = 0; b < c.B; ++b)
+      if (mode == DL_MERGE_ALL ? st->fill[b] > 0 : st->fill[b] == c.L) {
+        st->merge_list.seq[n] = static_cast<uint16_t>(b);
+        st->merge_list.f[n++] = static_cast<uint8_t>(st->fill[b]);
+      }
+    nctas = unsigned(n) * unsigned(c.H);
+  }
+  if (launch_merge(c, p, st->merge_list, nctas, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DL_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   for (int32_t& f : st->fill)
     if (mode == DL_MERGE_ALL || f == c.L) f = 0;
@@ -332,7 +349,11 @@ int dl_materialize(const dl_state* st, float* S_out, void* stream) {
   p.out = S_out;
   p.L = c.L;
   p.mode = 2;
-  if (launch_merge(c, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
+  p.H = c.H;
+  p.use_list = 0;
+  if (launch_merge(c, p, st->merge_list, unsigned(size_t(c.B) * c.H),
+                   static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DL_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DL_OK;
 }

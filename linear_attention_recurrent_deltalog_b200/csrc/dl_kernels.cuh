@@ -63,6 +63,15 @@ __device__ __forceinline__ int step_fill(const StepParams& p, const FillParam& f
   return p.fills_in_param ? int(fp.f[head / size_t(p.H)]) : p.fill_in[head];
 }
 
+// Sequences a merge launch covers, passed by value (the host mirror knows
+// exactly which logs qualify), so the grid is just their heads instead of
+// one CTA per head that mostly exits at once.
+constexpr int kListSeqs = 4096;
+struct SeqList {
+  uint16_t seq[kListSeqs];
+  uint8_t f[kListSeqs];  // log entries of each listed sequence (from the host mirror)
+};
+
 struct MergeParams {
   float* base;
   const void* logU;
@@ -73,6 +82,8 @@ struct MergeParams {
   float* out;    // merge: == base; materialize: caller buffer
   int L;
   int mode;      // 0 merge full logs, 1 merge every non-empty log, 2 materialize
+  int H;
+  int use_list;  // 1: CTA i merges head (list.seq[i / H], i % H)
 };
 
 struct EagerParams {
@@ -510,28 +521,33 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
 
 // ----------------------------------------------------------- merge / materialize
 
-template <int VAR, int DK, int DV, typename TIn>
+template <int VAR, int DK, int DV, int ROWS, typename TIn>
 struct MergeLayout {
   using TU = typename LogU<VAR, TIn>::type;
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
   size_t offU, offK, offKt, offG, offDec, offBar, total;
   __host__ __device__ explicit MergeLayout(int L) {
-    offU = Tile<DK, DV>::kTileBytes;
-    offK = offU + align_up(size_t(L) * DV * sizeof(TU), 128);
+    offU = Tile<DK, ROWS>::kTileBytes;
+    offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
     offKt = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
     offG = offKt + align_up(size_t(L) * DK * 4, 128);
     offDec = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
     offBar = offDec + align_up(size_t(DK) * 4, 128);
-    total = offBar + 8 * (Tile<DK, DV>::kChunks + 1);
+    total = offBar + 8 * (Tile<DK, ROWS>::kChunks + 1);
   }
 };
 
-template <int VAR, int DK, int DV, typename TIn>
-__global__ void __launch_bounds__(Tile<DK, DV>::kThreads)
-dl_merge_kernel(const MergeParams p) {
-  using Tl = Tile<DK, DV>;
+// One CTA per ROWS rows of a head (a head's rows may be split over
+// DV / ROWS CTAs, as in the step).  With a list, the fills come from the
+// list and only part 0 empties the log, so split CTAs never race on it;
+// without a list the kernel runs unsplit and reads the device fill.
+template <int VAR, int DK, int DV, int ROWS, typename TIn>
+__global__ void __launch_bounds__(Tile<DK, ROWS>::kThreads)
+dl_merge_kernel(const MergeParams p, const SeqList list) {
+  using Tl = Tile<DK, ROWS>;
   using TU = typename LogU<VAR, TIn>::type;
-  constexpr int GW = MergeLayout<VAR, DK, DV, TIn>::GW;
+  constexpr int SPLIT = DV / ROWS;
+  constexpr int GW = MergeLayout<VAR, DK, DV, ROWS, TIn>::GW;
   constexpr int NT = Tl::kThreads;
   constexpr int NV = Tl::kNV;
   constexpr int LPR = Tl::kLPR;
@@ -540,8 +556,13 @@ dl_merge_kernel(const MergeParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int L = p.L;
   const int GS = g_stride(VAR, L, DK);
-  const size_t head = blockIdx.x;
-  const int f = p.fill[head];
+  const unsigned item = blockIdx.x / SPLIT;
+  const int part = int(blockIdx.x % SPLIT);
+  const int r0 = part * ROWS;
+  const unsigned li = item / unsigned(p.H);
+  const size_t head = p.use_list ? size_t(list.seq[li]) * size_t(p.H) + item % unsigned(p.H)
+                                 : size_t(item);
+  const int f = p.use_list ? int(list.f[li]) : p.fill[head];
   if (f < 0 || f > L) {
     if (threadIdx.x == 0 && p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0)
       p.err[1] = int(head);
@@ -550,7 +571,7 @@ dl_merge_kernel(const MergeParams p) {
   if (p.mode == 0 && f != L) return;
   if (p.mode == 1 && f == 0) return;
 
-  const MergeLayout<VAR, DK, DV, TIn> lay(L);
+  const MergeLayout<VAR, DK, DV, ROWS, TIn> lay(L);
   float* sS = reinterpret_cast<float*>(smem);
   TU* sU = reinterpret_cast<TU*>(smem + lay.offU);
   TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);
@@ -563,14 +584,15 @@ dl_merge_kernel(const MergeParams p) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const float* gS = p.base + head * size_t(DV) * DK;
-  const TU* gU = static_cast<const TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
+  const float* gS = p.base + (head * size_t(DV) + r0) * DK;
+  const TU* gU = static_cast<const TU*>(p.logU) + u_offset(head, r0, 0, L, DV);
   const TIn* gK = static_cast<const TIn*>(p.logK) + head * size_t(L) * DK;
   const float* gG = p.logG + head * size_t(GS);
 
-  if (tid == 0) {
+  // warp 0 streams the tile, warp 1 the f log entries
+  if (warp == 0 && lane == 0) {
 #pragma unroll
-    for (int c = 0; c <= Tl::kChunks; ++c) mbar_init(&bars[c], 1);
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_init(&bars[c], 1);
     fence_mbar_init();
 #pragma unroll
     for (int c = 0; c < Tl::kChunks; ++c) {
@@ -578,12 +600,15 @@ dl_merge_kernel(const MergeParams p) {
       tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
                          Tl::kChunkBytes, &bars[c]);
     }
+  } else if (warp == 1 && lane == 0) {
+    mbar_init(barLog, 1);
+    fence_mbar_init();
     if (f > 0) {
       const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one row block
       const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
       const uint32_t bg = g_copy_bytes<VAR, DK>(f);
-      mbar_arrive_expect_tx(barLog, bu * uint32_t(DV / kURows) + bk + bg);
-      for (int rb = 0; rb < DV / kURows; ++rb)
+      mbar_arrive_expect_tx(barLog, bu * uint32_t(ROWS / kURows) + bk + bg);
+      for (int rb = 0; rb < ROWS / kURows; ++rb)
         tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, rb * kURows, 0, L, DV), bu, barLog);
       tma_load_1d(sK, gK, bk, barLog);
       tma_load_1d(sG, gG, bg, barLog);
@@ -592,14 +617,17 @@ dl_merge_kernel(const MergeParams p) {
   __syncthreads();
   bool ok = true;
   if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
-  // decay of the base and decayed keys k-tilde_i = k_i o e^{g_last - g_i}
-  for (int c = tid; c < DK; c += NT) {
-    const float gl = (f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f;
-    sDec[c] = expf(gl);
-    for (int i = 0; i < f; ++i)
-      sKt[size_t(i) * DK + c] = to_f(sK[size_t(i) * DK + c]) * expf(gl - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
+  // decay of the base and decayed keys k-tilde_i = k_i o e^{g_last - g_i},
+  // one (entry, channel) pair per thread
+  for (int c = tid; c < DK; c += NT)
+    sDec[c] = expf((f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f);
+  for (int x = tid; x < f * DK; x += NT) {
+    const int i = x / DK;
+    const int c = x % DK;
+    const float gl = sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)];
+    sKt[x] = to_f(sK[x]) * expf(gl - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
   }
-  if (tid == 0 && p.mode != 2) p.fill[head] = 0;
+  if (tid == 0 && part == 0 && p.mode != 2) p.fill[head] = 0;
   if (!__syncthreads_and(ok)) {
     if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
     for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
@@ -634,7 +662,7 @@ dl_merge_kernel(const MergeParams p) {
       acc[pi].w = fmaf(ui, k4.w, acc[pi].w);
     }
   }
-  float* gO = p.out + head * size_t(DV) * DK;
+  float* gO = p.out + (head * size_t(DV) + r0) * DK;
 #pragma unroll
   for (int pi = 0; pi < NV; ++pi)
     *reinterpret_cast<float4*>(gO + size_t(j0 + pi * RPI + rsub) * DK + c0) = acc[pi];
@@ -696,10 +724,12 @@ dl_eager_kernel(const EagerParams p) {
                          Tl::kChunkBytes, &bars[c]);
     }
   }
+  // warp 0 issues the tile copies; the other warps load the step's vectors
   const TIn* gq = static_cast<const TIn*>(p.q) + head * DK;
   const TIn* gk = static_cast<const TIn*>(p.k) + head * DK;
   const TIn* gv = static_cast<const TIn*>(p.v) + head * DV;
-  for (int c = tid; c < DK; c += NT) {
+  for (int c = tid - 32; c < DK; c += NT - 32) {
+    if (c < 0) break;
     const float kc = to_f(gk[c]);
     const float qc = to_f(gq[c]);
     const float dc = (VAR == kVarGDN) ? p.decay[head] : p.decay[head * DK + c];
@@ -714,7 +744,10 @@ dl_eager_kernel(const EagerParams p) {
       sQh[c] = qc;
     }
   }
-  for (int j = tid; j < DV; j += NT) sV[j] = to_f(gv[j]);
+  for (int j = tid - 32; j < DV; j += NT - 32) {
+    if (j < 0) break;
+    sV[j] = to_f(gv[j]);
+  }
   __syncthreads();
   if (warp == NW - 1) {
     float x = 0.f;

@@ -59,15 +59,27 @@ cudaError_t launch_step_t(const StepParams& p, const FillParam& fp, unsigned nhe
   return cudaGetLastError();
 }
 
-template <int VAR, int DK, int DV, typename TIn>
-cudaError_t launch_merge_t(const MergeParams& p, unsigned nheads, cudaStream_t s) {
+template <int VAR, int DK, int DV, int ROWS, typename TIn>
+cudaError_t launch_merge_rows(const MergeParams& p, const SeqList& list, unsigned nheads,
+                              cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
-  auto kern = dl_merge_kernel<VAR, DK, DV, TIn>;
+  auto kern = dl_merge_kernel<VAR, DK, DV, ROWS, TIn>;
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
-  const size_t smem = MergeLayout<VAR, DK, DV, TIn>(p.L).total;
-  kern<<<nheads, Tile<DK, DV>::kThreads, smem, s>>>(p);
+  const size_t smem = MergeLayout<VAR, DK, DV, ROWS, TIn>(p.L).total;
+  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p, list);
   return cudaGetLastError();
+}
+
+// Split heads into 64-row CTAs whenever no CTA has to read a fill another
+// CTA of the launch may reset (a listed merge, or materialize).
+template <int VAR, int DK, int DV, typename TIn>
+cudaError_t launch_merge_t(const MergeParams& p, const SeqList& list, unsigned nheads,
+                           cudaStream_t s) {
+  if constexpr (DV >= 128) {
+    if (p.use_list || p.mode == 2) return launch_merge_rows<VAR, DK, DV, DV / 2, TIn>(p, list, nheads, s);
+  }
+  return launch_merge_rows<VAR, DK, DV, DV, TIn>(p, list, nheads, s);
 }
 
 template <int VAR, int DK, int DV, typename TIn>
@@ -101,7 +113,8 @@ template <int VAR>
 cudaError_t launch_step(const Shape& sh, bool fused, const StepParams& p, const FillParam& fp,
                         unsigned nheads, cudaStream_t s);
 template <int VAR>
-cudaError_t launch_merge(const Shape& sh, const MergeParams& p, unsigned nheads, cudaStream_t s);
+cudaError_t launch_merge(const Shape& sh, const MergeParams& p, const SeqList& list,
+                         unsigned nheads, cudaStream_t s);
 template <int VAR>
 cudaError_t launch_eager(const Shape& sh, const EagerParams& p, unsigned nheads, cudaStream_t s);
 
@@ -116,7 +129,8 @@ size_t merge_smem_bytes(const Shape& sh, int L);
   cudaError_t launch_step<VAR>(const Shape&, bool, const StepParams&, const FillParam&, unsigned, \
                                cudaStream_t);                                                   \
   template <>                                                                                 \
-  cudaError_t launch_merge<VAR>(const Shape&, const MergeParams&, unsigned, cudaStream_t);    \
+  cudaError_t launch_merge<VAR>(const Shape&, const MergeParams&, const SeqList&, unsigned,    \
+                                cudaStream_t);                                                \
   template <>                                                                                 \
   cudaError_t launch_eager<VAR>(const Shape&, const EagerParams&, unsigned, cudaStream_t);    \
   template <>                                                                                 \
@@ -222,10 +236,11 @@ struct StepRun {
 template <int VAR>
 struct MergeRun {
   const MergeParams& p;
+  const SeqList& list;
   unsigned n;
   cudaStream_t s;
   template <int DK, int DV, typename T>
-  cudaError_t run() { return launch_merge_t<VAR, DK, DV, T>(p, n, s); }
+  cudaError_t run() { return launch_merge_t<VAR, DK, DV, T>(p, list, n, s); }
 };
 template <int VAR>
 struct EagerRun {
@@ -259,7 +274,7 @@ struct MergeSmem {
   size_t out;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    out = MergeLayout<VAR, DK, DV, T>(L).total;
+    out = MergeLayout<VAR, DK, DV, DV, T>(L).total;
     return cudaSuccess;
   }
 };
@@ -272,9 +287,9 @@ struct MergeSmem {
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
   template <>                                                                              \
-  cudaError_t launch_merge<VAR>(const Shape& sh, const MergeParams& p, unsigned nheads,    \
-                                cudaStream_t s) {                                          \
-    MergeRun<VAR> f{p, nheads, s};                                                         \
+  cudaError_t launch_merge<VAR>(const Shape& sh, const MergeParams& p, const SeqList& list, \
+                                unsigned nheads, cudaStream_t s) {                         \
+    MergeRun<VAR> f{p, list, nheads, s};                                                   \
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
   template <>                                                                              \

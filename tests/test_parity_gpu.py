@@ -109,3 +109,15 @@ def test_forced_merges_mid_log():
     _check(res)
     w = wl.WORKLOADS["rwkv6"].replace(B=4, H=3, L=16, T=40, ragged=True)
     _check(run_parity(w, snap_every=5, merge_all_at=(1, 17), workers=0, arms=("log", "fused")))
+
+
+@pytest.mark.parametrize("B", [4200, 16400])
+def test_large_batch_fallbacks(B):
+    # More than 4096 sequences merging at once: the merge reads the device fills
+    # (unsplit launch); more than 16384 sequences: the step reads the device
+    # fills instead of the launch argument.
+    w = wl.WORKLOADS["gdn_qwen"].replace(B=B, H=1, d_k=64, d_v=64, L=2, T=5, ragged=False)
+    _check(run_parity(w, heads=wl.sample_heads(w, 32), snap_every=2, workers=0))
+    w = wl.WORKLOADS["kda"].replace(B=B, H=1, d_k=64, d_v=128, L=3, T=7, ragged=True)
+    _check(run_parity(w, heads=wl.sample_heads(w, 32), snap_every=3, workers=0,
+                      arms=("log", "fused")))
