@@ -18,5 +18,5 @@ invariants and an exact-arithmetic brute force of the log form (see
 """
 
 from .recurrence import (  # noqa: F401
-    gdn_step, kda_step, rwkv6_step, run_eager, EagerResult,
+    gdn_step, kda_step, rwkv6_step, kla_beta, run_eager, EagerResult,
 )

@@ -28,6 +28,12 @@ recurrence exactly as written, forming the matrices the formula names
   library stores the transpose), w_t a d_k vector, u a fixed d_k vector per
   head.  The readout uses the state before the update.
 
+* KLA (Kaczmarz step size; "Kaczmarz Linear Attention" abstract): the GDN
+  (or KDA) recurrence with beta_t formed from a gate eta_t and the key norm,
+      beta_t = eta_t / (|k_t|_2^2 + eps),
+  so the write is a Kaczmarz projection: with alpha_t = 1 and eta_t = 1,
+  eps = 0, the updated state maps k_t exactly to v_t whatever |k_t| is.
+
 Outputs are float64.  Inputs are widened exactly from whatever the kernel
 received (fp32 or bf16 values), so input rounding is not counted as error.
 """
@@ -97,6 +103,15 @@ def rwkv6_step(S, r, k, v, w, u):
     return S_new, o
 
 
+def kla_beta(eta, k, eps):
+    """KLA step size beta_t = eta_t / (|k_t|_2^2 + eps) for N heads.
+
+    eta [N]; k [N, d_k]; eps a scalar.
+    """
+    eta, k = _f64(eta), _f64(k)
+    return eta / (np.sum(k * k, axis=-1) + float(eps))
+
+
 @dataclasses.dataclass
 class EagerResult:
     S: np.ndarray                 # final state, float64, recurrence orientation
@@ -112,7 +127,8 @@ def _select(x, heads):
 
 
 def run_eager(variant: str, S0, steps: Iterable, heads: Optional[Sequence[int]] = None,
-              bonus=None, snapshot_at: Sequence[int] = ()) -> EagerResult:
+              bonus=None, snapshot_at: Sequence[int] = (), kla_eps: Optional[float] = None
+              ) -> EagerResult:
     """Run the eager recurrence over ``steps``.
 
     ``S0``: float array [N, ...] in the recurrence's orientation for the
@@ -120,7 +136,9 @@ def run_eager(variant: str, S0, steps: Iterable, heads: Optional[Sequence[int]] 
     decay and beta, each shaped [B, H, ...]; ``heads`` picks N flat
     (b*H + h) heads from them (all heads when None).  ``bonus``: RWKV6 u per
     selected head [N, d_k].  ``snapshot_at``: 1-based step counts after which
-    a copy of the state is kept.
+    a copy of the state is kept.  ``kla_eps`` (GDN/KDA): when given, each
+    step's beta field holds the KLA gate eta_t and beta_t = kla_beta(eta_t,
+    k_t, kla_eps).
     """
     S = _f64(S0).copy()
     outs: List[np.ndarray] = []
@@ -131,10 +149,13 @@ def run_eager(variant: str, S0, steps: Iterable, heads: Optional[Sequence[int]] 
         k = _select(st.k, heads)
         v = _select(st.v, heads)
         dec = _select(st.decay, heads)
+        beta = None if st.beta is None else _select(st.beta, heads)
+        if kla_eps is not None and variant in ("gdn", "kda"):
+            beta = kla_beta(beta, k, kla_eps)
         if variant == "gdn":
-            S, o = gdn_step(S, q, k, v, dec, _select(st.beta, heads))
+            S, o = gdn_step(S, q, k, v, dec, beta)
         elif variant == "kda":
-            S, o = kda_step(S, q, k, v, dec, _select(st.beta, heads))
+            S, o = kda_step(S, q, k, v, dec, beta)
         elif variant == "rwkv6":
             S, o = rwkv6_step(S, q, k, v, dec, bonus)
         else:

@@ -321,3 +321,54 @@ def test_run_eager_matches_stepwise():
         if n == 2:
             np.testing.assert_array_equal(res.states[2], S)
     np.testing.assert_array_equal(res.S, S)
+
+
+# ------------------------------------------------------------- KLA step size
+
+def test_kla_beta_hand_example():
+    # k = (1, 2): |k|^2 = 5, so beta = eta / (5 + eps); eta = 1/2, eps = 1/4
+    # gives beta = (1/2) / (21/4) = 2/21.
+    b = rec.kla_beta(np.array([0.5]), np.array([[1.0, 2.0]]), 0.25)
+    assert b[0] == pytest.approx(2.0 / 21.0, rel=1e-15)
+
+
+def test_kla_write_is_a_kaczmarz_projection():
+    # alpha = 1, eta = 1, eps = 0: beta |k|^2 = 1, so after each write the
+    # state maps k_t exactly to v_t whatever the key's norm (GDN and KDA).
+    rng = np.random.default_rng(21)
+    N, d = 3, 8
+    for which in ("gdn", "kda"):
+        S = rng.standard_normal((N, d, d))
+        for _ in range(6):
+            k = rng.standard_normal((N, d)) * rng.uniform(0.2, 3.0, (N, 1))
+            v = rng.standard_normal((N, d))
+            beta = rec.kla_beta(np.ones(N), k, 0.0)
+            if which == "gdn":
+                S, _ = rec.gdn_step(S, rng.standard_normal((N, d)), k, v, np.ones(N), beta)
+            else:
+                S, _ = rec.kda_step(S, rng.standard_normal((N, d)), k, v, np.ones((N, d)), beta)
+            np.testing.assert_allclose(np.einsum("nij,nj->ni", S, k), v, rtol=1e-11, atol=1e-11)
+
+
+def test_run_eager_kla_uses_key_norms():
+    rng = np.random.default_rng(22)
+    B, H, d, T = 1, 2, 4, 3
+
+    class St:
+        pass
+
+    steps = []
+    for _ in range(T):
+        s = St()
+        s.q, s.k = rng.standard_normal((B, H, d)), rng.standard_normal((B, H, d))
+        s.v = rng.standard_normal((B, H, d))
+        s.decay, s.beta = rng.uniform(0.8, 1, (B, H)), rng.uniform(0, 1, (B, H))
+        steps.append(s)
+    S0 = rng.standard_normal((B * H, d, d))
+    res = oracle.run_eager("gdn", S0, steps, kla_eps=1e-3)
+    S = S0
+    for s in steps:
+        k = s.k.reshape(-1, d)
+        beta = s.beta.reshape(-1) / (np.sum(k * k, axis=1) + 1e-3)
+        S, o = rec.gdn_step(S, s.q.reshape(-1, d), k, s.v.reshape(-1, d), s.decay.reshape(-1), beta)
+    np.testing.assert_allclose(res.S, S, rtol=1e-13, atol=1e-13)
