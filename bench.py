@@ -283,8 +283,9 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
 
 
 def workload_desc(w, merge: str) -> str:
+    kla = f", KLA step size eps={w.kla_eps:g}" if w.kla_eps is not None else ""
     return (f"{w.variant.upper()} decode B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v} fp32 state, "
-            f"{w.in_dtype} q/k/v, {'ragged fills, ' if w.ragged else ''}L={w.L}, merge={merge}")
+            f"{w.in_dtype} q/k/v, {'ragged fills, ' if w.ragged else ''}L={w.L}, merge={merge}{kla}")
 
 
 def to_dev(s, device):
@@ -305,9 +306,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(device)
     fused = args.merge == "fused"
     w = wl.WORKLOADS[args.workload]
-    w = w.replace(L=args.L or w.L, B=args.B or w.B)
+    w = w.replace(L=args.L or w.L, B=args.B or w.B,
+                  kla_eps=args.kla_eps if args.kla_eps >= 0 else None)
     cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=fused,
-                     step_split=args.split, persistent=args.persistent)
+                     step_split=args.split, persistent=args.persistent, kla_eps=w.kla_eps)
     stream = torch.cuda.current_stream(device)
 
     # inputs: a device ring of RING pre-drawn steps (the generator's recipe)
@@ -608,6 +610,8 @@ def main():
                     help="synthetic workload (the headline line is gdn_serving)")
     ap.add_argument("--L", type=int, default=0, help="log length (0: the workload's)")
     ap.add_argument("--B", type=int, default=0, help="sequences (0: the workload's)")
+    ap.add_argument("--kla-eps", type=float, default=-1.0,
+                    help=">= 0: KLA step size beta = eta / (|k|^2 + eps) (GDN/KDA)")
     ap.add_argument("--persistent", action="store_true",
                     help="use the persistent warp-specialised step kernel (opt-in)")
     ap.add_argument("--split", type=int, default=0,

@@ -79,7 +79,12 @@ enum dl_flags {
    * producer lane streaming work items through a ring of shared-memory
    * stages) when its ring fits, instead of one CTA per work item.  A
    * performance choice only; on B200 the default measured faster. */
-  DL_FLAG_PERSISTENT = 2
+  DL_FLAG_PERSISTENT = 2,
+  /* Kaczmarz step size (KLA, GDN and KDA only): the `beta` argument of a
+   * step carries the gate eta_t and the kernels use
+   * beta_t = eta_t / (|k_t|_2^2 + kla_eps) ("Kaczmarz Linear Attention"
+   * abstract), so the write projects exactly whatever the key's norm. */
+  DL_FLAG_KLA = 4
 };
 
 /* Layer configuration.  d_k, d_v in {64, 128}; 1 <= L <= 64; B, H >= 1 and
@@ -98,6 +103,7 @@ typedef struct dl_config {
   int32_t in_dtype;   /* enum dl_dtype of q/r, k, v */
   int32_t flags;      /* enum dl_flags */
   int32_t step_split; /* 0 (default), 1, 2 or 4 */
+  float kla_eps;      /* epsilon of the KLA step size (DL_FLAG_KLA), >= 0 */
 } dl_config;
 
 typedef struct dl_state dl_state;

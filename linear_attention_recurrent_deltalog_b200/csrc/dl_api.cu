@@ -69,7 +69,9 @@ int check_config(const dl_config* c, bool need_L) {
   if (c->B < 1 || c->H < 1 || c->d_k < 1 || c->d_v < 1) return DL_ERR_ARG;
   if (c->in_dtype != DL_F32 && c->in_dtype != DL_BF16) return DL_ERR_ARG;
   if (need_L && (c->L < 1 || c->L > 64)) return DL_ERR_ARG;
-  if (need_L && (c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_PERSISTENT)) != 0)
+  if ((c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_PERSISTENT | DL_FLAG_KLA)) != 0)
+    return DL_ERR_ARG;
+  if ((c->flags & DL_FLAG_KLA) && (c->variant == DL_RWKV6 || !(c->kla_eps >= 0.f)))
     return DL_ERR_ARG;
   const uint64_t bh = uint64_t(c->B) * uint64_t(c->H);
   if (bh > 0x7fffffffull) return DL_ERR_ARG;  // one CTA per head in a 1-D grid
@@ -282,6 +284,8 @@ int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v, co
   p.H = c.H;
   p.L = c.L;
   p.fills_in_param = (c.B <= dl::kParamFills) ? 1 : 0;
+  p.kla = (c.flags & DL_FLAG_KLA) ? 1 : 0;
+  p.kla_eps = c.kla_eps;
   if (p.fills_in_param)
     for (int b = 0; b < c.B; ++b) st->fill_param.f[b] = static_cast<uint8_t>(st->fill[b]);
   if (launch_step(c, p, st->fill_param, static_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -379,6 +383,8 @@ int dl_eager_step(const dl_config* cfg, float* S, const void* q, const void* k, 
   p.bonus = bonus;
   p.o = o;
   p.H = cfg->H;
+  p.kla = (cfg->flags & DL_FLAG_KLA) ? 1 : 0;
+  p.kla_eps = cfg->kla_eps;
   if (launch_eager(*cfg, p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DL_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DL_OK;

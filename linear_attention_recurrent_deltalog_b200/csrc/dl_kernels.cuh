@@ -56,6 +56,8 @@ struct StepParams {
   int L;
   int nitems;    // work items (head rows) of a persistent launch
   int fills_in_param;  // 1: read fills from the FillParam argument
+  int kla;       // 1: beta carries the KLA gate eta; beta = eta / (|k|^2 + kla_eps)
+  float kla_eps;
 };
 
 // Entries in the log of `head` before this step.
@@ -97,6 +99,8 @@ struct EagerParams {
   const float* bonus;
   float* o;
   int H;
+  int kla;       // as in StepParams
+  float kla_eps;
 };
 
 template <int VAR, typename TIn>
@@ -387,18 +391,23 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     entry_weights<VAR, DK, TIn, TIn>(f, warp, NW, lane, sKr, sQr, sK, sG,
                                      (GW == 1) ? &sScal[3] : sDecV, sW, sZ);
   if (warp == NW - 1) {
-    // GDN/KDA: k_t . q_t (the current entry's own weight on q);
-    // RWKV6: the bonus sum_c r_c u_c k_c.
-    float x = 0.f;
+    // GDN/KDA: k_t . q_t (the current entry's own weight on q) and, for the
+    // KLA step size, |k_t|^2; RWKV6: the bonus sum_c r_c u_c k_c.
+    float x = 0.f, kk = 0.f;
 #pragma unroll
     for (int cc = 0; cc < CPL; ++cc) {
       const int c = lane * CPL + cc;
       const float kc = to_f(sKr[c]);
       const float qc = to_f(sQr[c]);
       x = (VAR == kVarRWKV6) ? fmaf(qc * p.bonus[size_t(h) * DK + c], kc, x) : fmaf(kc, qc, x);
+      kk = fmaf(kc, kc, kk);
     }
     x = warp_sum(x);
-    if (lane == 0) sScal[0] = x;
+    if (VAR != kVarRWKV6 && p.kla) kk = warp_sum(kk);
+    if (lane == 0) {
+      sScal[0] = x;
+      if (VAR != kVarRWKV6 && p.kla) sScal[1] = sScal[1] / (kk + p.kla_eps);  // eta -> beta
+    }
   }
   if (!__syncthreads_and(ok)) {
     mbar_wait(barLog, 0, nullptr, 0);
@@ -750,17 +759,20 @@ dl_eager_kernel(const EagerParams p) {
   }
   __syncthreads();
   if (warp == NW - 1) {
-    float x = 0.f;
+    float x = 0.f, kk = 0.f;
 #pragma unroll
     for (int cc = 0; cc < CPL; ++cc) {
       const int c = lane * CPL + cc;
       x = (VAR == kVarRWKV6) ? fmaf(sq[c] * p.bonus[size_t(h) * DK + c], sk[c], x)
                              : fmaf(sk[c], sq[c], x);
+      kk = fmaf(sk[c], sk[c], kk);
     }
     x = warp_sum(x);
+    if (VAR != kVarRWKV6 && p.kla) kk = warp_sum(kk);
     if (lane == 0) {
       sScal[0] = x;
-      sScal[1] = (VAR == kVarRWKV6) ? 0.f : p.beta[head];
+      sScal[1] = (VAR == kVarRWKV6) ? 0.f
+                 : (p.kla ? p.beta[head] / (kk + p.kla_eps) : p.beta[head]);
       sScal[2] = (VAR == kVarGDN) ? p.decay[head] : 1.f;
     }
   }

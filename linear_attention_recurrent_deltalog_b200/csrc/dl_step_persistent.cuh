@@ -262,7 +262,7 @@ dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam 
         sScal[2] = expf(gt);
         if (appender) gG[f] = gt;
       }
-      sScal[1] = hdr.beta;
+      if (!(VAR != kVarRWKV6 && p.kla)) sScal[1] = hdr.beta;
       if (part == 0) p.fill_out[head] = merge_now ? 0 : f + 1;
     }
     if (f > 0) {
@@ -270,16 +270,21 @@ dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam 
       entry_weights<VAR, DK, TIn, TIn>(f, cw, NCW, lane, sKr, sQr, sK, sG, dec, sW, sZ);
     }
     if (cw == NCW - 1) {
-      float x = 0.f;
+      float x = 0.f, kk = 0.f;
 #pragma unroll
       for (int cc = 0; cc < CPL; ++cc) {
         const int c = lane * CPL + cc;
         const float kc = to_f(sKr[c]);
         const float qc = to_f(sQr[c]);
         x = (VAR == kVarRWKV6) ? fmaf(qc * p.bonus[size_t(h) * DK + c], kc, x) : fmaf(kc, qc, x);
+        kk = fmaf(kc, kc, kk);
       }
       x = warp_sum(x);
-      if (lane == 0) sScal[0] = x;
+      if (VAR != kVarRWKV6 && p.kla) kk = warp_sum(kk);
+      if (lane == 0) {
+        sScal[0] = x;
+        if (VAR != kVarRWKV6 && p.kla) sScal[1] = hdr.beta / (kk + p.kla_eps);
+      }
     }
     named_bar_sync(bar_id, GT);
 

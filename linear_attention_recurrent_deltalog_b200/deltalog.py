@@ -33,6 +33,7 @@ DL_ERR_CUDA, DL_ERR_UNSUPPORTED, DL_ERR_DEVICE = -4, -5, -6
 DL_MERGE_FULL, DL_MERGE_ALL = 0, 1
 DL_FLAG_FUSED_MERGE = 1
 DL_FLAG_PERSISTENT = 2
+DL_FLAG_KLA = 4
 
 VARIANT_IDS = {"gdn": DL_GDN, "kda": DL_KDA, "rwkv6": DL_RWKV6}
 DTYPE_IDS = {"f32": DL_F32, "bf16": DL_BF16}
@@ -52,7 +53,8 @@ _lib = _load()
 
 class dl_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("variant", "B", "H", "d_k", "d_v", "L", "in_dtype", "flags", "step_split")]
+                ("variant", "B", "H", "d_k", "d_v", "L", "in_dtype", "flags", "step_split")] + \
+        [("kla_eps", ctypes.c_float)]
 
 
 _P = ctypes.c_void_p
@@ -120,12 +122,15 @@ class Config:
     fused_merge: bool = False
     step_split: int = 0
     persistent: bool = False
+    kla_eps: Optional[float] = None  # set: beta carries the KLA gate eta
 
     def c(self) -> dl_config:
         flags = (DL_FLAG_FUSED_MERGE if self.fused_merge else 0) | \
-            (DL_FLAG_PERSISTENT if self.persistent else 0)
+            (DL_FLAG_PERSISTENT if self.persistent else 0) | \
+            (DL_FLAG_KLA if self.kla_eps is not None else 0)
         return dl_config(VARIANT_IDS[self.variant], self.B, self.H, self.d_k, self.d_v, self.L,
-                         DTYPE_IDS[self.in_dtype], flags, self.step_split)
+                         DTYPE_IDS[self.in_dtype], flags, self.step_split,
+                         0.0 if self.kla_eps is None else float(self.kla_eps))
 
     @property
     def heads(self) -> int:

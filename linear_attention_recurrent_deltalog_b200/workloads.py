@@ -19,7 +19,8 @@ library is measured on:
 Draw recipe (fixed, so any single step can be regenerated on its own):
   * step t uses numpy ``Generator(PCG64(SeedSequence([seed, 1, t])))`` and
     draws, in order, q (or r), k, v, decay, beta, each shaped [B, H, .] in
-    C order (beta is not drawn for RWKV6);
+    C order (beta is not drawn for RWKV6; with the KLA step size the beta
+    draw is the gate eta and q, k are scaled by 1/sqrt(d_k), not normalised);
   * the initial state S0 uses ``SeedSequence([seed, 0, 0])``: fp32 N(0, 1)
     scaled by 0.01 (the "N(0, 0.01)" of the configs read as a standard
     deviation), shaped [B, H, d_v, d_k];
@@ -62,6 +63,9 @@ class Workload:
     ragged: bool = False  # sequences start at fill offsets U{0..L-1}
     alpha_kind: str = "softplus"  # GDN scalar decay recipe: "uniform" or "softplus"
     s0_std: float = 0.01
+    # KLA (Kaczmarz step size): q and k are scaled by 1/sqrt(d_k) instead of
+    # L2-normalised, and the beta draw is the gate eta; None: plain GDN/KDA.
+    kla_eps: Optional[float] = None
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -171,8 +175,12 @@ def step_inputs(w: Workload, t: int, B: Optional[int] = None) -> StepInputs:
         wdec = np.exp(-np.exp(g.normal(-1.0, 0.5, size=(B, H, dk))))
         return StepInputs(t, _to_in_dtype(r, w.in_dtype), _to_in_dtype(k, w.in_dtype),
                           _to_in_dtype(v, w.in_dtype), round_f32(wdec), None, w.in_dtype)
-    q = _l2norm(g.standard_normal((B, H, dk)))
-    k = _l2norm(g.standard_normal((B, H, dk)))
+    if w.kla_eps is None:
+        q = _l2norm(g.standard_normal((B, H, dk)))
+        k = _l2norm(g.standard_normal((B, H, dk)))
+    else:
+        q = g.standard_normal((B, H, dk)) / np.sqrt(dk)
+        k = g.standard_normal((B, H, dk)) / np.sqrt(dk)
     v = g.standard_normal((B, H, dv))
     if w.variant == GDN:
         if w.alpha_kind == "uniform":

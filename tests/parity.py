@@ -101,11 +101,12 @@ def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence
             dense[arm] = S0_d.clone()
         else:
             cfg = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype,
-                             fused_merge=(arm == "fused"), step_split=split, persistent=persistent)
+                             fused_merge=(arm == "fused"), step_split=split, persistent=persistent,
+                             kla_eps=w.kla_eps)
             st = dlb.DeltaLogState(cfg, device=device)
             st.reset(S0_d, fill0.tolist())
             states[arm] = st
-    cfg_e = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype)
+    cfg_e = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype, kla_eps=w.kla_eps)
     out = {arm: [] for arm in arms}
     snap_gpu = {arm: {} for arm in arms}
     recs = []
@@ -146,7 +147,7 @@ def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence
     if w.variant == wl.RWKV6:
         S0h = S0h.transpose(0, 2, 1)
     bon = None if bonus is None else bonus[heads % w.H]
-    ref = oracle.run_eager(w.variant, S0h, recs, bonus=bon, snapshot_at=snaps)
+    ref = oracle.run_eager(w.variant, S0h, recs, bonus=bon, snapshot_at=snaps, kla_eps=w.kla_eps)
     result = {}
     for arm in arms:
         out_err = max(_rel(a, r) for a, r in zip(out[arm], ref.outputs))

@@ -86,7 +86,14 @@ def test_bad_enums_rejected():
     c.in_dtype = 3
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
     c = cfg().c()
-    c.flags = 4
+    c.flags = 8
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+    # the KLA step size applies to GDN and KDA, with a non-negative epsilon
+    c = cfg(kla_eps=1e-6).c()
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_OK
+    c = cfg(variant="rwkv6", d_k=64, d_v=64, kla_eps=1e-6).c()
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+    c = cfg(kla_eps=-1.0).c()
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
 
 

@@ -121,3 +121,13 @@ def test_large_batch_fallbacks(B):
     w = wl.WORKLOADS["kda"].replace(B=B, H=1, d_k=64, d_v=128, L=3, T=7, ragged=True)
     _check(run_parity(w, heads=wl.sample_heads(w, 32), snap_every=3, workers=0,
                       arms=("log", "fused")))
+
+
+@pytest.mark.parametrize("persistent", [False, True])
+@pytest.mark.parametrize("name", ["gdn_qwen", "kda"])
+def test_kla_step_size(name, persistent):
+    # beta = eta / (|k|^2 + eps) formed in the kernels, unnormalised keys
+    w = wl.WORKLOADS[name].replace(B=6, H=5, L=8, T=27, ragged=True, kla_eps=1e-6)
+    _check(run_parity(w, snap_every=9, workers=0, persistent=persistent))
+    w = wl.WORKLOADS[name].replace(kla_eps=1e-3)
+    _check(run_parity(w, T=40, heads=wl.sample_heads(w, 24), arms=("fused", "eager")))

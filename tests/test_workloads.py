@@ -80,3 +80,11 @@ def test_sample_heads():
     h = wl.sample_heads(w, 50)
     assert len(h) == 50 and len(set(h.tolist())) == 50 and h.max() < w.heads
     np.testing.assert_array_equal(h, wl.sample_heads(w, 50))
+
+
+def test_kla_workload_keeps_key_norms():
+    w = wl.WORKLOADS["gdn_qwen"].replace(B=4, H=3, kla_eps=1e-6)
+    s = wl.step_inputs(w, 0)
+    n = np.linalg.norm(s.k.astype(np.float64), axis=-1)
+    assert n.std() > 0.02  # not normalised: the KLA step size sees the norms
+    assert abs(n.mean() - 1.0) < 0.2
