@@ -313,7 +313,10 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(device)
 
     # inputs: a device ring of RING pre-drawn steps (the generator's recipe)
-    host_steps = list(wl.StepStream(w, RING, workers=args.gen_workers))
+    workers = args.gen_workers
+    if workers is None:  # share the host cores among the ranks of this node
+        workers = max(0, min(16, ((os.cpu_count() or 1) - 1) // max(1, world)))
+    host_steps = list(wl.StepStream(w, RING, workers=workers))
     ring = [to_dev(s, device) for s in host_steps]
     gen = torch.Generator(device=device)
     gen.manual_seed(w.seed)

@@ -146,7 +146,10 @@ int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* st
  *   o: fp32 [B, H, d_v] output o_t
  * All pointers 16-byte aligned device addresses.  Without
  * DL_FLAG_FUSED_MERGE, returns DL_ERR_LOG_FULL (enqueuing nothing) when
- * some sequence's log already holds L entries: call dl_merge first. */
+ * some sequence's log already holds L entries: call dl_merge first.
+ * The launch carries each sequence's current fill (from the host-side
+ * mirror) by value, so a CUDA graph captured around this call would replay
+ * the fills of the captured step: do not capture it. */
 int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v,
                    const float* decay, const float* beta, const float* bonus,
                    float* o, void* stream);
@@ -154,7 +157,9 @@ int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v,
 /* Folds logs into the base: S_b <- S_b Diag(gamma) + sum_i u_i (k_i o
  * gamma / gamma_i)^T, then empties those logs.  mode DL_MERGE_FULL folds
  * the sequences whose log holds L entries, DL_MERGE_ALL every non-empty
- * log.  Enqueues nothing when no sequence qualifies. */
+ * log.  Enqueues nothing when no sequence qualifies.  Like
+ * dl_decode_step, the launch carries the qualifying sequences and their
+ * fills by value (do not capture it in a CUDA graph). */
 int dl_merge(dl_state* st, int mode, void* stream);
 
 /* Writes the dense state S_t = base folded with the log to S_out (fp32
