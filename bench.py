@@ -537,6 +537,75 @@ def run_ours(args, world, rank, local):
     return line
 
 
+# ------------------------------------------------------------ serving loop
+
+def run_serving(args, world, rank, local):
+    """A multi-layer decode loop with continuous batching: every token step
+    runs the DeltaLog step of `layers` layers (fused merges), and every
+    `admit_every` steps a fraction of the batch's slots take new sequences
+    (dl_state_load_seqs with zero states, in every layer).  Reports decode
+    tokens/s of the whole stack and the share of time spent on admission."""
+    from linear_attention_recurrent_deltalog_b200 import deltalog as dlb
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = wl.WORKLOADS[args.workload]
+    w = w.replace(L=args.L or w.L, B=args.B or w.B)
+    cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=True,
+                     step_split=args.split)
+    stream = torch.cuda.current_stream(device)
+    host_steps = list(wl.StepStream(w, RING, workers=args.gen_workers))
+    ring = [to_dev(s, device) for s in host_steps]
+    bonus = (torch.from_numpy(wl.rwkv6_bonus(w)).to(device).reshape(-1)
+             if w.variant == wl.RWKV6 else None)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    fills = wl.fill_offsets(w).tolist()
+    layers = []
+    for _ in range(args.layers):
+        st = dlb.DeltaLogState(cfg, device=device)
+        S0 = torch.randn(w.heads * w.d_v * w.d_k, generator=gen, device=device) * w.s0_std
+        st.reset(S0, fills)
+        del S0
+        layers.append(st)
+    o = torch.empty(w.heads * w.d_v, dtype=torch.float32, device=device)
+    churn = max(1, w.B // 64)
+    rng = np.random.default_rng(w.seed)
+
+    def token_step(i):
+        if args.admit_every > 0 and i % args.admit_every == args.admit_every - 1:
+            seqs = rng.choice(w.B, size=churn, replace=False).tolist()
+            for st in layers:
+                st.load_seqs(seqs)
+        q, k, v, dec, beta = ring[i % RING]
+        for st in layers:
+            st.step(q, k, v, dec, beta, bonus, o)
+
+    for i in range(args.warmup):
+        token_step(i)
+    torch.cuda.synchronize(device)
+    dist_barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(args.steps):
+        token_step(args.warmup + i)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    el = max_over_ranks(a.elapsed_time(b) / 1e3, world, device)
+    for st in layers:
+        code, head = st.device_error()
+        if code != 0:
+            raise RuntimeError(f"device error {code} at head {head}")
+        st.close()
+    return {"serving": True, "metric": "decode tokens/s through an N-layer state-update stack",
+            "value": round(aggregate_value(w.B * args.steps, world, el), 1), "unit": UNIT,
+            "layers": args.layers, "n_gpus": world, "steps": args.steps,
+            "ms_per_token_step": round(el * 1e3 / args.steps, 4),
+            "ms_per_layer_step": round(el * 1e3 / args.steps / args.layers, 4),
+            "admission": {"every_steps": args.admit_every, "sequences": churn if args.admit_every else 0},
+            "config": {"workload": workload_desc(w, "fused"), "B": w.B, "L": w.L}}
+
+
 # ------------------------------------------------------------ CPU oracle
 
 def oracle_tokens_per_s(w, target_s: float = 0.0, seqs: int = 2, steps: int = 0, warmup: int = 0):
@@ -627,6 +696,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gen-workers", type=int, default=None)
     ap.add_argument("--sweep", action="store_true", help="also print one line per L in 4..64")
+    ap.add_argument("--serving", action="store_true",
+                    help="multi-layer decode loop with slot admission instead of the headline line")
+    ap.add_argument("--layers", type=int, default=8, help="layers of the --serving loop")
+    ap.add_argument("--admit-every", type=int, default=8,
+                    help="--serving: admit B/64 new sequences every this many steps (0: never)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -636,6 +710,11 @@ def main():
         if args.impl == "reference":
             line = run_reference(args, world, rank)
             if line is not None:
+                print(json.dumps(line), flush=True)
+            return
+        if args.serving:
+            line = run_serving(args, world, rank, local)
+            if rank == 0:
                 print(json.dumps(line), flush=True)
             return
         line = run_ours(args, world, rank, local)

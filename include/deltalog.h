@@ -135,6 +135,15 @@ int dl_state_create(const dl_config* cfg, void* base, void* log, void* meta,
  * `stream` before returning (it copies the fill counts from host memory). */
 int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* stream);
 
+/* Loads dense states into some sequences and empties their logs, leaving
+ * every other sequence untouched: the slot admission of continuous
+ * batching (a finished sequence's slot takes a new one).  seqs: host int32
+ * [n], distinct, each in [0, B).  S: fp32 [n, H, d_v, d_k] device buffer
+ * (16-B aligned; entry i is the state of sequence seqs[i]) or NULL for zero
+ * states.  The loaded sequences' fills become 0.  Asynchronous on `stream`.
+ * Errors: DL_ERR_ARG (bad or repeated index, n < 0), DL_ERR_ALIGN. */
+int dl_state_load_seqs(dl_state* st, int n, const int32_t* seqs, const float* S, void* stream);
+
 /* One decode step for all B*H heads (one kernel launch).
  *   q: q_t (r_t for RWKV6)  [B, H, d_k] in_dtype
  *   k: k_t                  [B, H, d_k] in_dtype

@@ -141,6 +141,22 @@ int check_step_args(const dl_config& c, const void* q, const void* k, const void
   return DL_OK;
 }
 
+// Copies (or zeroes) the d_v x d_k tiles of the listed sequences' heads into
+// the base and empties their logs: CTA i handles head (list.seq[i / H], i % H).
+__global__ void __launch_bounds__(256)
+dl_load_seqs_kernel(float* base, int* fill, const float* S, const dl::SeqList list, int H,
+                    int tile_floats) {
+  const unsigned li = blockIdx.x / unsigned(H);
+  const size_t head = size_t(list.seq[li]) * size_t(H) + blockIdx.x % unsigned(H);
+  float4* dst = reinterpret_cast<float4*>(base + head * size_t(tile_floats));
+  const float4* src =
+      S != nullptr ? reinterpret_cast<const float4*>(S + size_t(blockIdx.x) * size_t(tile_floats))
+                   : nullptr;
+  for (int i = threadIdx.x; i < tile_floats / 4; i += blockDim.x)
+    dst[i] = (src != nullptr) ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (threadIdx.x == 0) fill[head] = 0;
+}
+
 }  // namespace
 
 struct dl_state {
@@ -254,6 +270,33 @@ int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* st
   if (e != cudaSuccess) return DL_ERR_CUDA;
   for (int b = 0; b < c.B; ++b) st->fill[b] = fill0 ? fill0[b] : 0;
   st->parity = 0;
+  st->recount();
+  return DL_OK;
+}
+
+int dl_state_load_seqs(dl_state* st, int n, const int32_t* seqs, const float* S, void* stream) {
+  if (st == nullptr || n < 0 || (n > 0 && seqs == nullptr)) return DL_ERR_ARG;
+  if (S != nullptr && !aligned(S, 16)) return DL_ERR_ALIGN;
+  if (n == 0) return DL_OK;
+  const dl_config& c = st->cfg;
+  std::vector<char> seen(size_t(c.B), 0);
+  for (int i = 0; i < n; ++i) {
+    if (seqs[i] < 0 || seqs[i] >= c.B || seen[size_t(seqs[i])]) return DL_ERR_ARG;
+    seen[size_t(seqs[i])] = 1;
+  }
+  if (c.B > 65536) return DL_ERR_UNSUPPORTED;  // 16-bit sequence indices in the launch
+  const int tile = c.d_v * c.d_k;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int base = 0; base < n; base += dl::kListSeqs) {
+    const int m = (n - base < dl::kListSeqs) ? n - base : dl::kListSeqs;
+    for (int i = 0; i < m; ++i) st->merge_list.seq[i] = static_cast<uint16_t>(seqs[base + i]);
+    const float* Sm = (S != nullptr) ? S + size_t(base) * c.H * tile : nullptr;
+    dl_load_seqs_kernel<<<unsigned(m) * unsigned(c.H), 256, 0, s>>>(st->base, st->dev_fill(), Sm,
+                                                                    st->merge_list, c.H, tile);
+    if (cudaGetLastError() != cudaSuccess) return DL_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+  }
+  for (int i = 0; i < n; ++i) st->fill[size_t(seqs[i])] = 0;
   st->recount();
   return DL_OK;
 }

@@ -66,6 +66,7 @@ _SIGS = {
     "dl_state_bytes": (_I, [_CFG, _SZ, _SZ, _SZ]),
     "dl_state_create": (_I, [_CFG, _P, _P, _P, ctypes.POINTER(_P)]),
     "dl_state_reset": (_I, [_P, _P, ctypes.POINTER(ctypes.c_int32), _P]),
+    "dl_state_load_seqs": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int32), _P, _P]),
     "dl_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "dl_merge": (_I, [_P, _I, _P]),
     "dl_materialize": (_I, [_P, _P, _P]),
@@ -223,6 +224,13 @@ def dl_state_reset(handle: int, cfg: Config, S0=None, fill0: Optional[Sequence[i
     _check(_lib.dl_state_reset(handle, _ptr(S0), arr, _stream(stream)), "dl_state_reset")
 
 
+def dl_state_load_seqs(handle: int, cfg: Config, seqs: Sequence[int], S=None, stream=None) -> None:
+    n = len(seqs)
+    _need(S, "S", n * cfg.H * cfg.d_v * cfg.d_k, torch.float32)
+    arr = (ctypes.c_int32 * max(n, 1))(*[int(x) for x in seqs])
+    _check(_lib.dl_state_load_seqs(handle, n, arr, _ptr(S), _stream(stream)), "dl_state_load_seqs")
+
+
 def dl_decode_step(handle: int, cfg: Config, q, k, v, decay, beta, bonus, o, stream=None) -> None:
     _check_step_tensors(cfg, q, k, v, decay, beta, bonus, o)
     _check(_lib.dl_decode_step(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(beta),
@@ -279,6 +287,9 @@ class DeltaLogState:
 
     def reset(self, S0=None, fill0=None, stream=None) -> None:
         dl_state_reset(self.handle, self.cfg, S0, fill0, stream)
+
+    def load_seqs(self, seqs, S=None, stream=None) -> None:
+        dl_state_load_seqs(self.handle, self.cfg, seqs, S, stream)
 
     def step(self, q, k, v, decay, beta=None, bonus=None, o=None, stream=None):
         if o is None:

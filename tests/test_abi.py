@@ -167,3 +167,20 @@ def test_binding_rejects_undersized_tensors():
     with pytest.raises(TypeError):
         dlb._check_step_tensors(c, torch.zeros(512), torch.zeros(512), torch.zeros(512),
                                 torch.zeros(4), torch.zeros(4), None, torch.zeros(512))
+
+
+def test_load_seqs_checks_indices_on_the_host():
+    c = cfg()
+    h = dlb.dl_state_create(c, 0x100000, 0x200000, 0x300000)
+    try:
+        ld = dlb._lib.dl_state_load_seqs
+        arr = lambda *x: (ctypes.c_int32 * len(x))(*x)
+        assert ld(h, 2, arr(0, 0), None, None) == dlb.DL_ERR_ARG     # repeated
+        assert ld(h, 1, arr(4), None, None) == dlb.DL_ERR_ARG        # out of range (B=4)
+        assert ld(h, 1, arr(-1), None, None) == dlb.DL_ERR_ARG
+        assert ld(h, -1, arr(0), None, None) == dlb.DL_ERR_ARG
+        assert ld(h, 1, None, None, None) == dlb.DL_ERR_ARG
+        assert ld(h, 1, arr(1), 0x1004, None) == dlb.DL_ERR_ALIGN
+        assert ld(h, 0, None, None, None) == dlb.DL_OK                # nothing to do
+    finally:
+        dlb.dl_state_destroy(h)

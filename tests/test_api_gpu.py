@@ -85,3 +85,62 @@ def test_python_binding_refuses_small_buffers_before_launch():
     with pytest.raises(ValueError):
         st.step(small, small, small, torch.empty(6, device="cuda"), torch.empty(6, device="cuda"))
     st.close()
+
+
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
+def test_slot_admission_matches_oracle(name, fused):
+    # Sequences 1 and 4 get new dense states mid-stream (different fill
+    # phases), sequence 2 a zero state later; the others run on untouched.
+    import types
+    import oracle
+    from tests.parity import OUT_TOL, STATE_TOL, host_to_device
+    w = wl.WORKLOADS[name].replace(B=6, H=3, L=5, T=20, ragged=True)
+    BH, dk, dv = w.heads, w.d_k, w.d_v
+    cfg = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype, fused_merge=fused)
+    st = dlb.DeltaLogState(cfg)
+    S0 = wl.initial_state(w)
+    st.reset(torch.from_numpy(S0).cuda().reshape(-1), wl.fill_offsets(w).tolist())
+    bonus = wl.rwkv6_bonus(w) if w.variant == "rwkv6" else None
+    bonus_d = None if bonus is None else torch.from_numpy(bonus).cuda().reshape(-1)
+    rec = w.variant == "rwkv6"
+    S_or = S0.reshape(BH, dv, dk).astype(np.float64)
+    if rec:
+        S_or = S_or.transpose(0, 2, 1).copy()
+    rng = np.random.default_rng(5)
+    o = torch.empty(BH * dv, device="cuda")
+    for t in range(w.T):
+        if t in (7, 13):
+            seqs = [1, 4] if t == 7 else [2]
+            if t == 7:
+                new = (rng.standard_normal((len(seqs), w.H, dv, dk)) * 0.05).astype(np.float32)
+                st.load_seqs(seqs, torch.from_numpy(new).cuda().reshape(-1))
+            else:
+                new = np.zeros((len(seqs), w.H, dv, dk), np.float32)
+                st.load_seqs(seqs)
+            for i, b in enumerate(seqs):
+                blk = new[i].astype(np.float64)
+                S_or[b * w.H:(b + 1) * w.H] = blk.transpose(0, 2, 1) if rec else blk
+            assert all(st.fill()[b] == 0 for b in seqs)
+        s = wl.step_inputs(w, t)
+        q, k, v = (host_to_device(s.device_array(n), "cuda").reshape(-1) for n in ("q", "k", "v"))
+        dec = host_to_device(s.decay, "cuda").reshape(-1)
+        beta = None if s.beta is None else host_to_device(s.beta, "cuda").reshape(-1)
+        st.step(q, k, v, dec, beta, bonus_d, o)
+        if not fused:
+            st.merge(dlb.DL_MERGE_FULL)
+        flat = lambda x: None if x is None else x.reshape((BH,) + x.shape[2:])
+        step = types.SimpleNamespace(q=flat(s.q)[:, None], k=flat(s.k)[:, None], v=flat(s.v)[:, None],
+                                     decay=flat(s.decay)[:, None],
+                                     beta=None if s.beta is None else flat(s.beta)[:, None])
+        res = oracle.run_eager(w.variant, S_or, [step],
+                               bonus=None if bonus is None else bonus[np.arange(BH) % w.H])
+        S_or = res.S
+        o_ref = res.outputs[0]
+        o_gpu = o.view(BH, dv).cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(o_gpu - o_ref)) <= OUT_TOL * np.max(np.abs(o_ref))
+    S_gpu = st.materialize().view(BH, dv, dk).cpu().numpy().astype(np.float64)
+    S_ref = S_or.transpose(0, 2, 1) if rec else S_or
+    assert np.max(np.abs(S_gpu - S_ref)) <= STATE_TOL * np.max(np.abs(S_ref))
+    assert st.device_error() == (0, 0)
+    st.close()
