@@ -208,6 +208,139 @@ __device__ __forceinline__ void load_u16(const TU* sU, int j0, int i, int L, flo
   load_f<16>(sU + su_offset(j0, i, L), u);
 }
 
+// ------------------------------------------------ per-warp row operations
+//
+// A warp owns 16 rows (local indices j0 .. j0+15) of a staged d_v x d_k tile;
+// lane l covers key columns c0 = 4 (l mod LPR) .. c0+3 of row j0 + p*RPI +
+// l/LPR, p = 0 .. NV-1 (Tile's geometry for this d_k).
+
+template <int DK>
+struct WarpRows {
+  static constexpr int LPR = DK / 4;
+  static constexpr int RPI = 32 / LPR;
+  static constexpr int NV = 16 / RPI;
+};
+
+// Row sums a_j = S_j . va and b_j = S_j . vb over the warp's rows in one pass
+// (a skipped unless WITH_A); returns them for the row `jl` this lane ends up
+// owning after the butterfly (lanes l and l^1 own the same row).
+template <int DK, bool WITH_A>
+__device__ __forceinline__ void rows_gemv(const float* sS, int j0, int lane, const float* va,
+                                          const float* vb, float& a, float& b, int& jl) {
+  using G = WarpRows<DK>;
+  const int c0 = (lane % G::LPR) * 4;
+  const int rsub = lane / G::LPR;
+  const float4 a4 = WITH_A ? *reinterpret_cast<const float4*>(va + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4 b4 = *reinterpret_cast<const float4*>(vb + c0);
+  float pa[G::NV], pb[G::NV];
+#pragma unroll
+  for (int pi = 0; pi < G::NV; ++pi) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * G::RPI + rsub) * DK + c0);
+    pa[pi] = WITH_A ? dot4(s4, a4) : 0.f;
+    pb[pi] = dot4(s4, b4);
+  }
+  a = WITH_A ? reduce_rows<G::NV, G::LPR>(pa, lane) : 0.f;
+  b = reduce_rows<G::NV, G::LPR>(pb, lane);
+  jl = j0 + reduced_index<G::NV, G::LPR>(lane) * G::RPI + rsub;
+}
+
+// The step's correction and readout for one row, given its base sums a, b:
+//   log correction ck = sum_i W_i u_i[j], cq = sum_i Z_i u_i[j] (two partial
+//   sums each for instruction-level parallelism), then
+//   GDN  : u = beta (v - gamma a - ck),  o = gamma b + cq + (k.q) u
+//   KDA  : u = beta (v - a - ck),        o = b + cq + (k.q) u
+//   RWKV6: u = v,                        o = b + cq + bonus v
+// sScal: [0] k.q or the RWKV6 bonus, [1] beta, [2] gamma = e^{g_t} (GDN).
+template <int VAR, typename TU>
+__device__ __forceinline__ void row_update(const TU* sU, int jl, int f, int L, const float* sW,
+                                           const float* sZ, const float* sScal, float vj, float a,
+                                           float b, float& u, float& o) {
+  float ck0 = 0.f, ck1 = 0.f, cq0 = 0.f, cq1 = 0.f;
+  int i = 0;
+  for (; i + 1 < f; i += 2) {
+    const float u0 = to_f(sU[su_offset(jl, i, L)]);
+    const float u1 = to_f(sU[su_offset(jl, i + 1, L)]);
+    if (VAR != kVarRWKV6) {
+      ck0 = fmaf(sW[i], u0, ck0);
+      ck1 = fmaf(sW[i + 1], u1, ck1);
+    }
+    cq0 = fmaf(sZ[i], u0, cq0);
+    cq1 = fmaf(sZ[i + 1], u1, cq1);
+  }
+  if (i < f) {
+    const float u0 = to_f(sU[su_offset(jl, i, L)]);
+    if (VAR != kVarRWKV6) ck0 = fmaf(sW[i], u0, ck0);
+    cq0 = fmaf(sZ[i], u0, cq0);
+  }
+  const float ck = ck0 + ck1;
+  const float cq = cq0 + cq1;
+  const float sdot = sScal[0];
+  if (VAR == kVarGDN) {
+    const float gamma = sScal[2];
+    u = sScal[1] * (vj - gamma * a - ck);
+    o = gamma * b + cq + sdot * u;
+  } else if (VAR == kVarKDA) {
+    u = sScal[1] * (vj - a - ck);
+    o = b + cq + sdot * u;
+  } else {
+    u = vj;
+    o = b + cq + sdot * vj;
+  }
+}
+
+// Fused merge of the warp's 16 rows into `gRows` (the rows' first element in
+// global memory): S <- S_b Diag(e^{g_t}) + sum_{i<=f} u_i (k_i o e^{g_t - g_i})^T,
+// entry f being the step's own (u_t, k_t) already staged at slot f.
+// gamma: e^{g_t} (GDN); sGt: g_t per key channel (KDA, RWKV6).
+template <int VAR, int DK, typename TU, typename TIn>
+__device__ __forceinline__ void merge_rows_fused(const float* sS, const TU* sU, const TIn* sK,
+                                                 const float* sG, const float* sGt, float gamma,
+                                                 int f, int L, int j0, int lane, float* gRows) {
+  using G = WarpRows<DK>;
+  const int c0 = (lane % G::LPR) * 4;
+  const int rsub = lane / G::LPR;
+  float4 dec;
+  if (VAR == kVarGDN) {
+    dec.x = dec.y = dec.z = dec.w = gamma;
+  } else {
+    dec = make_float4(expf(sGt[c0]), expf(sGt[c0 + 1]), expf(sGt[c0 + 2]), expf(sGt[c0 + 3]));
+  }
+  float4 acc[G::NV];
+#pragma unroll
+  for (int pi = 0; pi < G::NV; ++pi) {
+    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * G::RPI + rsub) * DK + c0);
+    acc[pi] = make_float4(s4.x * dec.x, s4.y * dec.y, s4.z * dec.z, s4.w * dec.w);
+  }
+  for (int e = 0; e <= f; ++e) {
+    float4 k4 = load4(sK + size_t(e) * DK + c0);
+    if (e < f) {
+      if (VAR == kVarGDN) {
+        const float x = expf(sGt[0] - sG[e]);
+        k4.x *= x; k4.y *= x; k4.z *= x; k4.w *= x;
+      } else {
+        const float* ge = sG + size_t(e) * DK + c0;
+        k4.x *= expf(sGt[c0] - ge[0]);
+        k4.y *= expf(sGt[c0 + 1] - ge[1]);
+        k4.z *= expf(sGt[c0 + 2] - ge[2]);
+        k4.w *= expf(sGt[c0 + 3] - ge[3]);
+      }
+    }
+    float u16[16];
+    load_u16(sU, j0, e, L, u16);
+#pragma unroll
+    for (int pi = 0; pi < G::NV; ++pi) {
+      const float ui = (G::RPI == 1) ? u16[pi] : (rsub ? u16[pi * G::RPI + 1] : u16[pi * G::RPI]);
+      acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
+      acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
+      acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
+      acc[pi].w = fmaf(ui, k4.w, acc[pi].w);
+    }
+  }
+#pragma unroll
+  for (int pi = 0; pi < G::NV; ++pi)
+    *reinterpret_cast<float4*>(gRows + size_t(j0 + pi * G::RPI + rsub) * DK + c0) = acc[pi];
+}
+
 // ------------------------------------------------------------------ step
 //
 // A head's rows may be split over SPLIT = DV / ROWS CTAs (blockIdx.x =
@@ -258,9 +391,6 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   constexpr int GW = StepLayout<VAR, DK, DV, ROWS, TIn>::GW;
   constexpr int NT = Tl::kThreads;
   constexpr int NW = Tl::kWarps;
-  constexpr int NV = Tl::kNV;
-  constexpr int LPR = Tl::kLPR;
-  constexpr int RPI = Tl::kRPI;
   constexpr int CPL = Tl::kCPL;
   static_assert(DV % ROWS == 0, "rows split evenly");
   static_assert(NW >= 2, "one warp issues the tile copies, another the small ones");
@@ -422,58 +552,12 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     mbar_wait(barMine, 0, nullptr, 0);
     return;
   }
-  const int c0 = (lane % LPR) * 4;
-  const int rsub = lane / LPR;
-  const float* vA = (VAR == kVarGDN) ? sk : sKh;
-  const float* vB = (VAR == kVarGDN) ? sq : sQh;
-  const float4 kh4 = *reinterpret_cast<const float4*>(vA + c0);
-  const float4 qh4 = *reinterpret_cast<const float4*>(vB + c0);
-  float pa[NV], pb[NV];
-#pragma unroll
-  for (int pi = 0; pi < NV; ++pi) {
-    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
-    pa[pi] = (VAR == kVarRWKV6) ? 0.f : dot4(s4, kh4);
-    pb[pi] = dot4(s4, qh4);
-  }
-  const float a = (VAR == kVarRWKV6) ? 0.f : reduce_rows<NV, LPR>(pa, lane);
-  const float b = reduce_rows<NV, LPR>(pb, lane);
-  const int jl = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;  // local row
-
-  // ---- log correction, delta-rule correction and readout for row r0 + jl
-  // (two partial sums per weight vector for instruction-level parallelism)
-  float ck0 = 0.f, ck1 = 0.f, cq0 = 0.f, cq1 = 0.f;
-  int i = 0;
-  for (; i + 1 < f; i += 2) {
-    const float u0 = to_f(sU[su_offset(jl, i, L)]);
-    const float u1 = to_f(sU[su_offset(jl, i + 1, L)]);
-    if (VAR != kVarRWKV6) {
-      ck0 = fmaf(sW[i], u0, ck0);
-      ck1 = fmaf(sW[i + 1], u1, ck1);
-    }
-    cq0 = fmaf(sZ[i], u0, cq0);
-    cq1 = fmaf(sZ[i + 1], u1, cq1);
-  }
-  if (i < f) {
-    const float u0 = to_f(sU[su_offset(jl, i, L)]);
-    if (VAR != kVarRWKV6) ck0 = fmaf(sW[i], u0, ck0);
-    cq0 = fmaf(sZ[i], u0, cq0);
-  }
-  const float ck = ck0 + ck1;
-  const float cq = cq0 + cq1;
-  const float vj = to_f(sVr[jl]);
-  const float sdot = sScal[0];
+  float a, b;
+  int jl;  // local row this lane finishes
+  rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
+                                  (VAR == kVarGDN) ? sq : sQh, a, b, jl);
   float u, o;
-  if (VAR == kVarGDN) {
-    const float gamma = sScal[2];
-    u = sScal[1] * (vj - gamma * a - ck);
-    o = gamma * b + cq + sdot * u;
-  } else if (VAR == kVarKDA) {
-    u = sScal[1] * (vj - a - ck);
-    o = b + cq + sdot * u;
-  } else {
-    u = vj;
-    o = b + cq + sdot * vj;
-  }
+  row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, to_f(sVr[jl]), a, b, u, o);
   if ((lane & 1) == 0) {
     p.o[head * DV + r0 + jl] = o;
     if (merge_now)
@@ -482,50 +566,9 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       gU[u_offset(0, r0 + jl, f, L, DV)] = Elem<TU>::from_f(u);
   }
   if (!merge_now) return;
-
-  // ---- fused merge: S_b <- S_b Diag(e^{g_t}) + sum_{i<=f} u_i (k_i o e^{g_t-g_i})^T
   __syncwarp();
-  float4 dec;
-  if (VAR == kVarGDN) {
-    dec.x = dec.y = dec.z = dec.w = sScal[2];
-  } else {
-    dec = make_float4(expf(sGt[c0]), expf(sGt[c0 + 1]), expf(sGt[c0 + 2]), expf(sGt[c0 + 3]));
-  }
-  float4 acc[NV];
-#pragma unroll
-  for (int pi = 0; pi < NV; ++pi) {
-    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
-    acc[pi] = make_float4(s4.x * dec.x, s4.y * dec.y, s4.z * dec.z, s4.w * dec.w);
-  }
-  for (int e = 0; e <= f; ++e) {
-    float4 k4 = load4(sK + size_t(e) * DK + c0);
-    if (e < f) {
-      if (VAR == kVarGDN) {
-        const float x = expf(sGt[0] - sG[e]);
-        k4.x *= x; k4.y *= x; k4.z *= x; k4.w *= x;
-      } else {
-        const float* ge = sG + size_t(e) * DK + c0;
-        k4.x *= expf(sGt[c0] - ge[0]);
-        k4.y *= expf(sGt[c0 + 1] - ge[1]);
-        k4.z *= expf(sGt[c0 + 2] - ge[2]);
-        k4.w *= expf(sGt[c0 + 3] - ge[3]);
-      }
-    }
-    float u16[16];
-    load_u16(sU, j0, e, L, u16);
-#pragma unroll
-    for (int pi = 0; pi < NV; ++pi) {
-      const float ui = (RPI == 1) ? u16[pi] : (rsub ? u16[pi * RPI + 1] : u16[pi * RPI]);
-      acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
-      acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
-      acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
-      acc[pi].w = fmaf(ui, k4.w, acc[pi].w);
-    }
-  }
-  float* gSw = p.base + (head * size_t(DV) + r0) * DK;
-#pragma unroll
-  for (int pi = 0; pi < NV; ++pi)
-    *reinterpret_cast<float4*>(gSw + size_t(j0 + pi * RPI + rsub) * DK + c0) = acc[pi];
+  merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,
+                                     p.base + (head * size_t(DV) + r0) * DK);
 }
 
 // ----------------------------------------------------------- merge / materialize
@@ -784,20 +827,9 @@ dl_eager_kernel(const EagerParams p) {
     mbar_wait(barMine, 0, nullptr, 0);
     return;
   }
-  const int c0 = (lane % LPR) * 4;
-  const int rsub = lane / LPR;
-  const float4 kh4 = *reinterpret_cast<const float4*>(sKh + c0);
-  const float4 qh4 = *reinterpret_cast<const float4*>(sQh + c0);
-  float pa[NV], pb[NV];
-#pragma unroll
-  for (int pi = 0; pi < NV; ++pi) {
-    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
-    pa[pi] = (VAR == kVarRWKV6) ? 0.f : dot4(s4, kh4);
-    pb[pi] = dot4(s4, qh4);
-  }
-  const float a = (VAR == kVarRWKV6) ? 0.f : reduce_rows<NV, LPR>(pa, lane);
-  const float b = reduce_rows<NV, LPR>(pb, lane);
-  const int j = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;
+  float a, b;
+  int j;
+  rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, sKh, sQh, a, b, j);
   const float vj = sV[j];
   const float sdot = sScal[0];
   float u, o;
@@ -818,6 +850,8 @@ dl_eager_kernel(const EagerParams p) {
   }
   __syncwarp();
   // S <- S Diag(decay) + u k^T  (GDN: alpha S + u k^T)
+  const int c0 = (lane % LPR) * 4;
+  const int rsub = lane / LPR;
   const float4 k4 = *reinterpret_cast<const float4*>(sk + c0);
   const float4 d4 = *reinterpret_cast<const float4*>(sDec + c0);
 #pragma unroll

@@ -86,9 +86,6 @@ dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam 
   constexpr int GW = Lay::GW;
   constexpr int NCW = G::kConsumerWarps;
   constexpr int GT = G::kGroupThreads;
-  constexpr int NV = Tl::kNV;
-  constexpr int LPR = Tl::kLPR;
-  constexpr int RPI = Tl::kRPI;
   constexpr int CPL = Tl::kCPL;
   static_assert(DV % ROWS == 0, "rows split evenly");
 
@@ -290,42 +287,12 @@ dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam 
 
     // ---- this warp's 16 rows: dual GEMV, correction, readout, append
     const int j0 = cw * Tl::kRowsPerWarp;
-    const int c0 = (lane % LPR) * 4;
-    const int rsub = lane / LPR;
-    const float* vA = (VAR == kVarGDN) ? sk : sKh;
-    const float* vB = (VAR == kVarGDN) ? sq : sQh;
-    const float4 kh4 = *reinterpret_cast<const float4*>(vA + c0);
-    const float4 qh4 = *reinterpret_cast<const float4*>(vB + c0);
-    float pa[NV], pb[NV];
-#pragma unroll
-    for (int pi = 0; pi < NV; ++pi) {
-      const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
-      pa[pi] = (VAR == kVarRWKV6) ? 0.f : dot4(s4, kh4);
-      pb[pi] = dot4(s4, qh4);
-    }
-    const float a = (VAR == kVarRWKV6) ? 0.f : reduce_rows<NV, LPR>(pa, lane);
-    const float b = reduce_rows<NV, LPR>(pb, lane);
-    const int jl = j0 + reduced_index<NV, LPR>(lane) * RPI + rsub;
-    float ck = 0.f, cq = 0.f;
-    for (int i = 0; i < f; ++i) {
-      const float uij = to_f(sU[su_offset(jl, i, L)]);
-      if (VAR != kVarRWKV6) ck = fmaf(sW[i], uij, ck);
-      cq = fmaf(sZ[i], uij, cq);
-    }
-    const float vj = to_f(sVr[jl]);
-    const float sdot = sScal[0];
+    float a, b;
+    int jl;
+    rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
+                                    (VAR == kVarGDN) ? sq : sQh, a, b, jl);
     float u, o;
-    if (VAR == kVarGDN) {
-      const float gamma = sScal[2];
-      u = sScal[1] * (vj - gamma * a - ck);
-      o = gamma * b + cq + sdot * u;
-    } else if (VAR == kVarKDA) {
-      u = sScal[1] * (vj - a - ck);
-      o = b + cq + sdot * u;
-    } else {
-      u = vj;
-      o = b + cq + sdot * vj;
-    }
+    row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, to_f(sVr[jl]), a, b, u, o);
     if ((lane & 1) == 0) {
       p.o[head * DV + r0 + jl] = o;
       if (merge_now)
@@ -335,47 +302,8 @@ dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam 
     }
     if (merge_now) {
       __syncwarp();
-      float4 dec;
-      if (VAR == kVarGDN) {
-        dec.x = dec.y = dec.z = dec.w = sScal[2];
-      } else {
-        dec = make_float4(expf(sGt[c0]), expf(sGt[c0 + 1]), expf(sGt[c0 + 2]), expf(sGt[c0 + 3]));
-      }
-      float4 acc[NV];
-#pragma unroll
-      for (int pi = 0; pi < NV; ++pi) {
-        const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
-        acc[pi] = make_float4(s4.x * dec.x, s4.y * dec.y, s4.z * dec.z, s4.w * dec.w);
-      }
-      for (int i = 0; i <= f; ++i) {
-        float4 k4 = load4(sK + size_t(i) * DK + c0);
-        if (i < f) {
-          if (VAR == kVarGDN) {
-            const float e = expf(sGt[0] - sG[i]);
-            k4.x *= e; k4.y *= e; k4.z *= e; k4.w *= e;
-          } else {
-            const float* gi = sG + size_t(i) * DK + c0;
-            k4.x *= expf(sGt[c0] - gi[0]);
-            k4.y *= expf(sGt[c0 + 1] - gi[1]);
-            k4.z *= expf(sGt[c0 + 2] - gi[2]);
-            k4.w *= expf(sGt[c0 + 3] - gi[3]);
-          }
-        }
-        float u16[16];
-        load_u16(sU, j0, i, L, u16);
-#pragma unroll
-        for (int pi = 0; pi < NV; ++pi) {
-          const float ui = (RPI == 1) ? u16[pi] : (rsub ? u16[pi * RPI + 1] : u16[pi * RPI]);
-          acc[pi].x = fmaf(ui, k4.x, acc[pi].x);
-          acc[pi].y = fmaf(ui, k4.y, acc[pi].y);
-          acc[pi].z = fmaf(ui, k4.z, acc[pi].z);
-          acc[pi].w = fmaf(ui, k4.w, acc[pi].w);
-        }
-      }
-      float* gSw = p.base + (head * size_t(DV) + r0) * DK;
-#pragma unroll
-      for (int pi = 0; pi < NV; ++pi)
-        *reinterpret_cast<float4*>(gSw + size_t(j0 + pi * RPI + rsub) * DK + c0) = acc[pi];
+      merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,
+                                         p.base + (head * size_t(DV) + r0) * DK);
     }
     // Release the stage once every lane of this warp is done with it.  The
     // fused merge wrote slot f of the staged log through the generic proxy;

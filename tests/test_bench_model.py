@@ -30,3 +30,24 @@ def test_eager_and_merge_bytes():
     mr, mw = bench.merge_bytes(cfg, np.array([16, 3]))
     assert mr == 2 * 32 * 4 + 32 * (65536 + 16 * 772)
     assert mw == 32 * (65536 + 4)
+
+
+def test_reference_arm_prints_the_contract_line():
+    # The reference arm (the fp64 oracle on the host cores) runs without a GPU.
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--steps", "2", "--warmup", "3"], capture_output=True, text=True,
+                         timeout=600, check=True).stdout.strip().splitlines()
+    line = json.loads(out[-1])
+    assert line["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["steps"] == 2 and line["warmup"] == 3 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["metric"] == bench.METRIC and line["unit"] == "tokens/s"
