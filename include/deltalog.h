@@ -195,6 +195,14 @@ int dl_state_destroy(dl_state* st);
  * uses on the current device.  Synchronizes `stream`. */
 int dl_device_error(dl_state* st, int32_t* code, int32_t* head, int clear, void* stream);
 
+/* Exercises the kernels' failure path on the current device without a
+ * fault: one warp waits, with the same bounded wait the kernels use, on a
+ * shared-memory barrier nothing completes; after about one second it gives
+ * up, records the timeout in the device error word the eager kernel uses
+ * and returns.  *code receives the recorded code (1 = wait timed out),
+ * read back and cleared.  Synchronizes `stream`. */
+int dl_selftest_wait_timeout(int32_t* code, void* stream);
+
 /* Total kernels this library has launched in this process. */
 uint64_t dl_launch_count(void);
 

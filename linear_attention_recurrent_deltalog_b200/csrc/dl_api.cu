@@ -157,6 +157,18 @@ dl_load_seqs_kernel(float* base, int* fill, const float* S, const dl::SeqList li
   if (threadIdx.x == 0) fill[head] = 0;
 }
 
+// One warp waits (bounded) on an mbarrier nothing arrives on, so the wait
+// gives up and records kDevErrTimeout: the failure path without a fault.
+__global__ void dl_selftest_wait_kernel(int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    dl::mbar_init(&bar, 1);
+    dl::fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) dl::mbar_wait(&bar, 0, err, -1);
+}
+
 }  // namespace
 
 struct dl_state {
@@ -455,6 +467,24 @@ int dl_device_error(dl_state* st, int32_t* code, int32_t* head, int clear, void*
   if (e != cudaSuccess) return DL_ERR_CUDA;
   if (code) *code = host[0];
   if (head) *head = host[1];
+  return DL_OK;
+}
+
+int dl_selftest_wait_timeout(int32_t* code, void* stream) {
+  if (code == nullptr) return DL_ERR_ARG;
+  int* word = global_err_word();
+  if (word == nullptr) return DL_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(word, 0, 2 * sizeof(int), s) != cudaSuccess) return DL_ERR_CUDA;
+  dl_selftest_wait_kernel<<<1, 32, 0, s>>>(word);
+  if (cudaGetLastError() != cudaSuccess) return DL_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  int host[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(host, word, sizeof(host), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(host), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return DL_ERR_CUDA;
+  *code = host[0];
   return DL_OK;
 }
 

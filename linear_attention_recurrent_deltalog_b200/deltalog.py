@@ -75,6 +75,7 @@ _SIGS = {
     "dl_state_destroy": (_I, [_P]),
     "dl_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                              _I, _P]),
+    "dl_selftest_wait_timeout": (_I, [ctypes.POINTER(ctypes.c_int32), _P]),
     "dl_launch_count": (ctypes.c_uint64, []),
     "dl_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -105,6 +106,14 @@ def dl_status_string(status: int) -> str:
 
 def dl_launch_count() -> int:
     return int(_lib.dl_launch_count())
+
+
+def dl_selftest_wait_timeout(stream=None) -> int:
+    """Runs the bounded-wait failure path once; returns the recorded code."""
+    code = ctypes.c_int32()
+    _check(_lib.dl_selftest_wait_timeout(ctypes.byref(code), _stream(stream)),
+           "dl_selftest_wait_timeout")
+    return code.value
 
 
 # ----------------------------------------------------------------- config
