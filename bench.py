@@ -174,6 +174,13 @@ class ClockSampler:
 
 # ------------------------------------------------------------ byte model
 
+def base_tile_bytes(cfg) -> int:
+    """Bytes of one head's base: fp32 d_v x d_k, or int8 codes + fp32 row scales."""
+    if getattr(cfg, "base", "f32") == "q8":
+        return cfg.d_v * cfg.d_k + cfg.d_v * 4
+    return cfg.d_v * cfg.d_k * 4
+
+
 def step_bytes(cfg, fills: np.ndarray, fused: bool) -> tuple:
     """Algorithmic bytes one step-kernel launch must move (read, write).
 
@@ -187,7 +194,7 @@ def step_bytes(cfg, fills: np.ndarray, fused: bool) -> tuple:
     gw = 1 if cfg.variant == "gdn" else dk
     uin = ein if cfg.variant == "rwkv6" else 4
     entry = dv * uin + dk * ein + gw * 4
-    tile = dv * dk * 4
+    tile = base_tile_bytes(cfg)
     vec = (2 * dk + dv) * ein + (4 if cfg.variant == "gdn" else dk * 4) + (4 if cfg.variant != "rwkv6" else 0)
     f = fills.astype(np.int64)
     merging = (f == cfg.L - 1) if fused else np.zeros_like(f, dtype=bool)
@@ -203,7 +210,7 @@ def merge_bytes(cfg, fills_after_step: np.ndarray) -> tuple:
     gw = 1 if cfg.variant == "gdn" else dk
     uin = ein if cfg.variant == "rwkv6" else 4
     entry = dv * uin + dk * ein + gw * 4
-    tile = dv * dk * 4
+    tile = base_tile_bytes(cfg)
     n = int((fills_after_step == cfg.L).sum())
     allfill = fills_after_step.size * H * 4
     return allfill + n * H * (tile + cfg.L * entry), n * H * (tile + 4)
@@ -237,7 +244,8 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
     cm = dc.replace(cfg, fused_merge=False)
     st = dlb.DeltaLogState(cm, device=device)
     o = torch.empty(w.heads * w.d_v, dtype=torch.float32, device=device)
-    tile = w.d_v * w.d_k * 4
+    tile = base_tile_bytes(cm)
+    dense = w.d_v * w.d_k * 4
     entry = log_entry_bytes(cm)
     ms_merge = []
     for r in range(reps):
@@ -268,7 +276,7 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
     b.record(stream)
     torch.cuda.synchronize(device)
     t_mat = a.elapsed_time(b) / reps / 1e3
-    mtb = w.heads * (2 * tile + half * entry + 4)
+    mtb = w.heads * (tile + dense + half * entry + 4)
     code, head = st.device_error()
     st.close()
     del out
@@ -282,9 +290,11 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
              "algorithmic_bytes": int(mtb)})
 
 
-def workload_desc(w, merge: str) -> str:
+def workload_desc(w, merge: str, base: str = "f32") -> str:
     kla = f", KLA step size eps={w.kla_eps:g}" if w.kla_eps is not None else ""
-    return (f"{w.variant.upper()} decode B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v} fp32 state, "
+    state = ("int8 base with fp32 row scales (requantized at each merge), fp32 log"
+             if base == "q8" else "fp32 state")
+    return (f"{w.variant.upper()} decode B={w.B} H={w.H} d_k={w.d_k} d_v={w.d_v} {state}, "
             f"{w.in_dtype} q/k/v, {'ragged fills, ' if w.ragged else ''}L={w.L}, merge={merge}{kla}")
 
 
@@ -309,7 +319,8 @@ def run_ours(args, world, rank, local):
     w = w.replace(L=args.L or w.L, B=args.B or w.B,
                   kla_eps=args.kla_eps if args.kla_eps >= 0 else None)
     cfg = dlb.Config(w.variant, w.B, w.H, w.d_k, w.d_v, w.L, w.in_dtype, fused_merge=fused,
-                     step_split=args.split, persistent=args.persistent, kla_eps=w.kla_eps)
+                     step_split=args.split, persistent=args.persistent, kla_eps=w.kla_eps,
+                     base=args.base)
     stream = torch.cuda.current_stream(device)
 
     # inputs: a device ring of RING pre-drawn steps (the generator's recipe)
@@ -375,7 +386,7 @@ def run_ours(args, world, rank, local):
     if code != 0:
         raise RuntimeError(f"device error {code} at head {head}")
     max_elapsed = max_over_ranks(elapsed, world, device)
-    state_mib = w.heads * w.d_v * w.d_k * 4 / 2**20
+    state_mib = w.heads * base_tile_bytes(cfg) / 2**20
     tokens = w.B * args.steps
     value = aggregate_value(tokens, world, max_elapsed)
 
@@ -389,7 +400,8 @@ def run_ours(args, world, rank, local):
         try:
             t = json.load(open(tfile))
             if (t.get("kernel_hash") == kernel_hash() and t.get("L") == w.L and t.get("merge") == args.merge
-                    and t.get("workload") == w.name and t.get("B") == w.B):
+                    and t.get("workload") == w.name and t.get("B") == w.B
+                    and t.get("base", "f32") == args.base):
                 traffic = t.get("bytes_per_launch")
         except Exception:
             traffic = None
@@ -398,7 +410,8 @@ def run_ours(args, world, rank, local):
         st.close()
         return {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "only_step": True,
-                "config": {"workload": w.name, "B": w.B, "L": w.L, "merge": args.merge, "split": args.split},
+                "config": {"workload": w.name, "B": w.B, "L": w.L, "merge": args.merge, "split": args.split,
+                           "base": args.base},
                 "roofline": {"achieved": round(achieved, 1), "peak": peak,
                              "frac": round(achieved / peak, 4), "launch_ms": round(step_avg * 1e3, 5)}}
 
@@ -526,12 +539,12 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": workload_desc(w, args.merge), "name": w.name,
+        "config": {"workload": workload_desc(w, args.merge, args.base), "name": w.name, "base": args.base,
                    "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "L": w.L, "merge": args.merge,
                    "step_split": args.split, "persistent": args.persistent,
                    "global_batch": w.B * world,
                    "parallelism": f"replicas x{world} (dp, no collective)",
-                   "l2": (f"state {state_mib:.0f} MiB > 126 MB L2 on every step: no flush needed"
+                   "l2": (f"base {state_mib:.0f} MiB > 126 MB L2 on every step: no flush needed"
                           if state_mib * 2**20 > L2_BYTES else f"state {state_mib:.0f} MiB fits L2: not a bench line"),
                    "input_ring_steps": RING},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -711,6 +724,8 @@ def main():
     ap.add_argument("--only-step", action="store_true",
                     help="time the DeltaLog step only (profiling); not a bench line")
     ap.add_argument("--merge", choices=("fused", "separate"), default="fused")
+    ap.add_argument("--base", choices=("f32", "q8"), default="f32",
+                    help="base storage: fp32, or int8 codes + row scales requantized per window")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

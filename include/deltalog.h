@@ -84,7 +84,22 @@ enum dl_flags {
    * step carries the gate eta_t and the kernels use
    * beta_t = eta_t / (|k_t|_2^2 + kla_eps) ("Kaczmarz Linear Attention"
    * abstract), so the write projects exactly whatever the key's norm. */
-  DL_FLAG_KLA = 4
+  DL_FLAG_KLA = 4,
+  /* int8 base quantized once per window ("LeapQuant" abstract: the state
+   * is quantized only at the end of a window of tokens, and outputs inside
+   * the window use the fixed low-bit state plus high-precision buffered
+   * updates; here the window is the stretch between two merges of a
+   * sequence's log, and the log stays fp32).  The base holds int8 codes
+   * and one fp32 scale per value row:
+   *   amax_j = max_c |x_jc|,  inv_j = 127 / amax_j,
+   *   code_jc = round-half-even(x_jc * inv_j),  scale_j = amax_j / 127,
+   * each an fp32 operation rounded once (rows with amax_j < 2^-120 store
+   * zero codes and scale 0); the base value is code_jc * scale_j.  Every
+   * merge (DL_MERGE_FULL, DL_MERGE_ALL, the fused merge) folds the log in
+   * fp32 and requantizes the rows it writes; dl_state_reset and
+   * dl_state_load_seqs quantize the states they load.  Not combinable with
+   * DL_FLAG_PERSISTENT (DL_ERR_UNSUPPORTED). */
+  DL_FLAG_BASE_Q8 = 8
 };
 
 /* Layer configuration.  d_k, d_v in {64, 128}; 1 <= L <= 64; B, H >= 1 and
@@ -109,7 +124,9 @@ typedef struct dl_config {
 typedef struct dl_state dl_state;
 
 /* Sizes in bytes of the three device buffers a state borrows:
- *   base: fp32 [B, H, d_v, d_k]                 the dense base S_b
+ *   base: fp32 [B, H, d_v, d_k]                 the dense base S_b; with
+ *         DL_FLAG_BASE_Q8 int8 codes [B, H, d_v, d_k] followed, at the
+ *         next 256-B boundary, by the fp32 row scales [B, H, d_v]
  *   log : per head L entries of u (fp32 [d_v]; in_dtype for RWKV6),
  *         k (in_dtype [d_k]) and log-decay g (fp32, [1] for GDN, [d_k]
  *         otherwise), laid out as three arrays [B,H,L,.], each 256-B aligned
@@ -127,7 +144,8 @@ int dl_state_create(const dl_config* cfg, void* base, void* log, void* meta,
                     dl_state** out);
 
 /* Loads a dense state and starts every log.  S0: fp32 [B, H, d_v, d_k]
- * device buffer 16-B aligned, or NULL for a zero state.  fill0: host int32
+ * device buffer 16-B aligned, or NULL for a zero state (an int8 base
+ * stores Q(S0), quantized row by row as described at DL_FLAG_BASE_Q8).  fill0: host int32
  * [B] with 0 <= fill0[b] < L, or NULL for zeros; sequence b starts with
  * fill0[b] log entries that change nothing (u = 0, k = 0, g = 0), so its
  * first merge comes after L - fill0[b] steps (ragged batches sit at
@@ -173,12 +191,13 @@ int dl_merge(dl_state* st, int mode, void* stream);
 
 /* Writes the dense state S_t = base folded with the log to S_out (fp32
  * [B, H, d_v, d_k], 16-B aligned, must not alias the base) without changing
- * the state. */
+ * the state.  An int8 base is dequantized (code * scale) before the fold. */
 int dl_materialize(const dl_state* st, float* S_out, void* stream);
 
 /* Eager dense step, the comparison point: reads and writes the whole fp32
  * state S [B, H, d_v, d_k] (16-B aligned) in place, same recurrence and
- * arguments as dl_decode_step.  cfg->L and cfg->flags are ignored. */
+ * arguments as dl_decode_step.  cfg->L and every flag but DL_FLAG_KLA are
+ * ignored (the state is always fp32). */
 int dl_eager_step(const dl_config* cfg, float* S, const void* q, const void* k,
                   const void* v, const float* decay, const float* beta,
                   const float* bonus, float* o, void* stream);

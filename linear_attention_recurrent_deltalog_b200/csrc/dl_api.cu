@@ -31,8 +31,11 @@ size_t pad(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct Layout {
-  size_t base, u_off, u_bytes, k_off, k_bytes, g_off, g_bytes, log, fill_bytes, err_off, meta;
+  size_t base, scale_off, u_off, u_bytes, k_off, k_bytes, g_off, g_bytes, log, fill_bytes, err_off,
+      meta;
 };
+
+bool is_q8(const dl_config& c) { return (c.flags & DL_FLAG_BASE_Q8) != 0; }
 
 // Default work items per head for the step kernel: 64-row items.
 int default_split(const dl_config& c) { return c.d_v >= 128 ? 2 : 1; }
@@ -46,7 +49,13 @@ int in_elem_size(const dl_config& c) { return c.in_dtype == DL_BF16 ? 2 : 4; }
 Layout layout_of(const dl_config& c) {
   const size_t bh = size_t(c.B) * size_t(c.H);
   Layout l{};
-  l.base = pad(bh * c.d_v * c.d_k * 4);
+  if (is_q8(c)) {  // int8 codes, then the fp32 row scales
+    l.scale_off = pad(bh * c.d_v * c.d_k);
+    l.base = l.scale_off + pad(bh * c.d_v * 4);
+  } else {
+    l.scale_off = 0;
+    l.base = pad(bh * c.d_v * c.d_k * 4);
+  }
   l.u_off = 0;
   l.u_bytes = pad(bh * c.L * c.d_v * u_elem_size(c));
   l.k_off = l.u_off + l.u_bytes;
@@ -69,7 +78,8 @@ int check_config(const dl_config* c, bool need_L) {
   if (c->B < 1 || c->H < 1 || c->d_k < 1 || c->d_v < 1) return DL_ERR_ARG;
   if (c->in_dtype != DL_F32 && c->in_dtype != DL_BF16) return DL_ERR_ARG;
   if (need_L && (c->L < 1 || c->L > 64)) return DL_ERR_ARG;
-  if ((c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_PERSISTENT | DL_FLAG_KLA)) != 0)
+  if ((c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_PERSISTENT | DL_FLAG_KLA |
+                           DL_FLAG_BASE_Q8)) != 0)
     return DL_ERR_ARG;
   if ((c->flags & DL_FLAG_KLA) && (c->variant == DL_RWKV6 || !(c->kla_eps >= 0.f)))
     return DL_ERR_ARG;
@@ -78,6 +88,7 @@ int check_config(const dl_config* c, bool need_L) {
   if (bh * uint64_t(c->d_v) * uint64_t(c->d_k) >= (1ull << 40)) return DL_ERR_ARG;
   if (!head_size_ok(c->d_k) || !head_size_ok(c->d_v)) return DL_ERR_UNSUPPORTED;
   if (c->step_split != 0 && !dl::split_ok(c->d_v, c->step_split)) return DL_ERR_ARG;
+  if ((c->flags & DL_FLAG_BASE_Q8) && (c->flags & DL_FLAG_PERSISTENT)) return DL_ERR_UNSUPPORTED;
   return DL_OK;
 }
 
@@ -90,20 +101,60 @@ cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, const dl::F
                         cudaStream_t s) {
   const unsigned n = unsigned(size_t(c.B) * c.H);
   const bool fused = (c.flags & DL_FLAG_FUSED_MERGE) != 0;
+  const Shape sh = shape_of(c);
+  if (is_q8(c)) {
+    switch (c.variant) {
+      case DL_GDN: return dl::launch_step<dl::kVarGDN, int8_t>(sh, fused, p, fp, n, s);
+      case DL_KDA: return dl::launch_step<dl::kVarKDA, int8_t>(sh, fused, p, fp, n, s);
+      default: return dl::launch_step<dl::kVarRWKV6, int8_t>(sh, fused, p, fp, n, s);
+    }
+  }
   switch (c.variant) {
-    case DL_GDN: return dl::launch_step<dl::kVarGDN>(shape_of(c), fused, p, fp, n, s);
-    case DL_KDA: return dl::launch_step<dl::kVarKDA>(shape_of(c), fused, p, fp, n, s);
-    default: return dl::launch_step<dl::kVarRWKV6>(shape_of(c), fused, p, fp, n, s);
+    case DL_GDN: return dl::launch_step<dl::kVarGDN, float>(sh, fused, p, fp, n, s);
+    case DL_KDA: return dl::launch_step<dl::kVarKDA, float>(sh, fused, p, fp, n, s);
+    default: return dl::launch_step<dl::kVarRWKV6, float>(sh, fused, p, fp, n, s);
   }
 }
 
 // `nctas`: B*H, or (with p.use_list) the listed sequences times H.
 cudaError_t launch_merge(const dl_config& c, const dl::MergeParams& p, const dl::SeqList& list,
                          unsigned nctas, cudaStream_t s) {
+  const Shape sh = shape_of(c);
+  if (is_q8(c)) {
+    switch (c.variant) {
+      case DL_GDN: return dl::launch_merge<dl::kVarGDN, int8_t>(sh, p, list, nctas, s);
+      case DL_KDA: return dl::launch_merge<dl::kVarKDA, int8_t>(sh, p, list, nctas, s);
+      default: return dl::launch_merge<dl::kVarRWKV6, int8_t>(sh, p, list, nctas, s);
+    }
+  }
   switch (c.variant) {
-    case DL_GDN: return dl::launch_merge<dl::kVarGDN>(shape_of(c), p, list, nctas, s);
-    case DL_KDA: return dl::launch_merge<dl::kVarKDA>(shape_of(c), p, list, nctas, s);
-    default: return dl::launch_merge<dl::kVarRWKV6>(shape_of(c), p, list, nctas, s);
+    case DL_GDN: return dl::launch_merge<dl::kVarGDN, float>(sh, p, list, nctas, s);
+    case DL_KDA: return dl::launch_merge<dl::kVarKDA, float>(sh, p, list, nctas, s);
+    default: return dl::launch_merge<dl::kVarRWKV6, float>(sh, p, list, nctas, s);
+  }
+}
+
+// Larger of the step's and the merge's shared memory for this config.
+template <int VAR, typename TB>
+size_t smem_need(const Shape& sh, int L) {
+  const size_t a = dl::step_smem_bytes<VAR, TB>(sh, L);
+  const size_t b = dl::merge_smem_bytes<VAR, TB>(sh, L);
+  return (a == 0 || b == 0) ? 0 : (a > b ? a : b);
+}
+
+size_t smem_need(const dl_config& c) {
+  const Shape sh = shape_of(c);
+  if (is_q8(c)) {
+    switch (c.variant) {
+      case DL_GDN: return smem_need<dl::kVarGDN, int8_t>(sh, c.L);
+      case DL_KDA: return smem_need<dl::kVarKDA, int8_t>(sh, c.L);
+      default: return smem_need<dl::kVarRWKV6, int8_t>(sh, c.L);
+    }
+  }
+  switch (c.variant) {
+    case DL_GDN: return smem_need<dl::kVarGDN, float>(sh, c.L);
+    case DL_KDA: return smem_need<dl::kVarKDA, float>(sh, c.L);
+    default: return smem_need<dl::kVarRWKV6, float>(sh, c.L);
   }
 }
 
@@ -157,6 +208,48 @@ dl_load_seqs_kernel(float* base, int* fill, const float* S, const dl::SeqList li
   if (threadIdx.x == 0) fill[head] = 0;
 }
 
+// Quantizes fp32 d_v x d_k tiles into an int8 base (codes and row scales),
+// one warp per row, with the rule the merge uses: inv = 127 / amax, code =
+// round-half-even(x * inv), scale = amax / 127, each rounded once in fp32;
+// rows with amax below 2^-120 become zero codes and scale 0.  CTA i covers
+// head i, or (use_list) head (list.seq[i / H], i % H) with source tile i;
+// S == nullptr loads zero states.  With `fill`, the covered heads' fills
+// become 0.
+__global__ void __launch_bounds__(256)
+dl_quantize_kernel(int8_t* codes, float* scales, int* fill, const float* S, const dl::SeqList list,
+                   int use_list, int H, int dv, int dk) {
+  const unsigned i = blockIdx.x;
+  const size_t head = use_list ? size_t(list.seq[i / unsigned(H)]) * size_t(H) + i % unsigned(H)
+                               : size_t(i);
+  const float* src = S != nullptr ? S + size_t(i) * dv * dk : nullptr;
+  const int lane = threadIdx.x & 31;
+  const int per = dk / 32;  // 2 or 4 values per lane
+  for (int row = threadIdx.x >> 5; row < dv; row += blockDim.x >> 5) {
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (src != nullptr)
+      for (int e = 0; e < per; ++e) x[e] = src[size_t(row) * dk + lane * per + e];
+    float m = 0.f;
+    for (int e = 0; e < per; ++e) m = fmaxf(m, fabsf(x[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    uint32_t w = 0u;
+    float sc = 0.f;
+    if (m >= dl::kTinyAmax) {
+      const float inv = __fdiv_rn(127.0f, m);
+      for (int e = 0; e < per; ++e)
+        w |= (uint32_t(__float2int_rn(__fmul_rn(x[e], inv))) & 0xffu) << (8 * e);
+      sc = __fdiv_rn(m, 127.0f);
+    }
+    int8_t* dst = codes + (head * dv + row) * size_t(dk) + lane * per;
+    if (per == 4)
+      *reinterpret_cast<uint32_t*>(dst) = w;
+    else
+      *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(w);
+    if (lane == 0) scales[head * dv + row] = sc;
+  }
+  if (fill != nullptr && threadIdx.x == 0) fill[head] = 0;
+}
+
 // One warp waits (bounded) on an mbarrier nothing arrives on, so the wait
 // gives up and records kDevErrTimeout: the failure path without a fault.
 __global__ void dl_selftest_wait_kernel(int* err) {
@@ -190,6 +283,10 @@ struct dl_state {
   }
   int* dev_fill() const { return dev_fill(parity); }
   int* dev_err() const { return reinterpret_cast<int*>(meta + lay.err_off); }
+  float* scales() const {
+    return is_q8(cfg) ? reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(base) + lay.scale_off)
+                      : nullptr;
+  }
   void* logU() const { return log + lay.u_off; }
   void* logK() const { return log + lay.k_off; }
   float* logG() const { return reinterpret_cast<float*>(log + lay.g_off); }
@@ -223,24 +320,7 @@ int dl_state_create(const dl_config* cfg, void* base, void* log, void* meta, dl_
   if (!base || !log || !meta) return DL_ERR_ARG;
   if (!aligned(base, kAlign) || !aligned(log, kAlign) || !aligned(meta, kAlign))
     return DL_ERR_ALIGN;
-  const Shape sh = shape_of(*cfg);
-  size_t need = 0;
-  switch (cfg->variant) {
-    case DL_GDN:
-      need = dl::step_smem_bytes<dl::kVarGDN>(sh, cfg->L);
-      need = need > dl::merge_smem_bytes<dl::kVarGDN>(sh, cfg->L) ? need
-                                                                : dl::merge_smem_bytes<dl::kVarGDN>(sh, cfg->L);
-      break;
-    case DL_KDA:
-      need = dl::step_smem_bytes<dl::kVarKDA>(sh, cfg->L);
-      need = need > dl::merge_smem_bytes<dl::kVarKDA>(sh, cfg->L) ? need
-                                                                : dl::merge_smem_bytes<dl::kVarKDA>(sh, cfg->L);
-      break;
-    default:
-      need = dl::step_smem_bytes<dl::kVarRWKV6>(sh, cfg->L);
-      need = need > dl::merge_smem_bytes<dl::kVarRWKV6>(sh, cfg->L) ? need
-                                                                  : dl::merge_smem_bytes<dl::kVarRWKV6>(sh, cfg->L);
-  }
+  const size_t need = smem_need(*cfg);
   if (need == 0 || need > size_t(dl::kMaxSmemOptIn)) return DL_ERR_UNSUPPORTED;
   dl_state* st = new (std::nothrow) dl_state();
   if (st == nullptr) return DL_ERR_ARG;
@@ -267,9 +347,21 @@ int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* st
       if (fill0[b] < 0 || fill0[b] >= c.L) return DL_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t state_bytes = size_t(c.B) * c.H * c.d_v * c.d_k * 4;
-  cudaError_t e = (S0 != nullptr)
-                      ? cudaMemcpyAsync(st->base, S0, state_bytes, cudaMemcpyDeviceToDevice, s)
-                      : cudaMemsetAsync(st->base, 0, state_bytes, s);
+  cudaError_t e = cudaSuccess;
+  if (is_q8(c)) {
+    if (S0 != nullptr) {
+      dl_quantize_kernel<<<unsigned(size_t(c.B) * c.H), 256, 0, s>>>(
+          static_cast<int8_t*>(static_cast<void*>(st->base)), st->scales(), nullptr, S0,
+          st->merge_list, 0, c.H, c.d_v, c.d_k);
+      e = cudaGetLastError();
+      if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+    } else {
+      e = cudaMemsetAsync(st->base, 0, st->lay.base, s);
+    }
+  } else {
+    e = (S0 != nullptr) ? cudaMemcpyAsync(st->base, S0, state_bytes, cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(st->base, 0, state_bytes, s);
+  }
   if (e == cudaSuccess) e = cudaMemsetAsync(st->log, 0, st->lay.log, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(st->meta, 0, st->lay.meta, s);
   for (int b = 0; b < c.B; ++b)
@@ -303,8 +395,13 @@ int dl_state_load_seqs(dl_state* st, int n, const int32_t* seqs, const float* S,
     const int m = (n - base < dl::kListSeqs) ? n - base : dl::kListSeqs;
     for (int i = 0; i < m; ++i) st->merge_list.seq[i] = static_cast<uint16_t>(seqs[base + i]);
     const float* Sm = (S != nullptr) ? S + size_t(base) * c.H * tile : nullptr;
-    dl_load_seqs_kernel<<<unsigned(m) * unsigned(c.H), 256, 0, s>>>(st->base, st->dev_fill(), Sm,
-                                                                    st->merge_list, c.H, tile);
+    if (is_q8(c))
+      dl_quantize_kernel<<<unsigned(m) * unsigned(c.H), 256, 0, s>>>(
+          static_cast<int8_t*>(static_cast<void*>(st->base)), st->scales(), st->dev_fill(), Sm,
+          st->merge_list, 1, c.H, c.d_v, c.d_k);
+    else
+      dl_load_seqs_kernel<<<unsigned(m) * unsigned(c.H), 256, 0, s>>>(st->base, st->dev_fill(), Sm,
+                                                                      st->merge_list, c.H, tile);
     if (cudaGetLastError() != cudaSuccess) return DL_ERR_CUDA;
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
@@ -323,6 +420,7 @@ int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v, co
   if (st->n_full > 0) return DL_ERR_LOG_FULL;
   dl::StepParams p{};
   p.base = st->base;
+  p.scale = st->scales();
   p.logU = st->logU();
   p.logK = st->logK();
   p.logG = st->logG();
@@ -362,6 +460,7 @@ int dl_merge(dl_state* st, int mode, void* stream) {
   const dl_config& c = st->cfg;
   dl::MergeParams p{};
   p.base = st->base;
+  p.scale = st->scales();
   p.logU = st->logU();
   p.logK = st->logK();
   p.logG = st->logG();
@@ -400,6 +499,7 @@ int dl_materialize(const dl_state* st, float* S_out, void* stream) {
   const dl_config& c = st->cfg;
   dl::MergeParams p{};
   p.base = st->base;
+  p.scale = st->scales();
   p.logU = st->logU();
   p.logK = st->logK();
   p.logG = st->logG();

@@ -8,6 +8,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace dl {
 
 constexpr int kVarGDN = 0;
@@ -229,9 +231,10 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// Tile geometry: ROWS rows (value indices) of a d_v x d_k fp32 tile, d_k
-// columns, handled by ROWS/16 warps of 16 rows each.
-template <int DK, int ROWS>
+// Tile geometry: ROWS rows (value indices) of a d_v x d_k tile of TB (fp32,
+// or int8 codes for a quantized base), d_k columns, handled by ROWS/16 warps
+// of 16 rows each.
+template <int DK, int ROWS, typename TB = float>
 struct Tile {
   static_assert(DK == 64 || DK == 128, "d_k in {64,128}");
   static_assert(ROWS == 32 || ROWS == 64 || ROWS == 128, "rows per CTA in {32,64,128}");
@@ -246,10 +249,82 @@ struct Tile {
   // tile goes out as several concurrent copies.
   static constexpr int kChunkRows = 16;
   static constexpr int kChunks = ROWS / kChunkRows;
-  static constexpr uint32_t kChunkBytes = kChunkRows * DK * 4;
-  static constexpr size_t kTileBytes = size_t(ROWS) * DK * 4;
+  static constexpr uint32_t kChunkBytes = kChunkRows * DK * sizeof(TB);
+  static constexpr size_t kTileBytes = size_t(ROWS) * DK * sizeof(TB);
   static constexpr int kCPL = DK / 32;              // key columns per lane in 32-lane dots
   static_assert(kLPR == 2 * kNV, "row reduction layout");
 };
+
+// ------------------------------------------------------ int8 base rows
+//
+// A quantized base row holds d_k int8 codes and one fp32 scale per value
+// row (the scale multiplies a finished row dot product).  A warp covers 16
+// rows with 16 consecutive codes (one 16-byte shared-memory load) per lane:
+// QL lanes per row, 32/QL rows per warp instruction, QNV rows per lane.
+
+template <int DK>
+struct QRows {
+  static constexpr int kCodes = 16;          // codes per lane per row
+  static constexpr int kLPR = DK / kCodes;   // lanes per row
+  static constexpr int kRPI = 32 / kLPR;     // rows per warp instruction
+  static constexpr int kNV = 16 / kRPI;      // rows per lane
+  static_assert(kLPR == 2 * kNV, "row reduction layout");
+};
+
+// Four int8 codes packed in a word -> exact fp32 values.  IEEE-754 single
+// precision has 23 fraction bits, so 2^23 + n for n in [0, 255] is exact and
+// its low fraction byte is n.  Flipping each code's sign bit gives n = code +
+// 128; a byte permute builds the word (0x4B, 0, 0, n) = 2^23 + n and one
+// subtraction of 2^23 + 128 leaves the code, with no integer-to-float
+// conversion instruction.
+__device__ __forceinline__ void codes4_to_f(uint32_t w, float* f) {
+  const uint32_t u = w ^ 0x80808080u;
+  constexpr float kBias = 8388736.0f;  // 2^23 + 128
+  f[0] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)) - kBias;
+  f[1] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541)) - kBias;
+  f[2] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)) - kBias;
+  f[3] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543)) - kBias;
+}
+
+// Sixteen codes (16-byte aligned) -> fp32.
+__device__ __forceinline__ void codes16_to_f(const int8_t* p, float (&f)[16]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  codes4_to_f(w.x, f);
+  codes4_to_f(w.y, f + 4);
+  codes4_to_f(w.z, f + 8);
+  codes4_to_f(w.w, f + 12);
+}
+
+// Rows whose absolute maximum is below this are stored as zero (127/amax
+// would overflow fp32 near the bottom of its range).
+constexpr float kTinyAmax = 7.52316384526264e-37f;  // 2^-120
+
+// Quantizes this lane's 16 values of a row whose absolute maximum is amax
+// (the same in every lane of the row): code = round-half-even(x * inv),
+// inv = 127 / amax, each one correctly rounded fp32 operation.  Returns the
+// codes packed for one 16-byte store; *scale = amax / 127.
+__device__ __forceinline__ uint4 quantize16(const float (&x)[16], float amax, float* scale) {
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  if (amax >= kTinyAmax) {
+    const float inv = __fdiv_rn(127.0f, amax);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = __float2int_rn(__fmul_rn(x[i], inv));
+      w[i >> 2] |= (uint32_t(c) & 0xffu) << (8 * (i & 3));
+    }
+    *scale = __fdiv_rn(amax, 127.0f);
+  } else {
+    *scale = 0.f;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Maximum over the kLPR lanes of a row (lanes differing in their low bits).
+template <int LPR>
+__device__ __forceinline__ float row_max(float x) {
+#pragma unroll
+  for (int o = 1; o < LPR; o <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
 
 }  // namespace dl

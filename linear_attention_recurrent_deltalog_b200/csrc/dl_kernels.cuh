@@ -1,8 +1,10 @@
 // dl_kernels.cuh -- the DeltaLog kernels for sm_100a.
 //
 // Notation ("DeltaLog: Deferred Materialization of Recurrent States for Linear
-// Attention Decoding", Abstract): each head keeps a dense base S_b (fp32,
-// d_v x d_k, row = value index) and a bounded log of f < L compact entries
+// Attention Decoding", Abstract): each head keeps a dense base S_b (fp32, or
+// int8 codes with one fp32 scale per row -- the base quantized once per
+// window, "LeapQuant" Abstract -- d_v x d_k, row = value index) and a
+// bounded log of f < L compact entries
 // (u_i, k_i, g_i), g_i = log of the decay accumulated since the base was
 // merged (a scalar for GDN, a d_k vector for KDA and RWKV6).  The dense state
 // the model sees is
@@ -20,7 +22,8 @@
 //                      append would fill the log writes the merged base
 //                      instead (it already holds S_b and the whole log).
 //   dl_merge_kernel  : folds a log into the base (or into a separate output
-//                      for materialize) -- a rank-f update of the tile.
+//                      for materialize) -- a rank-f update of the tile.  An
+//                      int8 base is requantized row by row as it is written.
 //   dl_eager_kernel  : the dense read-modify-write step eager decoding does.
 #pragma once
 
@@ -38,7 +41,8 @@ struct FillParam {
 };
 
 struct StepParams {
-  float* base;   // [BH, DV, DK]
+  void* base;    // [BH, DV, DK]  fp32, or int8 codes
+  float* scale;  // [BH, DV]  row scales of an int8 base (else null)
   void* logU;    // [BH, DV/32, L, 32]  fp32 (in_dtype for RWKV6): see u_offset
   void* logK;    // [BH, L, DK]  in_dtype
   float* logG;   // [BH, L, GW]
@@ -75,13 +79,14 @@ struct SeqList {
 };
 
 struct MergeParams {
-  float* base;
+  void* base;    // fp32, or int8 codes
+  float* scale;  // row scales of an int8 base (else null)
   const void* logU;
   const void* logK;
   const float* logG;
   int* fill;
   int* err;
-  float* out;    // merge: == base; materialize: caller buffer
+  float* out;    // materialize: caller buffer; merge of an fp32 base: == base
   int L;
   int mode;      // 0 merge full logs, 1 merge every non-empty log, 2 materialize
   int H;
@@ -341,6 +346,102 @@ __device__ __forceinline__ void merge_rows_fused(const float* sS, const TU* sU, 
     *reinterpret_cast<float4*>(gRows + size_t(j0 + pi * G::RPI + rsub) * DK + c0) = acc[pi];
 }
 
+// ---------------------------------------------------- int8 base rows
+//
+// The same per-warp operations on an int8 base (QRows layout: 16 codes per
+// lane per row).  The row scale multiplies the finished dot products.
+
+template <int DK, bool WITH_A>
+__device__ __forceinline__ void rows_gemv_q8(const int8_t* sQ, const float* sScale, int j0, int lane,
+                                             const float* va, const float* vb, float& a, float& b,
+                                             int& jl) {
+  using G = QRows<DK>;
+  const int c0 = (lane % G::kLPR) * G::kCodes;
+  const int rsub = lane / G::kLPR;
+  float ka[16], kb[16];
+  if (WITH_A) load_f<16>(va + c0, ka);
+  load_f<16>(vb + c0, kb);
+  float pa[G::kNV], pb[G::kNV];
+#pragma unroll
+  for (int pi = 0; pi < G::kNV; ++pi) {
+    float x[16];
+    codes16_to_f(sQ + size_t(j0 + pi * G::kRPI + rsub) * DK + c0, x);
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      if (WITH_A) {
+        a0 = fmaf(x[i], ka[i], a0);
+        a1 = fmaf(x[i + 1], ka[i + 1], a1);
+      }
+      b0 = fmaf(x[i], kb[i], b0);
+      b1 = fmaf(x[i + 1], kb[i + 1], b1);
+    }
+    pa[pi] = a0 + a1;
+    pb[pi] = b0 + b1;
+  }
+  a = WITH_A ? reduce_rows<G::kNV, G::kLPR>(pa, lane) : 0.f;
+  b = reduce_rows<G::kNV, G::kLPR>(pb, lane);
+  jl = j0 + reduced_index<G::kNV, G::kLPR>(lane) * G::kRPI + rsub;
+  const float s = sScale[jl];
+  a *= s;
+  b *= s;
+}
+
+// Folds nent log entries into the warp's 16 rows of an int8 base:
+//   x = deq(code) * dec + sum_e u_e[row] kt_e,  deq(code) = code * scale,
+// with kt_e the entries' decayed keys and dec the base's decay per key
+// channel, both staged in shared memory.  The rows are then requantized
+// into (gCodes, gScale), or written as fp32 into gOut when it is non-null.
+template <int DK, typename TU>
+__device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sScale, const TU* sU,
+                                             const float* sKt, const float* sDec, int nent, int L,
+                                             int j0, int lane, int8_t* gCodes, float* gScale,
+                                             float* gOut) {
+  using G = QRows<DK>;
+  const int c0 = (lane % G::kLPR) * G::kCodes;
+  const int rsub = lane / G::kLPR;
+  float d[16];
+  load_f<16>(sDec + c0, d);
+  float acc[G::kNV][16];
+#pragma unroll
+  for (int pi = 0; pi < G::kNV; ++pi) {
+    const int row = j0 + pi * G::kRPI + rsub;
+    codes16_to_f(sQ + size_t(row) * DK + c0, acc[pi]);
+    const float s = sScale[row];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[pi][i] = (acc[pi][i] * s) * d[i];
+  }
+  for (int e = 0; e < nent; ++e) {
+    float kt[16];
+    load_f<16>(sKt + size_t(e) * DK + c0, kt);
+#pragma unroll
+    for (int pi = 0; pi < G::kNV; ++pi) {
+      const float ui = to_f(sU[su_offset(j0 + pi * G::kRPI + rsub, e, L)]);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[pi][i] = fmaf(ui, kt[i], acc[pi][i]);
+    }
+  }
+#pragma unroll
+  for (int pi = 0; pi < G::kNV; ++pi) {
+    const int row = j0 + pi * G::kRPI + rsub;
+    if (gOut != nullptr) {
+      float4* o = reinterpret_cast<float4*>(gOut + size_t(row) * DK + c0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o[q] = make_float4(acc[pi][4 * q], acc[pi][4 * q + 1], acc[pi][4 * q + 2], acc[pi][4 * q + 3]);
+    } else {
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(acc[pi][i]));
+      m = row_max<G::kLPR>(m);
+      float sc;
+      const uint4 w = quantize16(acc[pi], m, &sc);
+      *reinterpret_cast<uint4*>(gCodes + size_t(row) * DK + c0) = w;
+      if (lane % G::kLPR == 0) gScale[row] = sc;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ step
 //
 // A head's rows may be split over SPLIT = DV / ROWS CTAs (blockIdx.x =
@@ -359,13 +460,15 @@ __device__ __forceinline__ void merge_rows_fused(const float* sS, const TU* sU, 
 // log-decay bookkeeping and the per-entry weights are computed together, a
 // second barrier publishes them, and each warp streams its rows.
 
-template <int VAR, int DK, int DV, int ROWS, typename TIn>
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB = float>
 struct StepLayout {
   using TU = typename LogU<VAR, TIn>::type;
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
-  size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offBar, total;
+  static constexpr bool Q8 = std::is_same<TB, int8_t>::value;
+  size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offScale,
+      offKt, offBar, total;
   __host__ __device__ explicit StepLayout(int L) {
-    offU = Tile<DK, ROWS>::kTileBytes;
+    offU = Tile<DK, ROWS, TB>::kTileBytes;
     offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
     offG = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
     offQr = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
@@ -377,18 +480,23 @@ struct StepLayout {
     offW = offVec + align_up(size_t(4 * DK + 2 * GW) * 4, 128);
     offZ = offW + align_up(size_t(L) * 4, 16);
     offScal = offZ + align_up(size_t(L) * 4, 16);
-    offBar = offScal + 64;
-    total = offBar + 8 * (Tile<DK, ROWS>::kChunks + 1);
+    // int8 base: the CTA's row scales, and for the fused merge the decayed
+    // keys of every entry [L][DK] plus the base decay [DK]
+    offScale = offScal + 64;
+    offKt = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
+    offBar = offKt + (Q8 ? align_up(size_t(L + 1) * DK * 4, 128) : 0);
+    total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
   }
 };
 
-template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
-__global__ void __launch_bounds__(Tile<DK, ROWS>::kThreads)
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB, bool FUSED>
+__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads)
 dl_step_kernel(const StepParams p, const FillParam fp) {
-  using Tl = Tile<DK, ROWS>;
+  using Tl = Tile<DK, ROWS, TB>;
   using TU = typename LogU<VAR, TIn>::type;
+  constexpr bool Q8 = std::is_same<TB, int8_t>::value;
   constexpr int SPLIT = DV / ROWS;
-  constexpr int GW = StepLayout<VAR, DK, DV, ROWS, TIn>::GW;
+  constexpr int GW = StepLayout<VAR, DK, DV, ROWS, TIn, TB>::GW;
   constexpr int NT = Tl::kThreads;
   constexpr int NW = Tl::kWarps;
   constexpr int CPL = Tl::kCPL;
@@ -398,8 +506,8 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int L = p.L;
   const int GS = g_stride(VAR, L, DK);
-  const StepLayout<VAR, DK, DV, ROWS, TIn> lay(L);
-  float* sS = reinterpret_cast<float*>(smem);                 // [ROWS][DK]
+  const StepLayout<VAR, DK, DV, ROWS, TIn, TB> lay(L);
+  TB* sS = reinterpret_cast<TB*>(smem);                       // [ROWS][DK]
   TU* sU = reinterpret_cast<TU*>(smem + lay.offU);            // [ROWS/32][L][32]
   TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);          // [L][DK]
   float* sG = reinterpret_cast<float*>(smem + lay.offG);      // [L][GW]
@@ -417,6 +525,9 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   float* sZ = reinterpret_cast<float*>(smem + lay.offZ);      // per-entry weights on q / r
   float* sScal = reinterpret_cast<float*>(smem + lay.offScal);  // [0] k.q / bonus [1] beta
                                                                 // [2] e^{g_t} [3] decay (GDN)
+  float* sScale = reinterpret_cast<float*>(smem + lay.offScale);  // int8 base: row scales
+  float* sKt = reinterpret_cast<float*>(smem + lay.offKt);        // int8 fused merge: [L][DK]
+  float* sDecF = sKt + size_t(L) * DK;                            // and the base decay [DK]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
   uint64_t* barLog = &bars[Tl::kChunks];
 
@@ -435,7 +546,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   const bool merge_now = FUSED && (f + 1 == L);
   const bool appender = (part == 0) && !merge_now;
 
-  const float* gS = p.base + (head * size_t(DV) + r0) * DK;
+  const TB* gS = static_cast<const TB*>(p.base) + (head * size_t(DV) + r0) * DK;
   TU* gU = static_cast<TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
   TIn* gK = static_cast<TIn*>(p.logK) + head * size_t(L) * DK;
   float* gG = p.logG + head * size_t(GS);
@@ -464,7 +575,9 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one row block
     const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
     const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
-    mbar_arrive_expect_tx(barLog, 2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg);
+    const uint32_t bs = Q8 ? ROWS * 4u : 0u;
+    mbar_arrive_expect_tx(barLog, 2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg + bs);
+    if (Q8) tma_load_1d(sScale, p.scale + head * DV + r0, bs, barLog);
     tma_load_1d(sQr, static_cast<const TIn*>(p.q) + head * DK, bq, barLog);
     tma_load_1d(sKr, static_cast<const TIn*>(p.k) + head * DK, bq, barLog);
     tma_load_1d(sVr, static_cast<const TIn*>(p.v) + head * DV + r0, bv, barLog);
@@ -548,14 +661,22 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   // ---- one pass over this warp's 16 rows of S_b
   const int j0 = warp * Tl::kRowsPerWarp;  // local row index
   uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
-  if (!mbar_wait(barMine, 0, p.err, int(head))) {
+  const bool mine = mbar_wait(barMine, 0, p.err, int(head));
+  // the int8 fused merge synchronises the whole CTA below, so there every
+  // warp has to know whether all tile chunks arrived
+  const bool all_in = (Q8 && merge_now) ? __syncthreads_and(mine) : mine;
+  if (!all_in) {
     mbar_wait(barMine, 0, nullptr, 0);
     return;
   }
   float a, b;
   int jl;  // local row this lane finishes
-  rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
-                                  (VAR == kVarGDN) ? sq : sQh, a, b, jl);
+  if constexpr (Q8)
+    rows_gemv_q8<DK, VAR != kVarRWKV6>(sS, sScale, j0, lane, (VAR == kVarGDN) ? sk : sKh,
+                                       (VAR == kVarGDN) ? sq : sQh, a, b, jl);
+  else
+    rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
+                                    (VAR == kVarGDN) ? sq : sQh, a, b, jl);
   float u, o;
   row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, to_f(sVr[jl]), a, b, u, o);
   if ((lane & 1) == 0) {
@@ -566,26 +687,46 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       gU[u_offset(0, r0 + jl, f, L, DV)] = Elem<TU>::from_f(u);
   }
   if (!merge_now) return;
-  __syncwarp();
-  merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,
-                                     p.base + (head * size_t(DV) + r0) * DK);
+  if constexpr (Q8) {
+    // every warp's u_t rows are in slot f; stage the decayed keys of the
+    // L entries and the base decay once for the CTA, then fold and requantize
+    __syncthreads();
+    for (int x = tid; x < (f + 1) * DK; x += NT) {
+      const int i = x / DK;
+      const int c = x % DK;
+      float kt = to_f(sK[x]);
+      if (i < f) kt *= expf(sGt[GW > 1 ? c : 0] - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
+      sKt[x] = kt;
+    }
+    for (int c = tid; c < DK; c += NT) sDecF[c] = (GW == 1) ? sScal[2] : expf(sGt[c]);
+    __syncthreads();
+    fold_rows_q8<DK, TU>(sS, sScale, sU, sKt, sDecF, f + 1, L, j0, lane,
+                         static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
+                         p.scale + head * size_t(DV) + r0, nullptr);
+  } else {
+    __syncwarp();
+    merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,
+                                       static_cast<float*>(p.base) + (head * size_t(DV) + r0) * DK);
+  }
 }
 
 // ----------------------------------------------------------- merge / materialize
 
-template <int VAR, int DK, int DV, int ROWS, typename TIn>
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB = float>
 struct MergeLayout {
   using TU = typename LogU<VAR, TIn>::type;
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
-  size_t offU, offK, offKt, offG, offDec, offBar, total;
+  static constexpr bool Q8 = std::is_same<TB, int8_t>::value;
+  size_t offU, offK, offKt, offG, offDec, offScale, offBar, total;
   __host__ __device__ explicit MergeLayout(int L) {
-    offU = Tile<DK, ROWS>::kTileBytes;
+    offU = Tile<DK, ROWS, TB>::kTileBytes;
     offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
     offKt = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
     offG = offKt + align_up(size_t(L) * DK * 4, 128);
     offDec = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
-    offBar = offDec + align_up(size_t(DK) * 4, 128);
-    total = offBar + 8 * (Tile<DK, ROWS>::kChunks + 1);
+    offScale = offDec + align_up(size_t(DK) * 4, 128);
+    offBar = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
+    total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
   }
 };
 
@@ -593,13 +734,14 @@ struct MergeLayout {
 // DV / ROWS CTAs, as in the step).  With a list, the fills come from the
 // list and only part 0 empties the log, so split CTAs never race on it;
 // without a list the kernel runs unsplit and reads the device fill.
-template <int VAR, int DK, int DV, int ROWS, typename TIn>
-__global__ void __launch_bounds__(Tile<DK, ROWS>::kThreads)
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB>
+__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads)
 dl_merge_kernel(const MergeParams p, const SeqList list) {
-  using Tl = Tile<DK, ROWS>;
+  using Tl = Tile<DK, ROWS, TB>;
   using TU = typename LogU<VAR, TIn>::type;
+  constexpr bool Q8 = std::is_same<TB, int8_t>::value;
   constexpr int SPLIT = DV / ROWS;
-  constexpr int GW = MergeLayout<VAR, DK, DV, ROWS, TIn>::GW;
+  constexpr int GW = MergeLayout<VAR, DK, DV, ROWS, TIn, TB>::GW;
   constexpr int NT = Tl::kThreads;
   constexpr int NV = Tl::kNV;
   constexpr int LPR = Tl::kLPR;
@@ -623,20 +765,21 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
   if (p.mode == 0 && f != L) return;
   if (p.mode == 1 && f == 0) return;
 
-  const MergeLayout<VAR, DK, DV, ROWS, TIn> lay(L);
-  float* sS = reinterpret_cast<float*>(smem);
+  const MergeLayout<VAR, DK, DV, ROWS, TIn, TB> lay(L);
+  TB* sS = reinterpret_cast<TB*>(smem);
   TU* sU = reinterpret_cast<TU*>(smem + lay.offU);
   TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);
   float* sKt = reinterpret_cast<float*>(smem + lay.offKt);
   float* sG = reinterpret_cast<float*>(smem + lay.offG);
   float* sDec = reinterpret_cast<float*>(smem + lay.offDec);
+  float* sScale = reinterpret_cast<float*>(smem + lay.offScale);  // int8 base: row scales
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
   uint64_t* barLog = &bars[Tl::kChunks];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const float* gS = p.base + (head * size_t(DV) + r0) * DK;
+  const TB* gS = static_cast<const TB*>(p.base) + (head * size_t(DV) + r0) * DK;
   const TU* gU = static_cast<const TU*>(p.logU) + u_offset(head, r0, 0, L, DV);
   const TIn* gK = static_cast<const TIn*>(p.logK) + head * size_t(L) * DK;
   const float* gG = p.logG + head * size_t(GS);
@@ -655,20 +798,26 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
   } else if (warp == 1 && lane == 0) {
     mbar_init(barLog, 1);
     fence_mbar_init();
-    if (f > 0) {
+    if (f > 0 || Q8) {
       const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one row block
       const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
-      const uint32_t bg = g_copy_bytes<VAR, DK>(f);
-      mbar_arrive_expect_tx(barLog, bu * uint32_t(ROWS / kURows) + bk + bg);
-      for (int rb = 0; rb < ROWS / kURows; ++rb)
-        tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, rb * kURows, 0, L, DV), bu, barLog);
-      tma_load_1d(sK, gK, bk, barLog);
-      tma_load_1d(sG, gG, bg, barLog);
+      const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
+      const uint32_t bs = Q8 ? ROWS * 4u : 0u;
+      mbar_arrive_expect_tx(barLog, bu * uint32_t(ROWS / kURows) + bk + bg + bs);
+      if (Q8) tma_load_1d(sScale, p.scale + head * DV + r0, bs, barLog);
+      if (f > 0) {
+        for (int rb = 0; rb < ROWS / kURows; ++rb)
+          tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, rb * kURows, 0, L, DV), bu,
+                      barLog);
+        tma_load_1d(sK, gK, bk, barLog);
+        tma_load_1d(sG, gG, bg, barLog);
+      }
     }
   }
   __syncthreads();
+  const bool log_copies = f > 0 || Q8;
   bool ok = true;
-  if (f > 0) ok = mbar_wait(barLog, 0, p.err, int(head));
+  if (log_copies) ok = mbar_wait(barLog, 0, p.err, int(head));
   // decay of the base and decayed keys k-tilde_i = k_i o e^{g_last - g_i},
   // one (entry, channel) pair per thread
   for (int c = tid; c < DK; c += NT)
@@ -681,7 +830,7 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
   }
   if (tid == 0 && part == 0 && p.mode != 2) p.fill[head] = 0;
   if (!__syncthreads_and(ok)) {
-    if (f > 0) mbar_wait(barLog, 0, nullptr, 0);
+    if (log_copies) mbar_wait(barLog, 0, nullptr, 0);
     for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
     return;
   }
@@ -692,13 +841,22 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
     mbar_wait(barMine, 0, nullptr, 0);
     return;
   }
+  if constexpr (Q8) {
+    const bool to_fp32 = (p.mode == 2);
+    fold_rows_q8<DK, TU>(sS, sScale, sU, sKt, sDec, f, L, j0, lane,
+                         static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
+                         p.scale + head * size_t(DV) + r0,
+                         to_fp32 ? p.out + (head * size_t(DV) + r0) * DK : nullptr);
+    return;
+  }
   const int c0 = (lane % LPR) * 4;
   const int rsub = lane / LPR;
   const float4 dec = *reinterpret_cast<const float4*>(sDec + c0);
   float4 acc[NV];
 #pragma unroll
   for (int pi = 0; pi < NV; ++pi) {
-    const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + pi * RPI + rsub) * DK + c0);
+    const float4 s4 =
+        *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(sS) + size_t(j0 + pi * RPI + rsub) * DK + c0);
     acc[pi] = make_float4(s4.x * dec.x, s4.y * dec.y, s4.z * dec.z, s4.w * dec.w);
   }
   for (int i = 0; i < f; ++i) {

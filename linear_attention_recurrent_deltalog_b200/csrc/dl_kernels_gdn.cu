@@ -1,6 +1,8 @@
-// Launchers for the GDN instantiations of the DeltaLog kernels.
+// Launchers for the GDN instantiations of the DeltaLog kernels (fp32 base,
+// and the eager step).
 #include "dl_launch.cuh"
 
 namespace dl {
-DL_DEFINE_VARIANT_LAUNCHERS(kVarGDN)
+DL_DEFINE_BASE_LAUNCHERS(kVarGDN, float)
+DL_DEFINE_EAGER_LAUNCHER(kVarGDN)
 }  // namespace dl

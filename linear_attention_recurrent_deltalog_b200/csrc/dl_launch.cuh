@@ -19,7 +19,7 @@ struct Shape {
   int dv;
   int bf16;        // 1: q/k/v are bf16, 0: fp32
   int split;       // step kernel: work items per head (1, 2 or 4; d_v / split >= 32)
-  int persistent;  // 1: persistent warp-specialised step kernel when its ring fits
+  int persistent;  // 1: persistent warp-specialised step kernel when its ring fits (fp32 base)
 };
 
 inline bool split_ok(int dv, int split) {
@@ -47,39 +47,40 @@ inline cudaError_t prepare_kernel(Kern kern, std::atomic<unsigned long long>& do
   return cudaSuccess;
 }
 
-template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB, bool FUSED>
 cudaError_t launch_step_t(const StepParams& p, const FillParam& fp, unsigned nheads,
                           cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
-  auto kern = dl_step_kernel<VAR, DK, DV, ROWS, TIn, FUSED>;
+  auto kern = dl_step_kernel<VAR, DK, DV, ROWS, TIn, TB, FUSED>;
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
-  const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn>(p.L).total;
+  const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn, TB>(p.L).total;
   kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p, fp);
   return cudaGetLastError();
 }
 
-template <int VAR, int DK, int DV, int ROWS, typename TIn>
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB>
 cudaError_t launch_merge_rows(const MergeParams& p, const SeqList& list, unsigned nheads,
                               cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
-  auto kern = dl_merge_kernel<VAR, DK, DV, ROWS, TIn>;
+  auto kern = dl_merge_kernel<VAR, DK, DV, ROWS, TIn, TB>;
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
-  const size_t smem = MergeLayout<VAR, DK, DV, ROWS, TIn>(p.L).total;
+  const size_t smem = MergeLayout<VAR, DK, DV, ROWS, TIn, TB>(p.L).total;
   kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p, list);
   return cudaGetLastError();
 }
 
 // Split heads into 64-row CTAs whenever no CTA has to read a fill another
 // CTA of the launch may reset (a listed merge, or materialize).
-template <int VAR, int DK, int DV, typename TIn>
+template <int VAR, int DK, int DV, typename TIn, typename TB>
 cudaError_t launch_merge_t(const MergeParams& p, const SeqList& list, unsigned nheads,
                            cudaStream_t s) {
   if constexpr (DV >= 128) {
-    if (p.use_list || p.mode == 2) return launch_merge_rows<VAR, DK, DV, DV / 2, TIn>(p, list, nheads, s);
+    if (p.use_list || p.mode == 2)
+      return launch_merge_rows<VAR, DK, DV, DV / 2, TIn, TB>(p, list, nheads, s);
   }
-  return launch_merge_rows<VAR, DK, DV, DV, TIn>(p, list, nheads, s);
+  return launch_merge_rows<VAR, DK, DV, DV, TIn, TB>(p, list, nheads, s);
 }
 
 template <int VAR, int DK, int DV, typename TIn>
@@ -108,35 +109,39 @@ inline cudaError_t dispatch_shape(const Shape& sh, F&& f) {
   return cudaErrorInvalidValue;
 }
 
-// Per-variant entry points (defined in dl_kernels_<variant>.cu).
-template <int VAR>
+// Per-variant, per-base-type entry points (defined in dl_kernels_<variant>.cu
+// for the fp32 base and dl_kernels_<variant>_q8.cu for the int8 base).
+template <int VAR, typename TB>
 cudaError_t launch_step(const Shape& sh, bool fused, const StepParams& p, const FillParam& fp,
                         unsigned nheads, cudaStream_t s);
-template <int VAR>
+template <int VAR, typename TB>
 cudaError_t launch_merge(const Shape& sh, const MergeParams& p, const SeqList& list,
                          unsigned nheads, cudaStream_t s);
 template <int VAR>
 cudaError_t launch_eager(const Shape& sh, const EagerParams& p, unsigned nheads, cudaStream_t s);
 
 // Shared-memory bytes a launch needs (host-side check before launching).
-template <int VAR>
+template <int VAR, typename TB>
 size_t step_smem_bytes(const Shape& sh, int L);
-template <int VAR>
+template <int VAR, typename TB>
 size_t merge_smem_bytes(const Shape& sh, int L);
 
+#define DL_DECLARE_BASE_LAUNCHERS(VAR, TB)                                                     \
+  template <>                                                                                  \
+  cudaError_t launch_step<VAR, TB>(const Shape&, bool, const StepParams&, const FillParam&,    \
+                                   unsigned, cudaStream_t);                                    \
+  template <>                                                                                  \
+  cudaError_t launch_merge<VAR, TB>(const Shape&, const MergeParams&, const SeqList&, unsigned, \
+                                    cudaStream_t);                                             \
+  template <>                                                                                  \
+  size_t step_smem_bytes<VAR, TB>(const Shape&, int);                                          \
+  template <>                                                                                  \
+  size_t merge_smem_bytes<VAR, TB>(const Shape&, int);
 #define DL_DECLARE_VARIANT_LAUNCHERS(VAR)                                                     \
+  DL_DECLARE_BASE_LAUNCHERS(VAR, float)                                                        \
+  DL_DECLARE_BASE_LAUNCHERS(VAR, int8_t)                                                       \
   template <>                                                                                 \
-  cudaError_t launch_step<VAR>(const Shape&, bool, const StepParams&, const FillParam&, unsigned, \
-                               cudaStream_t);                                                   \
-  template <>                                                                                 \
-  cudaError_t launch_merge<VAR>(const Shape&, const MergeParams&, const SeqList&, unsigned,    \
-                                cudaStream_t);                                                \
-  template <>                                                                                 \
-  cudaError_t launch_eager<VAR>(const Shape&, const EagerParams&, unsigned, cudaStream_t);    \
-  template <>                                                                                 \
-  size_t step_smem_bytes<VAR>(const Shape&, int);                                             \
-  template <>                                                                                 \
-  size_t merge_smem_bytes<VAR>(const Shape&, int);
+  cudaError_t launch_eager<VAR>(const Shape&, const EagerParams&, unsigned, cudaStream_t);
 
 DL_DECLARE_VARIANT_LAUNCHERS(kVarGDN)
 DL_DECLARE_VARIANT_LAUNCHERS(kVarKDA)
@@ -195,30 +200,34 @@ cudaError_t launch_step_persistent_t(const StepParams& p, const FillParam& fp, u
   return cudaGetLastError();
 }
 
-template <int VAR, int DK, int DV, int ROWS, typename T, bool FUSED>
+template <int VAR, int DK, int DV, int ROWS, typename T, typename TB, bool FUSED>
 cudaError_t launch_step_rows(bool persistent, const StepParams& p, const FillParam& fp, unsigned n,
                              cudaStream_t s) {
-  if (persistent) {
-    const cudaError_t e = launch_step_persistent_t<VAR, DK, DV, ROWS, T, FUSED>(p, fp, n, s);
-    if (e != cudaErrorNotSupported) return e;
+  if constexpr (std::is_same<TB, float>::value) {
+    if (persistent) {
+      const cudaError_t e = launch_step_persistent_t<VAR, DK, DV, ROWS, T, FUSED>(p, fp, n, s);
+      if (e != cudaErrorNotSupported) return e;
+    }
   }
-  return launch_step_t<VAR, DK, DV, ROWS, T, FUSED>(p, fp, n, s);
+  return launch_step_t<VAR, DK, DV, ROWS, T, TB, FUSED>(p, fp, n, s);
 }
 
-template <int VAR, int DK, int DV, typename T, bool FUSED>
+template <int VAR, int DK, int DV, typename T, typename TB, bool FUSED>
 cudaError_t launch_step_split(int split, bool persistent, const StepParams& p, const FillParam& fp,
                               unsigned n, cudaStream_t s) {
-  if (split == 1) return launch_step_rows<VAR, DK, DV, DV, T, FUSED>(persistent, p, fp, n, s);
+  if (split == 1) return launch_step_rows<VAR, DK, DV, DV, T, TB, FUSED>(persistent, p, fp, n, s);
   if constexpr (DV / 2 >= 32) {
-    if (split == 2) return launch_step_rows<VAR, DK, DV, DV / 2, T, FUSED>(persistent, p, fp, n, s);
+    if (split == 2)
+      return launch_step_rows<VAR, DK, DV, DV / 2, T, TB, FUSED>(persistent, p, fp, n, s);
   }
   if constexpr (DV / 4 >= 32) {
-    if (split == 4) return launch_step_rows<VAR, DK, DV, DV / 4, T, FUSED>(persistent, p, fp, n, s);
+    if (split == 4)
+      return launch_step_rows<VAR, DK, DV, DV / 4, T, TB, FUSED>(persistent, p, fp, n, s);
   }
   return cudaErrorInvalidValue;
 }
 
-template <int VAR>
+template <int VAR, typename TB>
 struct StepRun {
   const StepParams& p;
   const FillParam& fp;
@@ -229,18 +238,18 @@ struct StepRun {
   bool persistent;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    return fused ? launch_step_split<VAR, DK, DV, T, true>(split, persistent, p, fp, n, s)
-                 : launch_step_split<VAR, DK, DV, T, false>(split, persistent, p, fp, n, s);
+    return fused ? launch_step_split<VAR, DK, DV, T, TB, true>(split, persistent, p, fp, n, s)
+                 : launch_step_split<VAR, DK, DV, T, TB, false>(split, persistent, p, fp, n, s);
   }
 };
-template <int VAR>
+template <int VAR, typename TB>
 struct MergeRun {
   const MergeParams& p;
   const SeqList& list;
   unsigned n;
   cudaStream_t s;
   template <int DK, int DV, typename T>
-  cudaError_t run() { return launch_merge_t<VAR, DK, DV, T>(p, list, n, s); }
+  cudaError_t run() { return launch_merge_t<VAR, DK, DV, T, TB>(p, list, n, s); }
 };
 template <int VAR>
 struct EagerRun {
@@ -250,7 +259,7 @@ struct EagerRun {
   template <int DK, int DV, typename T>
   cudaError_t run() { return launch_eager_t<VAR, DK, DV, T>(p, n, s); }
 };
-template <int VAR>
+template <int VAR, typename TB>
 struct StepSmem {
   int L;
   int split;
@@ -258,55 +267,57 @@ struct StepSmem {
   template <int DK, int DV, typename T>
   cudaError_t run() {
     out = 0;
-    if (split == 1) out = StepLayout<VAR, DK, DV, DV, T>(L).total;
+    if (split == 1) out = StepLayout<VAR, DK, DV, DV, T, TB>(L).total;
     if constexpr (DV / 2 >= 32) {
-      if (split == 2) out = StepLayout<VAR, DK, DV, DV / 2, T>(L).total;
+      if (split == 2) out = StepLayout<VAR, DK, DV, DV / 2, T, TB>(L).total;
     }
     if constexpr (DV / 4 >= 32) {
-      if (split == 4) out = StepLayout<VAR, DK, DV, DV / 4, T>(L).total;
+      if (split == 4) out = StepLayout<VAR, DK, DV, DV / 4, T, TB>(L).total;
     }
     return out ? cudaSuccess : cudaErrorInvalidValue;
   }
 };
-template <int VAR>
+template <int VAR, typename TB>
 struct MergeSmem {
   int L;
   size_t out;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    out = MergeLayout<VAR, DK, DV, DV, T>(L).total;
+    out = MergeLayout<VAR, DK, DV, DV, T, TB>(L).total;
     return cudaSuccess;
   }
 };
 
-#define DL_DEFINE_VARIANT_LAUNCHERS(VAR)                                                   \
+#define DL_DEFINE_BASE_LAUNCHERS(VAR, TB)                                                   \
   template <>                                                                              \
-  cudaError_t launch_step<VAR>(const Shape& sh, bool fused, const StepParams& p,           \
-                               const FillParam& fp, unsigned nheads, cudaStream_t s) {     \
-    StepRun<VAR> f{p, fp, nheads, s, fused, sh.split, sh.persistent != 0};                                                   \
+  cudaError_t launch_step<VAR, TB>(const Shape& sh, bool fused, const StepParams& p,       \
+                                   const FillParam& fp, unsigned nheads, cudaStream_t s) { \
+    StepRun<VAR, TB> f{p, fp, nheads, s, fused, sh.split, sh.persistent != 0};              \
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
   template <>                                                                              \
-  cudaError_t launch_merge<VAR>(const Shape& sh, const MergeParams& p, const SeqList& list, \
-                                unsigned nheads, cudaStream_t s) {                         \
-    MergeRun<VAR> f{p, list, nheads, s};                                                   \
+  cudaError_t launch_merge<VAR, TB>(const Shape& sh, const MergeParams& p,                 \
+                                    const SeqList& list, unsigned nheads, cudaStream_t s) { \
+    MergeRun<VAR, TB> f{p, list, nheads, s};                                               \
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
+  template <>                                                                              \
+  size_t step_smem_bytes<VAR, TB>(const Shape& sh, int L) {                                \
+    StepSmem<VAR, TB> f{L, sh.split, 0};                                                   \
+    return dispatch_shape(sh, f) == cudaSuccess ? f.out : 0;                               \
+  }                                                                                        \
+  template <>                                                                              \
+  size_t merge_smem_bytes<VAR, TB>(const Shape& sh, int L) {                               \
+    MergeSmem<VAR, TB> f{L, 0};                                                            \
+    return dispatch_shape(sh, f) == cudaSuccess ? f.out : 0;                               \
+  }
+
+#define DL_DEFINE_EAGER_LAUNCHER(VAR)                                                      \
   template <>                                                                              \
   cudaError_t launch_eager<VAR>(const Shape& sh, const EagerParams& p, unsigned nheads,    \
                                 cudaStream_t s) {                                          \
     EagerRun<VAR> f{p, nheads, s};                                                         \
     return dispatch_shape(sh, f);                                                          \
-  }                                                                                        \
-  template <>                                                                              \
-  size_t step_smem_bytes<VAR>(const Shape& sh, int L) {                                    \
-    StepSmem<VAR> f{L, sh.split, 0};                                                                 \
-    return dispatch_shape(sh, f) == cudaSuccess ? f.out : 0;                               \
-  }                                                                                        \
-  template <>                                                                              \
-  size_t merge_smem_bytes<VAR>(const Shape& sh, int L) {                                   \
-    MergeSmem<VAR> f{L, 0};                                                                \
-    return dispatch_shape(sh, f) == cudaSuccess ? f.out : 0;                               \
   }
 
 }  // namespace dl

@@ -145,7 +145,7 @@ dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam 
       const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
       const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
       mbar_expect_tx(&full[s], tile_b + vec_b + bu * uint32_t(ROWS / kURows) + bk + bg);
-      const float* gS = p.base + (head * size_t(DV) + r0) * DK;
+      const float* gS = static_cast<const float*>(p.base) + (head * size_t(DV) + r0) * DK;
 #pragma unroll
       for (int c = 0; c < Tl::kChunks; ++c)
         tma_load_1d_stream(st + size_t(c) * Tl::kChunkBytes, gS + size_t(c) * Tl::kChunkRows * DK,
@@ -303,7 +303,7 @@ dl_step_persistent_kernel(const StepParams p, const int nstage, const FillParam 
     if (merge_now) {
       __syncwarp();
       merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,
-                                         p.base + (head * size_t(DV) + r0) * DK);
+                                         static_cast<float*>(p.base) + (head * size_t(DV) + r0) * DK);
     }
     // Release the stage once every lane of this warp is done with it.  The
     // fused merge wrote slot f of the staged log through the generic proxy;

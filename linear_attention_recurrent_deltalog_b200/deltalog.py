@@ -34,6 +34,7 @@ DL_MERGE_FULL, DL_MERGE_ALL = 0, 1
 DL_FLAG_FUSED_MERGE = 1
 DL_FLAG_PERSISTENT = 2
 DL_FLAG_KLA = 4
+DL_FLAG_BASE_Q8 = 8
 
 VARIANT_IDS = {"gdn": DL_GDN, "kda": DL_KDA, "rwkv6": DL_RWKV6}
 DTYPE_IDS = {"f32": DL_F32, "bf16": DL_BF16}
@@ -133,11 +134,15 @@ class Config:
     step_split: int = 0
     persistent: bool = False
     kla_eps: Optional[float] = None  # set: beta carries the KLA gate eta
+    base: str = "f32"                # "f32", or "q8": int8 codes + row scales
 
     def c(self) -> dl_config:
+        if self.base not in ("f32", "q8"):
+            raise ValueError(f"base must be 'f32' or 'q8', not {self.base!r}")
         flags = (DL_FLAG_FUSED_MERGE if self.fused_merge else 0) | \
             (DL_FLAG_PERSISTENT if self.persistent else 0) | \
-            (DL_FLAG_KLA if self.kla_eps is not None else 0)
+            (DL_FLAG_KLA if self.kla_eps is not None else 0) | \
+            (DL_FLAG_BASE_Q8 if self.base == "q8" else 0)
         return dl_config(VARIANT_IDS[self.variant], self.B, self.H, self.d_k, self.d_v, self.L,
                          DTYPE_IDS[self.in_dtype], flags, self.step_split,
                          0.0 if self.kla_eps is None else float(self.kla_eps))
@@ -318,6 +323,28 @@ class DeltaLogState:
 
     def fill(self):
         return dl_state_fill(self.handle, self.cfg)
+
+    # Views of an int8 base in the layout deltalog.h documents: codes
+    # [B*H, d_v, d_k], then the fp32 row scales [B*H, d_v] at the next
+    # 256-byte boundary.
+    def _scale_offset(self) -> int:
+        n = self.cfg.heads * self.cfg.d_v * self.cfg.d_k
+        return (n + 255) // 256 * 256
+
+    def base_codes(self) -> torch.Tensor:
+        if self.cfg.base != "q8":
+            raise ValueError("base_codes: the base is fp32")
+        c = self.cfg
+        raw = self.base.view(torch.uint8)
+        return raw[:c.heads * c.d_v * c.d_k].view(torch.int8).view(c.heads, c.d_v, c.d_k)
+
+    def base_scales(self) -> torch.Tensor:
+        if self.cfg.base != "q8":
+            raise ValueError("base_scales: the base is fp32")
+        c = self.cfg
+        off = self._scale_offset()
+        raw = self.base.view(torch.uint8)
+        return raw[off:off + c.heads * c.d_v * 4].view(torch.float32).view(c.heads, c.d_v)
 
     def device_error(self, clear: bool = False, stream=None):
         return dl_device_error(self.handle, clear, stream)

@@ -173,3 +173,113 @@ def heads_covering_phases(w: wl.Workload, n: int, L: Optional[int] = None) -> np
     rest = wl.sample_heads(w, n)
     allh = np.unique(np.concatenate([np.array(picked, dtype=np.int64), rest]))
     return allh
+
+
+# ------------------------------------------------------------- int8 base
+
+@dataclasses.dataclass
+class Q8Result:
+    reset_exact: bool        # Q(S0) codes and scales bit-identical to the oracle's
+    out_err: float           # as in run_parity, against the windowed oracle
+    state_err: float         # materialized state against the windowed oracle
+    code_excess: float       # max over requantized elements of
+                             #   |code_gpu - x inv| - 0.5 - delta  (<= 0 passes)
+    scale_excess: float      # max of |scale_gpu - scale_ref| - allowed  (<= 0 passes)
+    mismatch_frac: float     # fraction of requantized codes that differ
+    windows: int             # window ends checked
+
+
+def _lib_rows(S, rec):
+    return np.swapaxes(S, -1, -2) if rec else S
+
+
+def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence[int]] = None,
+                  fused: bool = True, split: int = 0, merge_all_at: Sequence[int] = (),
+                  resync: bool = True, snap_every: int = 8, workers: Optional[int] = 0,
+                  device="cuda") -> Q8Result:
+    """The int8-base path against the windowed oracle (oracle.run_windowed's
+    definition, stepped here one step at a time for the sampled heads).
+
+    At every window end the GPU's new codes must be a correct rounding of
+    the oracle's pre-quantization value x: |code - x inv| <= 0.5 + delta with
+    delta = 2 eps inv, eps = STATE_TOL * max|x| over the head (the GPU's x
+    and amax may differ from the oracle's by the state tolerance).  With
+    ``resync`` the oracle's codes and scales are then written into the GPU
+    base for those heads, so every window starts from identical values and
+    outputs and states are held to the fp32 tolerances."""
+    T = w.T if T is None else T
+    BH, dk, dv, H, L = w.heads, w.d_k, w.d_v, w.H, w.L
+    rec = w.variant == wl.RWKV6
+    heads = np.arange(BH) if heads is None else np.asarray(heads, dtype=np.int64)
+    heads_t = torch.from_numpy(heads).to(device)
+    S0 = cached_initial_state(w)
+    fill0 = wl.fill_offsets(w)
+    bonus = wl.rwkv6_bonus(w) if rec else None
+    bonus_d = None if bonus is None else torch.from_numpy(bonus).to(device).reshape(-1)
+    bon = None if bonus is None else bonus[heads % H]
+    cfg = dlb.Config(w.variant, w.B, H, dk, dv, L, w.in_dtype, fused_merge=fused, step_split=split,
+                     kla_eps=w.kla_eps, base="q8")
+    st = dlb.DeltaLogState(cfg, device=device)
+    st.reset(torch.from_numpy(S0).to(device).reshape(-1), fill0.tolist())
+    S0h = S0.reshape(BH, dv, dk)[heads]
+    c0, s0 = oracle.quantize_rows(S0h)
+    g_codes = st.base_codes().index_select(0, heads_t).cpu().numpy()
+    g_scales = st.base_scales().index_select(0, heads_t).cpu().numpy()
+    reset_exact = bool(np.array_equal(g_codes, c0) and np.array_equal(g_scales, s0))
+    S = _lib_rows(oracle.dequantize_rows(c0, s0), rec).copy()      # recurrence orientation
+    fill = fill0[heads // H].astype(np.int64)
+    o = torch.empty(BH * dv, dtype=torch.float32, device=device)
+    S_out = torch.empty(BH * dv * dk, dtype=torch.float32, device=device)
+    out_err = state_err = 0.0
+    code_excess = scale_excess = -np.inf
+    mismatches = total = windows = 0
+    forced = set(int(x) for x in merge_all_at)
+    for s in wl.StepStream(w, T, workers=workers):
+        q, k, v, dec, beta = step_to_device(s, device)
+        n = s.t + 1
+        st.step(q, k, v, dec, beta, bonus_d, o)
+        if not fused:
+            st.merge(dlb.DL_MERGE_FULL)
+        if n in forced:
+            st.merge(dlb.DL_MERGE_ALL)
+        o_gpu = o.view(BH, dv).index_select(0, heads_t).cpu().numpy().astype(np.float64)
+        flat = lambda x: None if x is None else x.reshape((BH,) + x.shape[2:])[heads][:, None]
+        step = types.SimpleNamespace(q=flat(s.q), k=flat(s.k), v=flat(s.v), decay=flat(s.decay),
+                                     beta=flat(s.beta))
+        res = oracle.run_eager(w.variant, S, [step], bonus=bon, kla_eps=w.kla_eps)
+        S = res.S
+        out_err = max(out_err, _rel(o_gpu, res.outputs[0]))
+        fill += 1
+        ended = (fill > 0) if n in forced else (fill == L)
+        idx = np.nonzero(ended)[0]
+        if idx.size:
+            pre = _lib_rows(S[idx], rec)
+            codes, scales = oracle.quantize_rows(pre)
+            inv = oracle.row_inverse(pre).astype(np.float64)
+            gidx = torch.from_numpy(heads[idx]).to(device)
+            gc = st.base_codes().index_select(0, gidx).cpu().numpy().astype(np.float64)
+            gs = st.base_scales().index_select(0, gidx).cpu().numpy().astype(np.float64)
+            eps = STATE_TOL * np.max(np.abs(pre), axis=(1, 2), keepdims=True)
+            delta = 2.0 * eps * inv[..., None] + 1e-6
+            dev_c = np.abs(gc - pre * inv[..., None]) - 0.5 - delta
+            code_excess = max(code_excess, float(np.max(dev_c)))
+            dev_s = np.abs(gs - scales) - (eps[..., 0] / 127.0 * 1.0001 + 1e-30)
+            scale_excess = max(scale_excess, float(np.max(dev_s)))
+            mismatches += int(np.count_nonzero(gc != codes))
+            total += codes.size
+            windows += idx.size
+            if resync:
+                st.base_codes().index_copy_(0, gidx, torch.from_numpy(codes).to(device))
+                st.base_scales().index_copy_(0, gidx, torch.from_numpy(scales).to(device))
+            S[idx] = _lib_rows(oracle.dequantize_rows(codes, scales), rec)
+            fill[idx] = 0
+        if n % snap_every == 0 or n == T:
+            st.materialize(S_out)
+            Sg = S_out.view(BH, dv, dk).index_select(0, heads_t).cpu().numpy().astype(np.float64)
+            state_err = max(state_err, _rel(Sg, _lib_rows(S, rec)))
+    torch.cuda.synchronize()
+    code, head = st.device_error()
+    assert code == 0, f"device error {code} at head {head}"
+    st.close()
+    return Q8Result(reset_exact, out_err, state_err, code_excess, scale_excess,
+                    mismatches / max(total, 1), windows)

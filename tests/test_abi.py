@@ -60,6 +60,13 @@ def test_state_bytes_layout():
     assert nl_kda == pad(BH * 16 * 128 * 4) + pad(BH * 16 * 128 * 2) + pad(BH * 16 * 128 * 4)
     _, nl_rw, _ = dlb.dl_state_bytes(cfg(variant="rwkv6", d_k=64, d_v=64, L=32))
     assert nl_rw == pad(BH * 32 * 64 * 2) + pad(BH * 32 * 64 * 2) + pad(BH * 32 * 64 * 4)
+    # int8 base: codes, then the fp32 row scales at the next 256-B boundary;
+    # the log and meta buffers do not change
+    nbq, nlq, nmq = dlb.dl_state_bytes(cfg(base="q8"))
+    assert nbq == pad(BH * 128 * 128) + pad(BH * 128 * 4)
+    assert (nlq, nmq) == (nl, nm)
+    nbq, _, _ = dlb.dl_state_bytes(cfg(base="q8", B=3, H=1, d_k=64, d_v=64))
+    assert nbq == pad(3 * 64 * 64) + pad(3 * 64 * 4)
 
 
 @pytest.mark.parametrize("bad,code", [
@@ -86,8 +93,15 @@ def test_bad_enums_rejected():
     c.in_dtype = 3
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
     c = cfg().c()
-    c.flags = 8
+    c.flags = 16
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+    # the int8 base does not combine with the persistent step kernel
+    c = cfg(base="q8").c()
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_OK
+    c = cfg(base="q8", persistent=True).c()
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_UNSUPPORTED
+    with pytest.raises(ValueError):
+        cfg(base="q4").c()
     # the KLA step size applies to GDN and KDA, with a non-negative epsilon
     c = cfg(kla_eps=1e-6).c()
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_OK

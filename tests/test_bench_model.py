@@ -22,6 +22,18 @@ def test_step_bytes_uniform_phases_gdn_L16():
     assert rd2 == rd and wr2 == 16 * 32 * (516 + 772)
 
 
+def test_step_bytes_int8_base():
+    # the int8 base reads 16,384 codes + 512 B of row scales per head instead
+    # of 65,536 B, and the fused merge writes the same 16,896 B
+    cfg = dlb.Config("gdn", 16, 32, 128, 128, 16, "bf16", fused_merge=True, base="q8")
+    fills = np.arange(16)
+    rd, wr = bench.step_bytes(cfg, fills, fused=True)
+    per = (rd + wr) / (16 * 32)
+    assert per == pytest.approx(16896 + 776 + 4 + 772 * 7.5 + 516 + (15 * 772 + 16896) / 16)
+    mr, mw = bench.merge_bytes(cfg, np.array([16, 3]))
+    assert mr == 2 * 32 * 4 + 32 * (16896 + 16 * 772) and mw == 32 * (16896 + 4)
+
+
 def test_eager_and_merge_bytes():
     cfg = dlb.Config("gdn", 2, 32, 128, 128, 16, "bf16")
     rd, wr = bench.eager_bytes(cfg)
