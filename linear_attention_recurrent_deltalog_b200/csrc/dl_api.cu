@@ -208,8 +208,9 @@ dl_load_seqs_kernel(float* base, int* fill, const float* S, const dl::SeqList li
   if (threadIdx.x == 0) fill[head] = 0;
 }
 
-// Quantizes fp32 d_v x d_k tiles into an int8 base (codes and row scales),
-// one warp per row, with the rule the merge uses: inv = 127 / amax, code =
+// Quantizes fp32 d_v x d_k tiles into an int8 base (codes, in the swizzled
+// order of q8_off, and row scales), one warp per row, with the rule the merge
+// uses: inv = 127 / amax, code =
 // round-half-even(x * inv), scale = amax / 127, each rounded once in fp32;
 // rows with amax below 2^-120 become zero codes and scale 0.  CTA i covers
 // head i, or (use_list) head (list.seq[i / H], i % H) with source tile i;
@@ -240,7 +241,10 @@ dl_quantize_kernel(int8_t* codes, float* scales, int* fill, const float* S, cons
         w |= (uint32_t(__float2int_rn(__fmul_rn(x[e], inv))) & 0xffu) << (8 * e);
       sc = __fdiv_rn(m, 127.0f);
     }
-    int8_t* dst = codes + (head * dv + row) * size_t(dk) + lane * per;
+    // the lane's `per` codes stay contiguous inside one 16-byte chunk of the
+    // row's swizzled order
+    int8_t* dst = codes + head * size_t(dv) * dk +
+                  (dk == 128 ? dl::q8_off<128>(row, lane * per) : dl::q8_off<64>(row, lane * per));
     if (per == 4)
       *reinterpret_cast<uint32_t*>(dst) = w;
     else

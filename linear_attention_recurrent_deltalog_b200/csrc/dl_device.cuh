@@ -6,6 +6,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <type_traits>
@@ -325,6 +326,82 @@ __device__ __forceinline__ float row_max(float x) {
 #pragma unroll
   for (int o = 1; o < LPR; o <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
   return x;
+}
+
+// ------------------------------------------- int8 codes on the tensor cores
+//
+// The int8 base is multiplied on the tensor cores with warp-level
+// m16n8k16 MMAs in fp16 with fp32 accumulation: every int8 code is exact in
+// fp16, and an fp32 operand x enters as the pair hi = fp16(x), lo =
+// fp16(x - hi), whose sum carries 22 significant bits.  Products of fp16
+// values are exact in fp32, so hi*hi + hi*lo + lo*hi reproduces an fp32
+// product to about 2^-22 relative.
+
+// Byte offset of logical (row, c) inside a tile of int8 rows.  The 16-byte
+// chunks of each row are stored XOR-swizzled by the row (d_k = 128: row mod
+// 8; d_k = 64: (row / 2) mod 4), so eight consecutive rows reading the same
+// logical chunk hit eight different bank groups.  Global memory holds the
+// same order, so plain contiguous bulk copies keep the swizzle.
+template <int DK>
+__host__ __device__ __forceinline__ int q8_off(int row, int c) {
+  const int sw = (DK == 128) ? (row & 7) : ((row >> 1) & 3);
+  return row * DK + (((c >> 4) ^ sw) << 4) + (c & 15);
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) {
+  return *reinterpret_cast<const __half2*>(&u);
+}
+
+// (x0, x1) -> fp16 pairs hi = fp16(x), lo = fp16(x - hi).
+__device__ __forceinline__ void split_h2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 f = __half22float2(h);
+  hi = h2_bits(h);
+  lo = h2_bits(__floats2half2_rn(x0 - f.x, x1 - f.y));
+}
+
+// Four int8 codes (one word) -> two fp16 pairs (codes 0,1) and (codes 2,3),
+// exactly: with the sign bits flipped each byte n = code + 128 becomes the
+// low fraction byte of 1024 in fp16 (0x64nn = 1024 + n, exact up to 2047),
+// and subtracting 1152 = 1024 + 128 leaves the code.
+__device__ __forceinline__ void codes4_to_h2(uint32_t w, uint32_t& h01, uint32_t& h23) {
+  const uint32_t u = w ^ 0x80808080u;
+  const __half2 bias = bits_h2(0x64806480u);  // (1152, 1152)
+  h01 = h2_bits(__hsub2(bits_h2(__byte_perm(u, 0x64646464u, 0x4140)), bias));
+  h23 = h2_bits(__hsub2(bits_h2(__byte_perm(u, 0x64646464u, 0x4342)), bias));
+}
+
+// Two int8 codes (low half of a word) -> fp32, exactly.
+__device__ __forceinline__ float2 codes2_to_f(uint32_t w) {
+  uint32_t h01, h23;
+  codes4_to_h2(w, h01, h23);
+  return __half22float2(bits_h2(h01));
+}
+
+// D += A B for one m16n8k16 tile (fp16 inputs, fp32 accumulators).
+// Fragments (lane = 4 g + t): a0 (row g, k 2t..2t+1), a1 (row g+8, same k),
+// a2 (row g, k 2t+8..2t+9), a3 (row g+8, k 2t+8..2t+9); b0 (k 2t..2t+1,
+// col g), b1 (k 2t+8..2t+9, col g); d0,d1 (row g, cols 2t, 2t+1), d2,d3
+// (row g+8, cols 2t, 2t+1).
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four 8x8 matrices of 16-bit elements from shared memory: lanes 8m .. 8m+7
+// give the row addresses (16 bytes each) of matrix m; register m of lane
+// 4g + t then holds bytes 4t .. 4t+3 of row g of matrix m.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row_addr)));
 }
 
 }  // namespace dl

@@ -348,97 +348,232 @@ __device__ __forceinline__ void merge_rows_fused(const float* sS, const TU* sU, 
 
 // ---------------------------------------------------- int8 base rows
 //
-// The same per-warp operations on an int8 base (QRows layout: 16 codes per
-// lane per row).  The row scale multiplies the finished dot products.
+// The same per-warp operations on an int8 base, on the tensor cores (see
+// dl_device.cuh): a warp's 16 rows are one m16 tile.  Codes sit in shared
+// memory in the swizzled order of q8_off.
 
-template <int DK, bool WITH_A>
+// Number of 16-entry chunks the fold's k dimension is cut into.
+__host__ __device__ constexpr int q8_chunks(int L) { return (L + 15) / 16; }
+
+// Row stride (in halves) of the GEMV's fp16 vectors: 32 bytes of padding put
+// the four rows (read together by lanes 4g + t, g < 4) in different banks.
+template <int DK>
+constexpr int kVecHStride = DK + 16;
+
+// Base GEMV on the tensor cores: A = the warp's 16 rows of codes, B = the
+// four fp16 vectors of sVecH [4][kVecHStride] (columns: k-hat hi, k-hat lo, q-hat hi,
+// q-hat lo; the other four columns are zero), so D's columns 0+1 hold S k-hat
+// and 2+3 hold S q-hat.  Inside each 16-channel k-step, logical k (2t, 2t+1,
+// 2t+8, 2t+9) is channel (4t .. 4t+3): A and B agree, so the dot products
+// are unchanged.  Lane 4g + t with t < 2 finishes row jl = j0 + g (t = 0) or
+// j0 + g + 8 (t = 1), scaled by its row scale; `owner` is false elsewhere.
+template <int DK>
 __device__ __forceinline__ void rows_gemv_q8(const int8_t* sQ, const float* sScale, int j0, int lane,
-                                             const float* va, const float* vb, float& a, float& b,
-                                             int& jl) {
-  using G = QRows<DK>;
-  const int c0 = (lane % G::kLPR) * G::kCodes;
-  const int rsub = lane / G::kLPR;
-  float ka[16], kb[16];
-  if (WITH_A) load_f<16>(va + c0, ka);
-  load_f<16>(vb + c0, kb);
-  float pa[G::kNV], pb[G::kNV];
+                                             const __half* sVecH, float& a, float& b, int& jl,
+                                             bool& owner) {
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  const int m = lane >> 3;                       // ldmatrix: which matrix this lane addresses
+  const int arow = j0 + (lane & 7) + 8 * (m & 1);
 #pragma unroll
-  for (int pi = 0; pi < G::kNV; ++pi) {
-    float x[16];
-    codes16_to_f(sQ + size_t(j0 + pi * G::kRPI + rsub) * DK + c0, x);
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      if (WITH_A) {
-        a0 = fmaf(x[i], ka[i], a0);
-        a1 = fmaf(x[i + 1], ka[i + 1], a1);
-      }
-      b0 = fmaf(x[i], kb[i], b0);
-      b1 = fmaf(x[i + 1], kb[i + 1], b1);
+  for (int kk = 0; kk < DK / 16; kk += 2) {
+    uint32_t w[4];
+    ldmatrix_x4(w, sQ + q8_off<DK>(arow, 16 * (kk + (m >> 1))));
+    uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+    codes4_to_h2(w[0], a0, a2);  // row g,   channels 16 kk + 4t ..
+    codes4_to_h2(w[1], a1, a3);  // row g+8
+    codes4_to_h2(w[2], c0, c2);  // row g,   next k-step
+    codes4_to_h2(w[3], c1, c3);  // row g+8, next k-step
+    uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
+    if (g < 4) {
+      b0 = *reinterpret_cast<const uint2*>(sVecH + g * kVecHStride<DK> + 16 * kk + 4 * t);
+      b1 = *reinterpret_cast<const uint2*>(sVecH + g * kVecHStride<DK> + 16 * (kk + 1) + 4 * t);
     }
-    pa[pi] = a0 + a1;
-    pb[pi] = b0 + b1;
+    mma_16816(d, a0, a1, a2, a3, b0.x, b0.y);
+    mma_16816(d, c0, c1, c2, c3, b1.x, b1.y);
   }
-  a = WITH_A ? reduce_rows<G::kNV, G::kLPR>(pa, lane) : 0.f;
-  b = reduce_rows<G::kNV, G::kLPR>(pb, lane);
-  jl = j0 + reduced_index<G::kNV, G::kLPR>(lane) * G::kRPI + rsub;
-  const float s = sScale[jl];
-  a *= s;
-  b *= s;
+  // t = 0 holds S k-hat (rows g, g+8), t = 1 holds S q-hat; trade halves
+  const float send = (t == 0) ? d[2] + d[3] : d[0] + d[1];
+  const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+  owner = t < 2;
+  jl = j0 + g + ((t == 1) ? 8 : 0);
+  const float own = (t == 1) ? d[2] + d[3] : d[0] + d[1];
+  a = (t == 0) ? own : recv;
+  b = (t == 0) ? recv : own;
+  const float sc = sScale[jl];
+  a *= sc;
+  b *= sc;
 }
 
-// Folds nent log entries into the warp's 16 rows of an int8 base:
-//   x = deq(code) * dec + sum_e u_e[row] kt_e,  deq(code) = code * scale,
-// with kt_e the entries' decayed keys and dec the base's decay per key
-// channel, both staged in shared memory.  The rows are then requantized
-// into (gCodes, gScale), or written as fp32 into gOut when it is non-null.
+// Key channel of column j (0..7) of n-tile n in the fold's MMAs.  The fold
+// permutes the N dimension so that lane 4g + t, whose accumulators hold
+// columns 2t and 2t+1 of every n-tile, owns the DK/4 contiguous channels
+// [DK/4 t, DK/4 (t+1)) of its two rows: whole 16-byte groups of codes to
+// load and store.
+template <int DK>
+__host__ __device__ constexpr int fold_channel(int n, int j) {
+  return (DK / 4) * (j >> 1) + 2 * n + (j & 1);
+}
+
+// Slot of lane l's 16-byte B fragment for n-tile n in the staged array: the
+// lane index is XOR-ed with n mod 8, which leaves the fold's loads (one
+// n-tile, 32 lanes) conflict-free and spreads the staging stores over all
+// bank groups.
+__host__ __device__ constexpr int kt_slot(int kc, int ntiles, int n, int l) {
+  return (kc * ntiles + n) * 32 + (l ^ (n & 7));
+}
+
+// Stages the decayed keys kt_e[c] = k_e[c] e^{gLast[c] - g_e[c]} (factor 1
+// for entries e >= nlog, 0 for e >= nent) as fp16 hi/lo B fragments of the
+// fold: for 16-entry chunk kc and n-tile n, lane l's 16 bytes {b0 hi, b1 hi,
+// b0 lo, b1 lo} sit at kt_slot (column l/4 of the n-tile is key channel
+// fold_channel(n, l/4)).  A thread takes one key channel of one chunk: it
+// reads the chunk's 16 keys of that channel (consecutive threads read
+// consecutive channels) and writes the four lanes' fragments that carry
+// them.  GDN's decay is one factor per entry, from sFac (filled by the
+// caller); the vector decays take it per channel.  All threads of the CTA
+// take part; the caller synchronises afterwards.
+template <int VAR, int DK, typename TIn>
+__device__ __forceinline__ void stage_kt_frags(const TIn* sK, const float* sG, const float* gLast,
+                                               const float* sFac, int nlog, int nent, int nchunks,
+                                               uint32_t* sB, int tid, int nt) {
+  constexpr int NTILE = DK / 8;
+  constexpr int CPL = DK / 4;
+  for (int idx = tid; idx < nchunks * DK; idx += nt) {
+    const int c = idx % DK;
+    const int kc = idx / DK;
+    // inverse of fold_channel: c = CPL (j / 2) + 2 n + (j mod 2)
+    const int n = (c % CPL) >> 1;
+    const int j = 2 * (c / CPL) + (c & 1);
+    float x[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = 16 * kc + q;
+      float v = 0.f;
+      if (e < nent) {
+        v = to_f(sK[size_t(e) * DK + c]);
+        if (e < nlog)
+          v *= (VAR == kVarGDN) ? sFac[e] : expf(gLast[c] - sG[size_t(e) * DK + c]);
+      }
+      x[q] = v;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      uint4 w;
+      split_h2(x[2 * t], x[2 * t + 1], w.x, w.z);          // b0: entries 2t, 2t+1
+      split_h2(x[2 * t + 8], x[2 * t + 9], w.y, w.w);      // b1: entries 2t+8, 2t+9
+      reinterpret_cast<uint4*>(sB)[kt_slot(kc, NTILE, n, 4 * j + t)] = w;
+    }
+  }
+}
+
+// Folds nent log entries into the warp's 16 rows of an int8 base on the
+// tensor cores, in one pass:
+//   x = deq(code) * dec + U Kt,   deq(code) = code * scale,
+// U = the rows' u values (A, split hi/lo in registers), Kt = the staged B
+// fragments.  Lane 4g + t holds rows j0+g and j0+g+8 over the key channels
+// [DK/4 t, DK/4 (t+1)) (fold_channel).  With gOut the rows are written to it
+// as fp32 (unswizzled); otherwise each row's absolute maximum is reduced
+// over its four lanes and the row is requantized straight from the
+// accumulators into gCodes (swizzled order) and gScale.
 template <int DK, typename TU>
 __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sScale, const TU* sU,
-                                             const float* sKt, const float* sDec, int nent, int L,
-                                             int j0, int lane, int8_t* gCodes, float* gScale,
-                                             float* gOut) {
-  using G = QRows<DK>;
-  const int c0 = (lane % G::kLPR) * G::kCodes;
-  const int rsub = lane / G::kLPR;
-  float d[16];
-  load_f<16>(sDec + c0, d);
-  float acc[G::kNV][16];
+                                             const uint32_t* sB, const float* sDec, int nent,
+                                             int nchunks, int L, int j0, int lane, int8_t* gCodes,
+                                             float* gScale, float* gOut) {
+  constexpr int NTILE = DK / 8;      // n-tiles; lane holds 2 channels of each
+  constexpr int CPL = DK / 4;        // contiguous channels per lane
+  constexpr int WORDS = CPL / 4;     // 4-code words per lane per row
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int cbase = CPL * t;
+  const int rows[2] = {j0 + g, j0 + g + 8};
+  // acc[n][0..1]: row g, channels cbase + 2n, +1; acc[n][2..3]: row g+8
+  float acc[NTILE][4];
 #pragma unroll
-  for (int pi = 0; pi < G::kNV; ++pi) {
-    const int row = j0 + pi * G::kRPI + rsub;
-    codes16_to_f(sQ + size_t(row) * DK + c0, acc[pi]);
-    const float s = sScale[row];
+  for (int half = 0; half < 2; ++half) {
+    const int r = rows[half];
+    const float s = sScale[r];
+    uint32_t w[WORDS];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[pi][i] = (acc[pi][i] * s) * d[i];
+    for (int v = 0; v < WORDS / 4; ++v) {
+      const uint4 q = *reinterpret_cast<const uint4*>(sQ + q8_off<DK>(r, cbase + 16 * v));
+      w[4 * v] = q.x;
+      w[4 * v + 1] = q.y;
+      w[4 * v + 2] = q.z;
+      w[4 * v + 3] = q.w;
+    }
+#pragma unroll
+    for (int v = 0; v < WORDS; ++v) {
+      uint32_t h01, h23;
+      codes4_to_h2(w[v], h01, h23);
+      const float2 c01 = __half22float2(bits_h2(h01));
+      const float2 c23 = __half22float2(bits_h2(h23));
+      const float4 d4 = *reinterpret_cast<const float4*>(sDec + cbase + 4 * v);
+      acc[2 * v][2 * half] = (c01.x * s) * d4.x;
+      acc[2 * v][2 * half + 1] = (c01.y * s) * d4.y;
+      acc[2 * v + 1][2 * half] = (c23.x * s) * d4.z;
+      acc[2 * v + 1][2 * half + 1] = (c23.y * s) * d4.w;
+    }
   }
-  for (int e = 0; e < nent; ++e) {
-    float kt[16];
-    load_f<16>(sKt + size_t(e) * DK + c0, kt);
+  const uint4* sB4 = reinterpret_cast<const uint4*>(sB);
+  for (int kc = 0; kc < nchunks; ++kc) {
+    const int e0 = 16 * kc + 2 * t;
+    float u[8];  // (g, e0), (g, e0+1), (g+8, e0), (g+8, e0+1), then the same at e0+8
 #pragma unroll
-    for (int pi = 0; pi < G::kNV; ++pi) {
-      const float ui = to_f(sU[su_offset(j0 + pi * G::kRPI + rsub, e, L)]);
+    for (int q = 0; q < 8; ++q) {
+      const int e = e0 + (q & 1) + ((q & 4) ? 8 : 0);
+      u[q] = (e < nent) ? to_f(sU[su_offset(rows[(q >> 1) & 1], e, L)]) : 0.f;
+    }
+    uint32_t ah[4], al[4];
+    split_h2(u[0], u[1], ah[0], al[0]);  // a0: row g,   k 2t..
+    split_h2(u[2], u[3], ah[1], al[1]);  // a1: row g+8
+    split_h2(u[4], u[5], ah[2], al[2]);  // a2: row g,   k 2t+8..
+    split_h2(u[6], u[7], ah[3], al[3]);  // a3: row g+8
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[pi][i] = fmaf(ui, kt[i], acc[pi][i]);
+    for (int n = 0; n < NTILE; ++n) {
+      const uint4 bf = sB4[kt_slot(kc, NTILE, n, lane)];
+      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.x, bf.y);
+      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.z, bf.w);
+      mma_16816(acc[n], al[0], al[1], al[2], al[3], bf.x, bf.y);
     }
   }
 #pragma unroll
-  for (int pi = 0; pi < G::kNV; ++pi) {
-    const int row = j0 + pi * G::kRPI + rsub;
+  for (int half = 0; half < 2; ++half) {
+    const int r = rows[half];
     if (gOut != nullptr) {
-      float4* o = reinterpret_cast<float4*>(gOut + size_t(row) * DK + c0);
+      float4* o = reinterpret_cast<float4*>(gOut + size_t(r) * DK + cbase);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        o[q] = make_float4(acc[pi][4 * q], acc[pi][4 * q + 1], acc[pi][4 * q + 2], acc[pi][4 * q + 3]);
-    } else {
-      float m = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(acc[pi][i]));
-      m = row_max<G::kLPR>(m);
-      float sc;
-      const uint4 w = quantize16(acc[pi], m, &sc);
-      *reinterpret_cast<uint4*>(gCodes + size_t(row) * DK + c0) = w;
-      if (lane % G::kLPR == 0) gScale[row] = sc;
+      for (int v = 0; v < WORDS; ++v)
+        o[v] = make_float4(acc[2 * v][2 * half], acc[2 * v][2 * half + 1], acc[2 * v + 1][2 * half],
+                           acc[2 * v + 1][2 * half + 1]);
+      continue;
     }
+    float m = 0.f;
+#pragma unroll
+    for (int n = 0; n < NTILE; ++n)
+      m = fmaxf(m, fmaxf(fabsf(acc[n][2 * half]), fabsf(acc[n][2 * half + 1])));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    // rows below the tiny threshold store zero codes (inv = 0) and scale 0
+    const float inv = (m >= kTinyAmax) ? __fdiv_rn(127.0f, m) : 0.f;
+    uint32_t w[WORDS];
+#pragma unroll
+    for (int v = 0; v < WORDS; ++v) {
+      const float x[4] = {acc[2 * v][2 * half], acc[2 * v][2 * half + 1], acc[2 * v + 1][2 * half],
+                          acc[2 * v + 1][2 * half + 1]};
+      uint32_t word = 0u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        word |= (uint32_t(__float2int_rn(__fmul_rn(x[b], inv))) & 0xffu) << (8 * b);
+      w[v] = word;
+    }
+#pragma unroll
+    for (int v = 0; v < WORDS / 4; ++v)
+      *reinterpret_cast<uint4*>(gCodes + q8_off<DK>(r, cbase + 16 * v)) =
+          make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    if (t == 0) gScale[r] = (m >= kTinyAmax) ? __fdiv_rn(m, 127.0f) : 0.f;
   }
 }
 
@@ -465,8 +600,8 @@ struct StepLayout {
   using TU = typename LogU<VAR, TIn>::type;
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
   static constexpr bool Q8 = std::is_same<TB, int8_t>::value;
-  size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offScale,
-      offKt, offBar, total;
+  size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offBonus,
+      offScale, offVecH, offDecF, offKt, offBar, total;
   __host__ __device__ explicit StepLayout(int L) {
     offU = Tile<DK, ROWS, TB>::kTileBytes;
     offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
@@ -480,17 +615,30 @@ struct StepLayout {
     offW = offVec + align_up(size_t(4 * DK + 2 * GW) * 4, 128);
     offZ = offW + align_up(size_t(L) * 4, 16);
     offScal = offZ + align_up(size_t(L) * 4, 16);
-    // int8 base: the CTA's row scales, and for the fused merge the decayed
-    // keys of every entry [L][DK] plus the base decay [DK]
-    offScale = offScal + 64;
-    offKt = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
-    offBar = offKt + (Q8 ? align_up(size_t(L + 1) * DK * 4, 128) : 0);
+    // int8 base: the CTA's row scales, the GEMV's fp16 vectors [4][DK], the
+    // base decay [DK] and, for the fused merge, the staged key fragments
+    offBonus = offScal + 64;
+    offScale = offBonus + (VAR == kVarRWKV6 ? align_up(size_t(DK) * 4, 128) : 0);
+    offVecH = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
+    offDecF = offVecH + (Q8 ? align_up(size_t(4) * kVecHStride<DK> * 2, 128) : 0);
+    offKt = offDecF + (Q8 ? align_up(size_t(DK) * 4, 128) : 0);
+    offBar = offKt + (Q8 ? size_t(q8_chunks(L)) * DK * 64 : 0);
     total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
   }
 };
 
+// Resident CTAs per SM the int8 kernels are compiled for: the plain step
+// 1152 threads per SM (56 registers a thread), the step with the fused merge
+// and the merge 768 (80 registers; the fold's accumulators may spill a
+// little), so the rare fold does not set the occupancy of every step.  The
+// fp32 kernels keep the compiler's choice.
+template <typename TB, int THREADS, bool FOLDS>
+constexpr int kMinBlocks =
+    std::is_same<TB, int8_t>::value ? (FOLDS ? 768 : 1152) / THREADS : 1;
+
 template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB, bool FUSED>
-__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads)
+__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads,
+                                  kMinBlocks<TB, Tile<DK, ROWS, TB>::kThreads, FUSED>)
 dl_step_kernel(const StepParams p, const FillParam fp) {
   using Tl = Tile<DK, ROWS, TB>;
   using TU = typename LogU<VAR, TIn>::type;
@@ -524,10 +672,12 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   float* sW = reinterpret_cast<float*>(smem + lay.offW);      // per-entry weights on k
   float* sZ = reinterpret_cast<float*>(smem + lay.offZ);      // per-entry weights on q / r
   float* sScal = reinterpret_cast<float*>(smem + lay.offScal);  // [0] k.q / bonus [1] beta
-                                                                // [2] e^{g_t} [3] decay (GDN)
+                                                                // [2] e^{g_t}
+  float* sBonus = reinterpret_cast<float*>(smem + lay.offBonus);  // RWKV6: u [DK]
   float* sScale = reinterpret_cast<float*>(smem + lay.offScale);  // int8 base: row scales
-  float* sKt = reinterpret_cast<float*>(smem + lay.offKt);        // int8 fused merge: [L][DK]
-  float* sDecF = sKt + size_t(L) * DK;                            // and the base decay [DK]
+  __half* sVecH = reinterpret_cast<__half*>(smem + lay.offVecH);  // GEMV vectors, fp16 hi/lo
+  float* sDecF = reinterpret_cast<float*>(smem + lay.offDecF);    // fused merge: base decay
+  uint32_t* sB = reinterpret_cast<uint32_t*>(smem + lay.offKt);   // fused merge: key fragments
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
   uint64_t* barLog = &bars[Tl::kChunks];
 
@@ -552,8 +702,11 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   float* gG = p.logG + head * size_t(GS);
 
   // Warp 0 streams the tile; warp 1 fetches everything small (the step's
-  // vectors and the f log entries) and the two scalars no bulk copy can
-  // carry.  No other thread touches global memory before the data is in.
+  // vectors and the f log entries).  Each thread reads the two per-head
+  // scalars no bulk copy can carry (GDN's decay, beta) into registers, so
+  // no barrier waits on those loads.
+  const float dec_s = (GW == 1) ? __ldg(p.decay + head) : 0.f;
+  const float beta_s = (VAR == kVarRWKV6) ? 0.f : __ldg(p.beta + head);
   if (warp == 0 && lane == 0) {
 #pragma unroll
     for (int c = 0; c < Tl::kChunks; ++c) mbar_init(&bars[c], 1);
@@ -565,8 +718,6 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
                          Tl::kChunkBytes, &bars[c]);
     }
   } else if (warp == 1 && lane == 0) {
-    const float dec_s = (GW == 1) ? p.decay[head] : 0.f;      // loads in flight while
-    const float beta_s = (VAR == kVarRWKV6) ? 0.f : p.beta[head];  // the copies go out
     mbar_init(barLog, 1);
     fence_mbar_init();
     const uint32_t bq = DK * sizeof(TIn);
@@ -576,8 +727,11 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
     const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
     const uint32_t bs = Q8 ? ROWS * 4u : 0u;
-    mbar_arrive_expect_tx(barLog, 2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg + bs);
+    const uint32_t bb = (VAR == kVarRWKV6) ? DK * 4u : 0u;
+    mbar_arrive_expect_tx(barLog,
+                          2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg + bs + bb);
     if (Q8) tma_load_1d(sScale, p.scale + head * DV + r0, bs, barLog);
+    if (VAR == kVarRWKV6) tma_load_1d(sBonus, p.bonus + size_t(h) * DK, bb, barLog);
     tma_load_1d(sQr, static_cast<const TIn*>(p.q) + head * DK, bq, barLog);
     tma_load_1d(sKr, static_cast<const TIn*>(p.k) + head * DK, bq, barLog);
     tma_load_1d(sVr, static_cast<const TIn*>(p.v) + head * DV + r0, bv, barLog);
@@ -589,8 +743,6 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
         tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, r0 + rb * kURows, 0, L, DV), bu,
                     barLog);
     }
-    sScal[1] = beta_s;
-    sScal[3] = dec_s;
     if (part == 0) p.fill_out[head] = merge_now ? 0 : f + 1;
   }
   __syncthreads();
@@ -621,10 +773,22 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       sK[size_t(f) * DK + c] = kraw;
     else if (appender)
       gK[size_t(f) * DK + c] = kraw;
+    if constexpr (Q8) {  // the GEMV's B columns: k-hat and q-hat as fp16 hi/lo pairs
+      const float va = (VAR == kVarGDN) ? kc : (VAR == kVarKDA ? sKh[c] : 0.f);
+      const float vb = (VAR == kVarGDN) ? qc : sQh[c];
+      uint32_t hi, lo;
+      split_h2(va, vb, hi, lo);
+      const __half2 h = bits_h2(hi), l = bits_h2(lo);
+      constexpr int VS = kVecHStride<DK>;
+      sVecH[c] = __low2half(h);
+      sVecH[VS + c] = __low2half(l);
+      sVecH[2 * VS + c] = __high2half(h);
+      sVecH[3 * VS + c] = __high2half(l);
+    }
   }
   if (GW == 1 && tid == NT - 1) {
     const float gp = (f > 0) ? sG[f - 1] : 0.f;
-    const float gt = gp + logf(sScal[3]);
+    const float gt = gp + logf(dec_s);
     sGp[0] = gp;
     sGt[0] = gt;
     sScal[2] = expf(gt);
@@ -632,7 +796,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   }
   if (f > 0)
     entry_weights<VAR, DK, TIn, TIn>(f, warp, NW, lane, sKr, sQr, sK, sG,
-                                     (GW == 1) ? &sScal[3] : sDecV, sW, sZ);
+                                     (GW == 1) ? &dec_s : sDecV, sW, sZ);
   if (warp == NW - 1) {
     // GDN/KDA: k_t . q_t (the current entry's own weight on q) and, for the
     // KLA step size, |k_t|^2; RWKV6: the bonus sum_c r_c u_c k_c.
@@ -642,14 +806,14 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       const int c = lane * CPL + cc;
       const float kc = to_f(sKr[c]);
       const float qc = to_f(sQr[c]);
-      x = (VAR == kVarRWKV6) ? fmaf(qc * p.bonus[size_t(h) * DK + c], kc, x) : fmaf(kc, qc, x);
+      x = (VAR == kVarRWKV6) ? fmaf(qc * sBonus[c], kc, x) : fmaf(kc, qc, x);
       kk = fmaf(kc, kc, kk);
     }
     x = warp_sum(x);
     if (VAR != kVarRWKV6 && p.kla) kk = warp_sum(kk);
     if (lane == 0) {
       sScal[0] = x;
-      if (VAR != kVarRWKV6 && p.kla) sScal[1] = sScal[1] / (kk + p.kla_eps);  // eta -> beta
+      sScal[1] = (VAR != kVarRWKV6 && p.kla) ? beta_s / (kk + p.kla_eps) : beta_s;  // eta -> beta
     }
   }
   if (!__syncthreads_and(ok)) {
@@ -671,15 +835,17 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   }
   float a, b;
   int jl;  // local row this lane finishes
-  if constexpr (Q8)
-    rows_gemv_q8<DK, VAR != kVarRWKV6>(sS, sScale, j0, lane, (VAR == kVarGDN) ? sk : sKh,
-                                       (VAR == kVarGDN) ? sq : sQh, a, b, jl);
-  else
+  bool owner;  // the one lane that writes row jl
+  if constexpr (Q8) {
+    rows_gemv_q8<DK>(sS, sScale, j0, lane, sVecH, a, b, jl, owner);
+  } else {
     rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
                                     (VAR == kVarGDN) ? sq : sQh, a, b, jl);
+    owner = (lane & 1) == 0;
+  }
   float u, o;
   row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, to_f(sVr[jl]), a, b, u, o);
-  if ((lane & 1) == 0) {
+  if (owner) {
     p.o[head * DV + r0 + jl] = o;
     if (merge_now)
       sU[su_offset(jl, f, L)] = Elem<TU>::from_f(u);
@@ -691,16 +857,14 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     // every warp's u_t rows are in slot f; stage the decayed keys of the
     // L entries and the base decay once for the CTA, then fold and requantize
     __syncthreads();
-    for (int x = tid; x < (f + 1) * DK; x += NT) {
-      const int i = x / DK;
-      const int c = x % DK;
-      float kt = to_f(sK[x]);
-      if (i < f) kt *= expf(sGt[GW > 1 ? c : 0] - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
-      sKt[x] = kt;
+    if (GW == 1) {  // GDN: one decay factor per entry (sW's weights are no longer needed)
+      for (int e = tid; e < f; e += NT) sW[e] = expf(sGt[0] - sG[e]);
+      __syncthreads();
     }
+    stage_kt_frags<VAR, DK, TIn>(sK, sG, sGt, sW, f, f + 1, q8_chunks(f + 1), sB, tid, NT);
     for (int c = tid; c < DK; c += NT) sDecF[c] = (GW == 1) ? sScal[2] : expf(sGt[c]);
     __syncthreads();
-    fold_rows_q8<DK, TU>(sS, sScale, sU, sKt, sDecF, f + 1, L, j0, lane,
+    fold_rows_q8<DK, TU>(sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L, j0, lane,
                          static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
                          p.scale + head * size_t(DV) + r0, nullptr);
   } else {
@@ -722,9 +886,10 @@ struct MergeLayout {
     offU = Tile<DK, ROWS, TB>::kTileBytes;
     offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
     offKt = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
-    offG = offKt + align_up(size_t(L) * DK * 4, 128);
+    // fp32 decayed keys [L][DK], or (int8 base) their staged fp16 fragments
+    offG = offKt + align_up(Q8 ? size_t(q8_chunks(L)) * DK * 64 : size_t(L) * DK * 4, 128);
     offDec = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
-    offScale = offDec + align_up(size_t(DK) * 4, 128);
+    offScale = offDec + align_up(size_t(DK + (Q8 ? 64 : 0)) * 4, 128);  // + GDN entry factors
     offBar = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
     total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
   }
@@ -735,7 +900,8 @@ struct MergeLayout {
 // list and only part 0 empties the log, so split CTAs never race on it;
 // without a list the kernel runs unsplit and reads the device fill.
 template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB>
-__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads)
+__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads,
+                                  kMinBlocks<TB, Tile<DK, ROWS, TB>::kThreads, true>)
 dl_merge_kernel(const MergeParams p, const SeqList list) {
   using Tl = Tile<DK, ROWS, TB>;
   using TU = typename LogU<VAR, TIn>::type;
@@ -822,11 +988,23 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
   // one (entry, channel) pair per thread
   for (int c = tid; c < DK; c += NT)
     sDec[c] = expf((f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f);
-  for (int x = tid; x < f * DK; x += NT) {
-    const int i = x / DK;
-    const int c = x % DK;
-    const float gl = sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)];
-    sKt[x] = to_f(sK[x]) * expf(gl - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
+  if constexpr (Q8) {
+    if (f > 0) {
+      float* sFac = sDec + DK;  // GDN: e^{g_last - g_i} per entry
+      if (GW == 1) {
+        for (int e = tid; e < f; e += NT) sFac[e] = expf(sG[f - 1] - sG[e]);
+        __syncthreads();
+      }
+      stage_kt_frags<VAR, DK, TIn>(sK, sG, sG + size_t(f - 1) * GW, sFac, f, f, q8_chunks(f),
+                                   reinterpret_cast<uint32_t*>(sKt), tid, NT);
+    }
+  } else {
+    for (int x = tid; x < f * DK; x += NT) {
+      const int i = x / DK;
+      const int c = x % DK;
+      const float gl = sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)];
+      sKt[x] = to_f(sK[x]) * expf(gl - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
+    }
   }
   if (tid == 0 && part == 0 && p.mode != 2) p.fill[head] = 0;
   if (!__syncthreads_and(ok)) {
@@ -843,7 +1021,8 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
   }
   if constexpr (Q8) {
     const bool to_fp32 = (p.mode == 2);
-    fold_rows_q8<DK, TU>(sS, sScale, sU, sKt, sDec, f, L, j0, lane,
+    fold_rows_q8<DK, TU>(sS, sScale, sU, reinterpret_cast<const uint32_t*>(sKt), sDec, f,
+                         q8_chunks(f), L, j0, lane,
                          static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
                          p.scale + head * size_t(DV) + r0,
                          to_fp32 ? p.out + (head * size_t(DV) + r0) * DK : nullptr);

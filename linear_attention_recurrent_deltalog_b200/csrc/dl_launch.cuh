@@ -267,14 +267,18 @@ struct StepSmem {
   template <int DK, int DV, typename T>
   cudaError_t run() {
     out = 0;
-    if (split == 1) out = StepLayout<VAR, DK, DV, DV, T, TB>(L).total;
+    if (split == 1) out = need<DK, DV, DV, T>();
     if constexpr (DV / 2 >= 32) {
-      if (split == 2) out = StepLayout<VAR, DK, DV, DV / 2, T, TB>(L).total;
+      if (split == 2) out = need<DK, DV, DV / 2, T>();
     }
     if constexpr (DV / 4 >= 32) {
-      if (split == 4) out = StepLayout<VAR, DK, DV, DV / 4, T, TB>(L).total;
+      if (split == 4) out = need<DK, DV, DV / 4, T>();
     }
     return out ? cudaSuccess : cudaErrorInvalidValue;
+  }
+  template <int DK, int DV, int ROWS, typename T>
+  size_t need() const {
+    return StepLayout<VAR, DK, DV, ROWS, T, TB>(L).total;
   }
 };
 template <int VAR, typename TB>

@@ -324,21 +324,50 @@ class DeltaLogState:
     def fill(self):
         return dl_state_fill(self.handle, self.cfg)
 
-    # Views of an int8 base in the layout deltalog.h documents: codes
-    # [B*H, d_v, d_k], then the fp32 row scales [B*H, d_v] at the next
-    # 256-byte boundary.
+    # An int8 base in the layout deltalog.h documents: codes [B*H, d_v, d_k]
+    # with each row's 16-byte chunks stored XOR-swizzled (chunk ^ (row mod 8)
+    # for d_k = 128, chunk ^ ((row / 2) mod 4) for d_k = 64), then the fp32
+    # row scales [B*H, d_v] at the next 256-byte boundary.
     def _scale_offset(self) -> int:
         n = self.cfg.heads * self.cfg.d_v * self.cfg.d_k
         return (n + 255) // 256 * 256
 
-    def base_codes(self) -> torch.Tensor:
+    def _q8_perm(self) -> torch.Tensor:
+        """Physical position of each logical (row, c) code within a head."""
+        if getattr(self, "_perm", None) is None:
+            dv, dk = self.cfg.d_v, self.cfg.d_k
+            r = torch.arange(dv).view(dv, 1)
+            c = torch.arange(dk).view(1, dk)
+            sw = (r & 7) if dk == 128 else ((r >> 1) & 3)
+            self._perm = (r * dk + (((c >> 4) ^ sw) << 4) + (c & 15)).reshape(-1).to(self.base.device)
+        return self._perm
+
+    def base_codes_raw(self) -> torch.Tensor:
+        """The stored int8 codes [B*H, d_v*d_k] in their swizzled order (a view)."""
         if self.cfg.base != "q8":
-            raise ValueError("base_codes: the base is fp32")
+            raise ValueError("base_codes_raw: the base is fp32")
         c = self.cfg
-        raw = self.base.view(torch.uint8)
-        return raw[:c.heads * c.d_v * c.d_k].view(torch.int8).view(c.heads, c.d_v, c.d_k)
+        return self.base.view(torch.uint8)[:c.heads * c.d_v * c.d_k].view(torch.int8).view(
+            c.heads, c.d_v * c.d_k)
+
+    def base_codes(self, heads=None) -> torch.Tensor:
+        """The codes of `heads` (all when None) in logical order [n, d_v, d_k] (a copy)."""
+        raw = self.base_codes_raw()
+        if heads is not None:
+            raw = raw.index_select(0, torch.as_tensor(heads, device=raw.device))
+        return raw[:, self._q8_perm()].view(-1, self.cfg.d_v, self.cfg.d_k)
+
+    def set_base_codes(self, heads, codes: torch.Tensor) -> None:
+        """Writes logical-order codes [n, d_v, d_k] of `heads` into the base."""
+        raw = self.base_codes_raw()
+        heads = torch.as_tensor(heads, device=raw.device)
+        tmp = torch.empty((heads.numel(), raw.shape[1]), dtype=torch.int8, device=raw.device)
+        tmp[:, self._q8_perm()] = codes.reshape(heads.numel(), -1).to(device=raw.device,
+                                                                      dtype=torch.int8)
+        raw.index_copy_(0, heads, tmp)
 
     def base_scales(self) -> torch.Tensor:
+        """The fp32 row scales [B*H, d_v] (a view)."""
         if self.cfg.base != "q8":
             raise ValueError("base_scales: the base is fp32")
         c = self.cfg

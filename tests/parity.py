@@ -223,7 +223,7 @@ def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Seque
     st.reset(torch.from_numpy(S0).to(device).reshape(-1), fill0.tolist())
     S0h = S0.reshape(BH, dv, dk)[heads]
     c0, s0 = oracle.quantize_rows(S0h)
-    g_codes = st.base_codes().index_select(0, heads_t).cpu().numpy()
+    g_codes = st.base_codes(heads_t).cpu().numpy()
     g_scales = st.base_scales().index_select(0, heads_t).cpu().numpy()
     reset_exact = bool(np.array_equal(g_codes, c0) and np.array_equal(g_scales, s0))
     S = _lib_rows(oracle.dequantize_rows(c0, s0), rec).copy()      # recurrence orientation
@@ -257,7 +257,7 @@ def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Seque
             codes, scales = oracle.quantize_rows(pre)
             inv = oracle.row_inverse(pre).astype(np.float64)
             gidx = torch.from_numpy(heads[idx]).to(device)
-            gc = st.base_codes().index_select(0, gidx).cpu().numpy().astype(np.float64)
+            gc = st.base_codes(gidx).cpu().numpy().astype(np.float64)
             gs = st.base_scales().index_select(0, gidx).cpu().numpy().astype(np.float64)
             eps = STATE_TOL * np.max(np.abs(pre), axis=(1, 2), keepdims=True)
             delta = 2.0 * eps * inv[..., None] + 1e-6
@@ -269,7 +269,7 @@ def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Seque
             total += codes.size
             windows += idx.size
             if resync:
-                st.base_codes().index_copy_(0, gidx, torch.from_numpy(codes).to(device))
+                st.set_base_codes(gidx, torch.from_numpy(codes))
                 st.base_scales().index_copy_(0, gidx, torch.from_numpy(scales).to(device))
             S[idx] = _lib_rows(oracle.dequantize_rows(codes, scales), rec)
             fill[idx] = 0

@@ -198,3 +198,22 @@ def test_load_seqs_checks_indices_on_the_host():
         assert ld(h, 0, None, None, None) == dlb.DL_OK                # nothing to do
     finally:
         dlb.dl_state_destroy(h)
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_int8_code_swizzle_is_a_chunk_permutation(dk, dv):
+    # logical (row, c) -> physical position: each row's 16-byte chunks are
+    # permuted (XOR with row mod 8, or (row / 2) mod 4 for d_k = 64), bytes
+    # inside a chunk stay in place, and eight consecutive rows put one logical
+    # chunk into eight different 16-byte bank groups
+    import torch
+    st = object.__new__(dlb.DeltaLogState)
+    st.cfg = cfg(d_k=dk, d_v=dv, base="q8")
+    st.base = torch.empty(8)
+    perm = st._q8_perm().view(dv, dk)
+    assert sorted(perm.reshape(-1).tolist()) == list(range(dv * dk))
+    assert torch.all(perm // dk == torch.arange(dv).view(dv, 1))
+    assert torch.all(perm % 16 == torch.arange(dk).view(1, dk) % 16)
+    groups = (perm[:8, ::16] // 16) % 8          # rows 0..7, each logical chunk
+    for j in range(dk // 16):
+        assert len(set(groups[:, j].tolist())) == 8

@@ -121,7 +121,7 @@ def test_q8_reset_edge_rows():
     M = st.materialize().view(B * H, d, d).cpu().numpy().astype(np.float64)
     assert np.array_equal(M, oracle.dequantize_rows(codes, scales))
     st.reset(None)
-    assert torch.count_nonzero(st.base_codes()) == 0 and torch.count_nonzero(st.base_scales()) == 0
+    assert torch.count_nonzero(st.base_codes_raw()) == 0 and torch.count_nonzero(st.base_scales()) == 0
     st.close()
 
 
