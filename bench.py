@@ -395,16 +395,18 @@ def run_ours(args, world, rank, local):
     step_bytes_avg = (rd + wr) / args.steps
     achieved = step_bytes_avg / step_avg / 1e9
     traffic = None
-    tfile = os.path.join(ROOT, "profiles", "step_kernel_traffic.json")
-    if os.path.exists(tfile):
+    for tname in ("step_kernel_traffic.json", "step_kernel_traffic_q8.json"):
+        tfile = os.path.join(ROOT, "profiles", tname)
+        if not os.path.exists(tfile):
+            continue
         try:
             t = json.load(open(tfile))
-            if (t.get("kernel_hash") == kernel_hash() and t.get("L") == w.L and t.get("merge") == args.merge
-                    and t.get("workload") == w.name and t.get("B") == w.B
-                    and t.get("base", "f32") == args.base):
-                traffic = t.get("bytes_per_launch")
         except Exception:
-            traffic = None
+            continue
+        if (t.get("kernel_hash") == kernel_hash() and t.get("L") == w.L and t.get("merge") == args.merge
+                and t.get("workload") == w.name and t.get("B") == w.B
+                and t.get("base", "f32") == args.base):
+            traffic = t.get("bytes_per_launch")
 
     if args.only_step:
         st.close()
