@@ -13,6 +13,8 @@ library is measured on:
   gdn_tiny      GDN   B=1   H=2  d=64  T=32   L=8   fp32 inputs
   gdn_qwen      GDN   B=64  H=32 d=128 T=256  L=16  bf16 q/k/v
   kda           KDA   B=128 H=32 d=128 T=256  L=16  bf16 q/k/v, per-channel decay
+  gdn2          GDN-2 B=128 H=32 d=128 T=256  L=16  as kda, plus per-channel erase
+                                                    and write gates
   rwkv6         RWKV6 B=256 H=64 d=64  T=512  L=32  bf16 r/k/v, u-bonus per head
   gdn_serving   GDN   B=512 H=32 d=128 T=1024 L in {4,8,16,32,64}, ragged fills
 
@@ -20,7 +22,9 @@ Draw recipe (fixed, so any single step can be regenerated on its own):
   * step t uses numpy ``Generator(PCG64(SeedSequence([seed, 1, t])))`` and
     draws, in order, q (or r), k, v, decay, beta, each shaped [B, H, .] in
     C order (beta is not drawn for RWKV6; with the KLA step size the beta
-    draw is the gate eta and q, k are scaled by 1/sqrt(d_k), not normalised);
+    draw is the gate eta and q, k are scaled by 1/sqrt(d_k), not normalised;
+    GDN-2 draws the erase gate b = sigmoid(N(0,1)) [B, H, d_k] in beta's
+    place and then the write gate w = sigmoid(N(0,1)) [B, H, d_v]);
   * the initial state S0 uses ``SeedSequence([seed, 0, 0])``: fp32 N(0, 1)
     scaled by 0.01 (the "N(0, 0.01)" of the configs read as a standard
     deviation), shaped [B, H, d_v, d_k];
@@ -43,7 +47,8 @@ import numpy as np
 GDN = "gdn"
 KDA = "kda"
 RWKV6 = "rwkv6"
-VARIANTS = (GDN, KDA, RWKV6)
+GDN2 = "gdn2"
+VARIANTS = (GDN, KDA, RWKV6, GDN2)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -72,7 +77,7 @@ class Workload:
 
     @property
     def decay_is_vector(self) -> bool:
-        return self.variant in (KDA, RWKV6)
+        return self.variant in (KDA, RWKV6, GDN2)
 
     @property
     def heads(self) -> int:
@@ -85,6 +90,7 @@ WORKLOADS = {
     "gdn_qwen": Workload("gdn_qwen", GDN, 64, 32, 128, 128, 256, 16, "bf16", 2),
     "kda": Workload("kda", KDA, 128, 32, 128, 128, 256, 16, "bf16", 3),
     "rwkv6": Workload("rwkv6", RWKV6, 256, 64, 64, 64, 512, 32, "bf16", 4),
+    "gdn2": Workload("gdn2", GDN2, 128, 32, 128, 128, 256, 16, "bf16", 6),
     "gdn_serving": Workload("gdn_serving", GDN, 512, 32, 128, 128, 1024, 16,
                             "bf16", 5, ragged=True),
 }
@@ -127,8 +133,9 @@ class StepInputs:
 
     ``q`` holds r for RWKV6.  For bf16 workloads every value of q/k/v is
     exactly bf16-representable; ``device_bits`` gives the bit patterns.
-    ``decay`` is [B,H] (GDN alpha) or [B,H,d_k] (KDA alpha, RWKV6 w);
-    ``beta`` is [B,H] or None (RWKV6).
+    ``decay`` is [B,H] (GDN alpha) or [B,H,d_k] (KDA and GDN-2 alpha, RWKV6
+    w); ``beta`` is [B,H], the GDN-2 erase gate [B,H,d_k], or None (RWKV6);
+    ``wgate`` is the GDN-2 write gate [B,H,d_v], None otherwise.
     """
 
     t: int
@@ -138,6 +145,7 @@ class StepInputs:
     decay: np.ndarray
     beta: Optional[np.ndarray]
     in_dtype: str
+    wgate: Optional[np.ndarray] = None
 
     def device_array(self, name: str) -> np.ndarray:
         """q/k/v as the kernel reads them: uint16 bf16 bits or fp32."""
@@ -188,8 +196,14 @@ def step_inputs(w: Workload, t: int, B: Optional[int] = None) -> StepInputs:
         else:
             x = g.standard_normal((B, H))
             alpha = np.exp(-np.logaddexp(0.0, x) * 0.1)  # exp(-softplus(x) * 0.1)
-    else:  # KDA: per-key-channel decay
+    else:  # KDA, GDN-2: per-key-channel decay
         alpha = g.uniform(0.80, 1.00, size=(B, H, dk))
+    if w.variant == GDN2:
+        bgate = 1.0 / (1.0 + np.exp(-g.standard_normal((B, H, dk))))
+        wgate = 1.0 / (1.0 + np.exp(-g.standard_normal((B, H, dv))))
+        return StepInputs(t, _to_in_dtype(q, w.in_dtype), _to_in_dtype(k, w.in_dtype),
+                          _to_in_dtype(v, w.in_dtype), round_f32(alpha), round_f32(bgate),
+                          w.in_dtype, round_f32(wgate))
     beta = 1.0 / (1.0 + np.exp(-g.standard_normal((B, H))))
     return StepInputs(t, _to_in_dtype(q, w.in_dtype), _to_in_dtype(k, w.in_dtype),
                       _to_in_dtype(v, w.in_dtype), round_f32(alpha), round_f32(beta),

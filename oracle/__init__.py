@@ -1,7 +1,7 @@
 """fp64 CPU oracle for DeltaLog decoding -- TEST INFRASTRUCTURE ONLY.
 
-This package is the plain, slow, eager definition of the three recurrences
-DeltaLog decodes (GDN, KDA, RWKV6), written in float64 numpy, and of the same
+This package is the plain, slow, eager definition of the recurrences DeltaLog
+decodes (GDN, KDA, RWKV6, and GDN-2 with separate erase and write gates), written in float64 numpy, and of the same
 recurrences with the state quantized to int8 once per window
 (``window_quant``).  It is what the
 GPU path must reproduce: DeltaLog's claim is that the model observes the same
@@ -20,7 +20,7 @@ invariants and an exact-arithmetic brute force of the log form (see
 """
 
 from .recurrence import (  # noqa: F401
-    gdn_step, kda_step, rwkv6_step, kla_beta, run_eager, EagerResult,
+    gdn_step, kda_step, gdn2_step, rwkv6_step, kla_beta, run_eager, EagerResult,
 )
 from .window_quant import (  # noqa: F401
     quantize_rows, dequantize_rows, row_inverse, run_windowed, WindowedResult, WindowEnd,

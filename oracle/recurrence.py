@@ -28,6 +28,16 @@ recurrence exactly as written, forming the matrices the formula names
   library stores the transpose), w_t a d_k vector, u a fixed d_k vector per
   head.  The readout uses the state before the update.
 
+* GDN-2 (Gated DeltaNet-2 abstract: a channel-wise erase gate b_t on the
+  key side and a channel-wise write gate w_t on the value side replace the
+  delta rule's single beta; it reduces to KDA when both gates are the same
+  scalar):
+      S_t = S_{t-1} Diag(alpha_t) (I - (b_t o k_t) k_t^T) + (w_t o v_t) k_t^T,
+      o_t = S_t q_t,
+  alpha_t and b_t vectors over the d_k key channels, w_t over the d_v value
+  rows.  The erase reads the decayed state through the gated key b_t o k_t
+  and removes it along k_t, so every step stays a rank-1 update in k_t.
+
 * KLA (Kaczmarz step size; "Kaczmarz Linear Attention" abstract): the GDN
   (or KDA) recurrence with beta_t formed from a gate eta_t and the key norm,
       beta_t = eta_t / (|k_t|_2^2 + eps),
@@ -86,6 +96,24 @@ def kda_step(S, q, k, v, alpha, beta):
     return S_new, o
 
 
+def gdn2_step(S, q, k, v, alpha, b, w):
+    """One GDN-2 step for N heads.
+
+    S [N, d_v, d_k]; q, k [N, d_k]; v [N, d_v]; alpha, b [N, d_k] (decay and
+    erase gate per key channel); w [N, d_v] (write gate per value row).
+    """
+    S, q, k, v = _f64(S), _f64(q), _f64(k), _f64(v)
+    alpha, b, w = _f64(alpha), _f64(b), _f64(w)
+    dk = k.shape[-1]
+    eye = np.eye(dk)[None, :, :]
+    diag_alpha = alpha[:, :, None] * eye                      # Diag(alpha)
+    erase = eye - (b * k)[:, :, None] * k[:, None, :]         # I - (b o k) k^T
+    write = (w * v)[:, :, None] * k[:, None, :]               # (w o v) k^T
+    S_new = (S @ diag_alpha) @ erase + write
+    o = (S_new @ q[:, :, None])[:, :, 0]
+    return S_new, o
+
+
 def rwkv6_step(S, r, k, v, w, u):
     """One RWKV6 step for N heads.
 
@@ -133,7 +161,8 @@ def run_eager(variant: str, S0, steps: Iterable, heads: Optional[Sequence[int]] 
 
     ``S0``: float array [N, ...] in the recurrence's orientation for the
     selected heads.  ``steps``: objects with fields q (r for RWKV6), k, v,
-    decay and beta, each shaped [B, H, ...]; ``heads`` picks N flat
+    decay and beta (GDN-2: the erase gate b), and for GDN-2 wgate, each shaped
+    [B, H, ...]; ``heads`` picks N flat
     (b*H + h) heads from them (all heads when None).  ``bonus``: RWKV6 u per
     selected head [N, d_k].  ``snapshot_at``: 1-based step counts after which
     a copy of the state is kept.  ``kla_eps`` (GDN/KDA): when given, each
@@ -156,6 +185,8 @@ def run_eager(variant: str, S0, steps: Iterable, heads: Optional[Sequence[int]] 
             S, o = gdn_step(S, q, k, v, dec, beta)
         elif variant == "kda":
             S, o = kda_step(S, q, k, v, dec, beta)
+        elif variant == "gdn2":
+            S, o = gdn2_step(S, q, k, v, dec, beta, _select(st.wgate, heads))
         elif variant == "rwkv6":
             S, o = rwkv6_step(S, q, k, v, dec, bonus)
         else:

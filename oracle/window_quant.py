@@ -11,7 +11,7 @@ buffer, a window is the stretch between two merges of a sequence's log, so
 the definition is:
 
     S <- deq(Q(S0)) at the start;
-    every step: S, o_t <- the eager step (GDN / KDA / RWKV6) on S;
+    every step: S, o_t <- the eager step (GDN / KDA / GDN-2 / RWKV6) on S;
     after a step that ends the sequence's window: S <- deq(Q(S)).
 
 A window ends when the step's append fills the log (L entries, counting the
@@ -47,7 +47,7 @@ from typing import Dict, Iterable, List, Optional, Sequence
 
 import numpy as np
 
-from .recurrence import gdn_step, kda_step, kla_beta, rwkv6_step
+from .recurrence import gdn2_step, gdn_step, kda_step, kla_beta, rwkv6_step
 
 TINY_AMAX = np.float32(2.0 ** -120)
 
@@ -164,6 +164,8 @@ def run_windowed(variant: str, S0, steps: Iterable, L: int, fill0, H: int,
             S, o = gdn_step(S, q, k, v, dec, beta)
         elif variant == "kda":
             S, o = kda_step(S, q, k, v, dec, beta)
+        elif variant == "gdn2":
+            S, o = gdn2_step(S, q, k, v, dec, beta, _select(st.wgate, heads))
         elif variant == "rwkv6":
             S, o = rwkv6_step(S, q, k, v, dec, bonus)
         else:

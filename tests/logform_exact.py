@@ -33,7 +33,8 @@ def _dot(a: Sequence[Fraction], b: Sequence[Fraction]) -> Fraction:
 
 
 class ExactDeltaLog:
-    """One head of DeltaLog, exact.  ``variant`` in {"gdn", "kda", "rwkv6"}."""
+    """One head of DeltaLog, exact.  ``variant`` in {"gdn", "kda", "rwkv6",
+    "gdn2"}."""
 
     def __init__(self, variant: str, S0: Mat, L: int, fill0: int = 0,
                  bonus: Optional[Vec] = None):
@@ -76,7 +77,10 @@ class ExactDeltaLog:
         return [_dot(row, xs) for row in self.base]
 
     # ---- the decode step: reads base + log, appends one factor
-    def step(self, q, k, v, decay, beta=None) -> Vec:
+    def step(self, q, k, v, decay, beta=None, wgate=None) -> Vec:
+        """GDN-2: ``beta`` is the erase gate b (per key channel) and
+        ``wgate`` the write gate w (per value row): the read key is b o k and
+        the written value w o v, u_t = w o v - S'(b o k)."""
         if len(self.log) >= self.L:
             raise RuntimeError("log full: merge first")
         q = [Fraction(x) for x in q]
@@ -94,15 +98,22 @@ class ExactDeltaLog:
             o = [oj + bonus * vj for oj, vj in zip(o, v)]
             self.log.append((v, k, gt))
             return o
-        beta = Fraction(beta)
-        a = self._base_times(k, gt)
+        if self.variant == "gdn2":
+            kread = [Fraction(bc) * kc for bc, kc in zip(beta, k)]
+        else:
+            beta = Fraction(beta)
+            kread = k
+        a = self._base_times(kread, gt)
         b = self._base_times(q, gt)
         for (u_i, k_i, g_i) in self.log:
-            ck = self._ratio_dot(k_i, k, gt, g_i)
+            ck = self._ratio_dot(k_i, kread, gt, g_i)
             cq = self._ratio_dot(k_i, q, gt, g_i)
             a = [aj + ck * uj for aj, uj in zip(a, u_i)]
             b = [bj + cq * uj for bj, uj in zip(b, u_i)]
-        u_t = [beta * (vj - aj) for vj, aj in zip(v, a)]
+        if self.variant == "gdn2":
+            u_t = [Fraction(wj) * vj - aj for wj, vj, aj in zip(wgate, v, a)]
+        else:
+            u_t = [beta * (vj - aj) for vj, aj in zip(v, a)]
         kq = _dot(k, q)
         o = [bj + kq * uj for bj, uj in zip(b, u_t)]
         self.log.append((u_t, k, gt))

@@ -113,6 +113,44 @@ def rwkv6_write_not_decayed_order(S, r, k, v, w, u):
     return S_new, o
 
 
+# ---- GDN-2 mutants -------------------------------------------------------
+
+def _gdn2_parts(S, k, alpha):
+    d = k.shape[-1]
+    return _eye(d), np.asarray(S) @ (np.asarray(alpha)[:, :, None] * _eye(d))
+
+
+def gdn2_erase_transposed(S, q, k, v, alpha, b, w):
+    # the other placement of the gate: S' (I - k (b o k)^T)
+    eye, P = _gdn2_parts(S, k, alpha)
+    S_new = P @ (eye - k[:, :, None] * (b * k)[:, None, :]) + (w * v)[:, :, None] * k[:, None, :]
+    return S_new, (S_new @ q[:, :, None])[:, :, 0]
+
+
+def gdn2_erase_ungated(S, q, k, v, alpha, b, w):
+    eye, P = _gdn2_parts(S, k, alpha)
+    S_new = P @ (eye - k[:, :, None] * k[:, None, :]) + (w * v)[:, :, None] * k[:, None, :]
+    return S_new, (S_new @ q[:, :, None])[:, :, 0]
+
+
+def gdn2_write_ungated(S, q, k, v, alpha, b, w):
+    eye, P = _gdn2_parts(S, k, alpha)
+    S_new = P @ (eye - (b * k)[:, :, None] * k[:, None, :]) + v[:, :, None] * k[:, None, :]
+    return S_new, (S_new @ q[:, :, None])[:, :, 0]
+
+
+def gdn2_decay_after_erase(S, q, k, v, alpha, b, w):
+    eye, _ = _gdn2_parts(S, k, alpha)
+    S_new = (np.asarray(S) @ (eye - (b * k)[:, :, None] * k[:, None, :])) @ \
+        (np.asarray(alpha)[:, :, None] * eye) + (w * v)[:, :, None] * k[:, None, :]
+    return S_new, (S_new @ q[:, :, None])[:, :, 0]
+
+
+def gdn2_readout_before_update(S, q, k, v, alpha, b, w):
+    S_new, _ = rec.gdn2_step(S, q, k, v, alpha, b, w)
+    return S_new, (np.asarray(S) @ q[:, :, None])[:, :, 0]
+
+
 MUTANTS = {
     "gdn_no_beta_on_write": ("gdn_step", gdn_no_beta_on_write),
     "gdn_plus_projection": ("gdn_step", gdn_plus_projection),
@@ -129,6 +167,11 @@ MUTANTS = {
     "rwkv6_decay_on_value_axis": ("rwkv6_step", rwkv6_decay_on_value_axis),
     "rwkv6_bonus_without_u": ("rwkv6_step", rwkv6_bonus_without_u),
     "rwkv6_write_not_decayed_order": ("rwkv6_step", rwkv6_write_not_decayed_order),
+    "gdn2_erase_transposed": ("gdn2_step", gdn2_erase_transposed),
+    "gdn2_erase_ungated": ("gdn2_step", gdn2_erase_ungated),
+    "gdn2_write_ungated": ("gdn2_step", gdn2_write_ungated),
+    "gdn2_decay_after_erase": ("gdn2_step", gdn2_decay_after_erase),
+    "gdn2_readout_before_update": ("gdn2_step", gdn2_readout_before_update),
 }
 
 
@@ -136,7 +179,7 @@ MUTANTS = {
 def test_mutant_is_caught(name):
     slot, fn = MUTANTS[name]
     impl = types.SimpleNamespace(gdn_step=rec.gdn_step, kda_step=rec.kda_step,
-                                 rwkv6_step=rec.rwkv6_step)
+                                 rwkv6_step=rec.rwkv6_step, gdn2_step=rec.gdn2_step)
     setattr(impl, slot, fn)
     failed = []
     for pin in pins.PINS:

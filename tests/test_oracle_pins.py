@@ -36,7 +36,7 @@ from oracle import recurrence as rec
 from tests.logform_exact import ExactDeltaLog
 
 REAL = types.SimpleNamespace(gdn_step=rec.gdn_step, kda_step=rec.kda_step,
-                             rwkv6_step=rec.rwkv6_step)
+                             rwkv6_step=rec.rwkv6_step, gdn2_step=rec.gdn2_step)
 
 
 def _fa(rows):
@@ -97,6 +97,23 @@ def pin_rwkv6_hand(impl):
                              _v([F(1, 2), F(1, 3)])[None], _v([2, F(1, 2)])[None])
     np.testing.assert_allclose(o1[0], _v([10, 11]), rtol=0, atol=1e-14)
     np.testing.assert_allclose(S1[0], _fa([[F(7, 2), 2], [-2, F(1, 3)]]), rtol=0, atol=1e-15)
+
+
+def pin_gdn2_hand(impl):
+    # GDN-2, same S0, k, q, v as pin_kda_hand; alpha = (1/2, 1/4), erase gate
+    # b = (1/2, 1/4), write gate w = (1, 1/2).
+    # P = S0 Diag(alpha) = [[1/2, 1/2], [3/2, 1]];  b o k = (3/10, 1/5)
+    # P (b o k) = (1/4, 13/20);  w o v = (2, 1/2);  u = w o v - P (b o k) = (7/4, -3/20)
+    # S1 = P + u k^T = [[31/20, 19/10], [141/100, 22/25]],  o1 = S1 (1, -1) = (-7/20, 53/100).
+    # (Check by the projection form: P (I - (b o k) k^T) = [[7/20, 3/10], [111/100, 12/25]],
+    #  plus (w o v) k^T = [[6/5, 8/5], [3/10, 2/5]] -- same matrix.)
+    S = _fa([[1, 2], [3, 4]])[None]
+    S1, o1 = impl.gdn2_step(S, _v([1, -1])[None], _v([F(3, 5), F(4, 5)])[None], _v([2, 1])[None],
+                            _v([F(1, 2), F(1, 4)])[None], _v([F(1, 2), F(1, 4)])[None],
+                            _v([1, F(1, 2)])[None])
+    np.testing.assert_allclose(S1[0], _fa([[F(31, 20), F(19, 10)], [F(141, 100), F(22, 25)]]),
+                               rtol=0, atol=1e-15)
+    np.testing.assert_allclose(o1[0], _v([F(-7, 20), F(53, 100)]), rtol=0, atol=1e-15)
 
 
 # ------------------------------------------------------------- closed forms
@@ -220,6 +237,46 @@ def pin_kda_constant_decay_is_gdn(impl):
         np.testing.assert_allclose(o_k, o_g, rtol=1e-12, atol=1e-13)
 
 
+def pin_gdn2_equal_gates_is_kda(impl):
+    # both gates the same scalar beta: GDN-2 is KDA (Gated DeltaNet-2 abstract)
+    rng = np.random.default_rng(17)
+    N, d, T = 3, 8, 6
+    S_2 = S_k = rng.standard_normal((N, d, d))
+    for _ in range(T):
+        q, k = _unit(rng, N, d), _unit(rng, N, d)
+        v = rng.standard_normal((N, d))
+        a, b = rng.uniform(0.8, 1.0, (N, d)), rng.uniform(0, 1, N)
+        gate = np.repeat(b[:, None], d, axis=1)
+        S_2, o_2 = impl.gdn2_step(S_2, q, k, v, a, gate, gate)
+        S_k, o_k = impl.kda_step(S_k, q, k, v, a, b)
+        np.testing.assert_allclose(S_2, S_k, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(o_2, o_k, rtol=1e-12, atol=1e-13)
+
+
+def pin_gdn2_open_erase_retrieves_gated_value(impl):
+    # b = 1 and |k| = 1: the erase removes exactly what the decayed state
+    # returns for k, so S_t k = w o v whatever S_{t-1} and alpha are
+    rng = np.random.default_rng(18)
+    N, dk, dv = 4, 6, 5
+    S = rng.standard_normal((N, dv, dk))
+    k = _unit(rng, N, dk)
+    v, w = rng.standard_normal((N, dv)), rng.uniform(0, 1, (N, dv))
+    S1, _ = impl.gdn2_step(S, _unit(rng, N, dk), k, v, rng.uniform(0.5, 1.0, (N, dk)),
+                           np.ones((N, dk)), w)
+    np.testing.assert_allclose(np.einsum("nvk,nk->nv", S1, k), w * v, rtol=1e-12, atol=1e-12)
+
+
+def pin_gdn2_closed_gates_is_pure_decay(impl):
+    # b = 0 and w = 0: no erase, no write, S_t = S_{t-1} Diag(alpha)
+    rng = np.random.default_rng(19)
+    N, dk, dv = 3, 5, 4
+    S = rng.standard_normal((N, dv, dk))
+    a = rng.uniform(0.5, 1.0, (N, dk))
+    S1, o1 = impl.gdn2_step(S, _unit(rng, N, dk), _unit(rng, N, dk), rng.standard_normal((N, dv)),
+                            a, np.zeros((N, dk)), np.zeros((N, dv)))
+    np.testing.assert_allclose(S1, S * a[:, None, :], rtol=1e-14, atol=0)
+
+
 # ------------------------------------------------- exact log form vs oracle
 
 def _rat(rng, shape, den=8, lo=-8, hi=8):
@@ -244,16 +301,23 @@ def _run_exact_vs_oracle(impl, variant, L, fill0, T, d=3, seed=0, merge_every_fu
             dec = F(int(rng.integers(5, 9)), 8)
         else:
             dec = list(np.vectorize(lambda n: F(int(n), 8), otypes=[object])(rng.integers(5, 9, size=d)))
-        beta = F(int(rng.integers(0, 9)), 8)
+        if variant == "gdn2":
+            beta = list(_rat(rng, (d,), lo=0, hi=8))      # erase gate per key channel
+            wgate = list(_rat(rng, (d,), lo=0, hi=8))     # write gate per value row
+        else:
+            beta = F(int(rng.integers(0, 9)), 8)
+            wgate = None
         if dl.fill == L:
             dl.merge()
-        o_ex = dl.step(list(q), list(k), list(v), dec, beta)
+        o_ex = dl.step(list(q), list(k), list(v), dec, beta, wgate)
         f64 = lambda x: np.array(x, dtype=np.float64)[None]
         if variant == "gdn":
             S_or, o_or = impl.gdn_step(S_or, f64(q), f64(k), f64(v), np.array([float(dec)]),
                                        np.array([float(beta)]))
         elif variant == "kda":
             S_or, o_or = impl.kda_step(S_or, f64(q), f64(k), f64(v), f64(dec), np.array([float(beta)]))
+        elif variant == "gdn2":
+            S_or, o_or = impl.gdn2_step(S_or, f64(q), f64(k), f64(v), f64(dec), f64(beta), f64(wgate))
         else:
             S_or, o_or = impl.rwkv6_step(S_or, f64(q), f64(k), f64(v), f64(dec), f64(bonus))
         np.testing.assert_allclose(o_or[0], np.array(o_ex, dtype=np.float64), rtol=1e-12, atol=1e-12)
@@ -263,7 +327,7 @@ def _run_exact_vs_oracle(impl, variant, L, fill0, T, d=3, seed=0, merge_every_fu
 
 
 def pin_log_form_equals_oracle(impl):
-    for variant in ("gdn", "kda", "rwkv6"):
+    for variant in ("gdn", "kda", "rwkv6", "gdn2"):
         for (L, fill0, T) in ((4, 0, 9), (3, 2, 8), (1, 0, 4)):
             _run_exact_vs_oracle(impl, variant, L, fill0, T, seed=L * 10 + fill0)
 
@@ -271,7 +335,8 @@ def pin_log_form_equals_oracle(impl):
 PINS = [pin_gdn_hand, pin_kda_hand, pin_rwkv6_hand, pin_beta_zero_is_pure_decay,
         pin_rwkv6_zero_keys_is_pure_decay, pin_rwkv6_unit_decay_sums_outer_products,
         pin_exact_retrieval, pin_non_expansive_without_writes, pin_kda_constant_decay_is_gdn,
-        pin_log_form_equals_oracle]
+        pin_gdn2_hand, pin_gdn2_equal_gates_is_kda, pin_gdn2_open_erase_retrieves_gated_value,
+        pin_gdn2_closed_gates_is_pure_decay, pin_log_form_equals_oracle]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])

@@ -43,15 +43,21 @@ def test_shapes_dtypes_and_ranges():
             assert s.beta is None and s.decay.shape == (w.B, w.H, w.d_k)
             assert np.all((s.decay > 0) & (s.decay < 1))
         else:
-            assert s.beta.shape == (w.B, w.H)
+            bshape = (w.B, w.H, w.d_k) if w.variant == wl.GDN2 else (w.B, w.H)
+            assert s.beta.shape == bshape
             assert np.all((s.beta > 0) & (s.beta < 1))
             # q and k are unit vectors up to input rounding
             tol = 1e-2 if w.in_dtype == "bf16" else 1e-6
             np.testing.assert_allclose(np.linalg.norm(s.k.astype(np.float64), axis=-1), 1, atol=tol)
             np.testing.assert_allclose(np.linalg.norm(s.q.astype(np.float64), axis=-1), 1, atol=tol)
-        if w.variant == wl.KDA:
+        if w.variant in (wl.KDA, wl.GDN2):
             assert s.decay.shape == (w.B, w.H, w.d_k)
             assert np.all((s.decay >= 0.8) & (s.decay <= 1.0))
+        if w.variant == wl.GDN2:
+            assert s.wgate.shape == (w.B, w.H, w.d_v)
+            assert np.all((s.wgate > 0) & (s.wgate < 1))
+        else:
+            assert s.wgate is None
         if w.variant == wl.GDN:
             assert s.decay.shape == (w.B, w.H)
             assert np.all((s.decay > 0.5) & (s.decay <= 1.0))
