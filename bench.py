@@ -195,7 +195,11 @@ def step_bytes(cfg, fills: np.ndarray, fused: bool) -> tuple:
     uin = ein if cfg.variant == "rwkv6" else 4
     entry = dv * uin + dk * ein + gw * 4
     tile = base_tile_bytes(cfg)
-    vec = (2 * dk + dv) * ein + (4 if cfg.variant == "gdn" else dk * 4) + (4 if cfg.variant != "rwkv6" else 0)
+    vec = (2 * dk + dv) * ein + (4 if cfg.variant == "gdn" else dk * 4)
+    if cfg.variant == "gdn2":
+        vec += dk * 4 + dv * 4            # erase gate b_t [d_k], write gate w_t [d_v]
+    elif cfg.variant != "rwkv6":
+        vec += 4                          # beta
     f = fills.astype(np.int64)
     merging = (f == cfg.L - 1) if fused else np.zeros_like(f, dtype=bool)
     rd = H * (tile + vec + 4 + f * entry)
@@ -220,7 +224,11 @@ def eager_bytes(cfg) -> tuple:
     ein = 2 if cfg.in_dtype == "bf16" else 4
     dk, dv = cfg.d_k, cfg.d_v
     tile = dv * dk * 4
-    vec = (2 * dk + dv) * ein + 8
+    vec = (2 * dk + dv) * ein + (4 if cfg.variant == "gdn" else dk * 4)
+    if cfg.variant == "gdn2":
+        vec += dk * 4 + dv * 4            # erase gate b_t [d_k], write gate w_t [d_v]
+    elif cfg.variant != "rwkv6":
+        vec += 4                          # beta
     return cfg.heads * (tile + vec), cfg.heads * (tile + dv * 4)
 
 
@@ -251,8 +259,8 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
     for r in range(reps):
         st.reset(S0, [0] * w.B)
         for i in range(w.L):
-            q, k, v, dec, beta = ring[i % len(ring)]
-            st.step(q, k, v, dec, beta, bonus, o)
+            q, k, v, dec, beta, wg = ring[i % len(ring)]
+            st.step(q, k, v, dec, beta, wg if wg is not None else bonus, o)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         st.merge(dlb.DL_MERGE_FULL)
@@ -264,8 +272,8 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
     st.reset(S0, [0] * w.B)
     half = w.L // 2
     for i in range(half):
-        q, k, v, dec, beta = ring[i % len(ring)]
-        st.step(q, k, v, dec, beta, bonus, o)
+        q, k, v, dec, beta, wg = ring[i % len(ring)]
+        st.step(q, k, v, dec, beta, wg if wg is not None else bonus, o)
     out = torch.empty(w.heads * w.d_v * w.d_k, dtype=torch.float32, device=device)
     st.materialize(out)
     torch.cuda.synchronize(device)
@@ -306,7 +314,7 @@ def to_dev(s, device):
             return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(device).view(torch.bfloat16).reshape(-1)
         return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device).reshape(-1)
     return (up(s.device_array("q")), up(s.device_array("k")), up(s.device_array("v")),
-            up(s.decay), up(s.beta))
+            up(s.decay), up(s.beta), up(s.wgate))
 
 
 def run_ours(args, world, rank, local):
@@ -341,10 +349,10 @@ def run_ours(args, world, rank, local):
     o = torch.empty(w.heads * w.d_v, dtype=torch.float32, device=device)
 
     def one_step(i, ev=None):
-        q, k, v, dec, beta = ring[i % RING]
+        q, k, v, dec, beta, wg = ring[i % RING]
         if ev is not None:
             ev[0].record(stream)
-        st.step(q, k, v, dec, beta, bonus, o)
+        st.step(q, k, v, dec, beta, wg if wg is not None else bonus, o)
         if ev is not None:
             ev[1].record(stream)
         if not fused:
@@ -420,14 +428,14 @@ def run_ours(args, world, rank, local):
     # eager dense step on a separate 1 GiB state, same inputs
     S_e = S0.clone()
     for i in range(args.warmup):
-        q, k, v, dec, beta = ring[i % RING]
-        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, bonus, o)
+        q, k, v, dec, beta, wg = ring[i % RING]
+        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, wg if wg is not None else bonus, o)
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
-        q, k, v, dec, beta = ring[i % RING]
-        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, bonus, o)
+        q, k, v, dec, beta, wg = ring[i % RING]
+        dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, wg if wg is not None else bonus, o)
     e1.record(stream)
     torch.cuda.synchronize(device)
     eager_s = e0.elapsed_time(e1) / 1e3
@@ -451,9 +459,15 @@ def run_ours(args, world, rank, local):
         a = np.ascontiguousarray(a if a.dtype == np.uint16 else a.astype(np.float32))
         return a.view(np.uint8).reshape(-1)
 
-    parts0 = [_bytes(x) for x in (host_steps[0].device_array("q"), host_steps[0].device_array("k"),
-                                 host_steps[0].device_array("v"), host_steps[0].decay)
-              + ((host_steps[0].beta,) if host_steps[0].beta is not None else ())]
+    def _parts(s):
+        ps = [s.device_array("q"), s.device_array("k"), s.device_array("v"), s.decay]
+        if s.beta is not None:
+            ps.append(s.beta)
+        if s.wgate is not None:
+            ps.append(s.wgate)
+        return ps
+
+    parts0 = [_bytes(x) for x in _parts(host_steps[0])]
     offs, total = [], 0
     for part in parts0:
         offs.append(total)
@@ -461,10 +475,7 @@ def run_ours(args, world, rank, local):
     pinned = []
     for s in host_steps:
         buf = np.zeros(total, dtype=np.uint8)
-        parts = [s.device_array("q"), s.device_array("k"), s.device_array("v"), s.decay]
-        if s.beta is not None:
-            parts.append(s.beta)
-        for off, part in zip(offs, parts):
+        for off, part in zip(offs, _parts(s)):
             pb = _bytes(part)
             buf[off:off + pb.size] = pb
         pinned.append(torch.from_numpy(buf).pin_memory())
@@ -478,7 +489,7 @@ def run_ours(args, world, rank, local):
         for j, (off, part) in enumerate(zip(offs, parts0)):
             raw = d[off:off + part.size]
             views.append(raw.view(tin) if j < 3 else raw.view(torch.float32))
-        if len(views) == 4:
+        while len(views) < 6:
             views.append(None)
         dviews.append(views)
     obufs = [torch.empty(o.numel(), dtype=torch.float32, device=device) for _ in range(NB)]
@@ -500,8 +511,8 @@ def run_ours(args, world, rank, local):
         ev_h2d[b].record(s_h2d)
         s_cmp.wait_event(ev_h2d[b])
         s_cmp.wait_event(ev_d2h[b])          # step i-NB's output has left obufs[b]
-        q, k, v, dec, beta = dviews[b]
-        st.step(q, k, v, dec, beta, bonus, obufs[b], stream=s_cmp)
+        q, k, v, dec, beta, wg = dviews[b]
+        st.step(q, k, v, dec, beta, wg if wg is not None else bonus, obufs[b], stream=s_cmp)
         if not fused:
             st.merge(dlb.DL_MERGE_FULL, stream=s_cmp)
         ev_cmp[b].record(s_cmp)
@@ -612,9 +623,9 @@ def run_serving(args, world, rank, local):
             seqs = rng.choice(w.B, size=churn, replace=False).tolist()
             for st in layers:
                 st.load_seqs(seqs)
-        q, k, v, dec, beta = ring[i % RING]
+        q, k, v, dec, beta, wg = ring[i % RING]
         for st in layers:
-            st.step(q, k, v, dec, beta, bonus, o)
+            st.step(q, k, v, dec, beta, wg if wg is not None else bonus, o)
 
     for i in range(args.warmup):
         token_step(i)
@@ -662,9 +673,10 @@ def oracle_tokens_per_s(w, target_s: float = 0.0, seqs: int = 2, steps: int = 0,
     while (done < steps) if steps > 0 else (el < target_s):
         s = wl.step_inputs(w, t)
         sl = lambda x: None if x is None else x.reshape((w.heads,) + x.shape[2:])[heads][:, None]
-        st = types.SimpleNamespace(q=sl(s.q), k=sl(s.k), v=sl(s.v), decay=sl(s.decay), beta=sl(s.beta))
+        st = types.SimpleNamespace(q=sl(s.q), k=sl(s.k), v=sl(s.v), decay=sl(s.decay), beta=sl(s.beta),
+                                   wgate=sl(s.wgate))
         a = time.perf_counter()
-        S = oracle.run_eager(w.variant, S, [st], bonus=bonus).S
+        S = oracle.run_eager(w.variant, S, [st], bonus=bonus, kla_eps=w.kla_eps).S
         dt = time.perf_counter() - a
         t += 1
         if t > warmup:

@@ -16,6 +16,9 @@
  *   RWKV6 (stored as the transpose of its d_k x d_v matrix)
  *         S_t = S_{t-1} Diag(w_t) + v_t k_t^T,
  *         o_t = S_{t-1} r_t + (sum_c r_c u_c k_c) v_t
+ *   GDN-2 S_t = S_{t-1} Diag(a_t) (I - (e_t o k_t) k_t^T) + (w_t o v_t) k_t^T,
+ *         o_t = S_t q_t   (e_t: erase gate per key channel, w_t: write gate
+ *         per value row; the log is KDA's, u_t = w_t o v_t - S' (e_t o k_t))
  * With gamma_t the decay accumulated since the base was last merged and
  * u_t = b_t (v_t - a_t S_{t-1} k_t) (GDN; KDA uses S_{t-1}(a_t o k_t)),
  *   S_t = S_b Diag(gamma_t) + sum_i u_i (k_i o gamma_t / gamma_i)^T,
@@ -46,8 +49,10 @@
 extern "C" {
 #endif
 
-/* Recurrence family ("We implement DeltaLog for GDN, KDA, and RWKV6"). */
-enum dl_variant { DL_GDN = 0, DL_KDA = 1, DL_RWKV6 = 2 };
+/* Recurrence family ("We implement DeltaLog for GDN, KDA, and RWKV6"), plus
+ * GDN-2 (Gated DeltaNet-2 abstract: separate channel-wise erase and write
+ * gates; KDA when both are the same scalar). */
+enum dl_variant { DL_GDN = 0, DL_KDA = 1, DL_RWKV6 = 2, DL_GDN2 = 3 };
 
 /* Element type of q (r), k and v as stored by the caller. */
 enum dl_dtype { DL_F32 = 0, DL_BF16 = 1 };
@@ -78,12 +83,14 @@ enum dl_flags {
   /* Run the step as a persistent warp-specialised kernel (one CTA per SM, a
    * producer lane streaming work items through a ring of shared-memory
    * stages) when its ring fits, instead of one CTA per work item.  A
-   * performance choice only; on B200 the default measured faster. */
+   * performance choice only; on B200 the default measured faster.  fp32
+   * base and GDN / KDA / RWKV6 only (else DL_ERR_UNSUPPORTED). */
   DL_FLAG_PERSISTENT = 2,
   /* Kaczmarz step size (KLA, GDN and KDA only): the `beta` argument of a
    * step carries the gate eta_t and the kernels use
    * beta_t = eta_t / (|k_t|_2^2 + kla_eps) ("Kaczmarz Linear Attention"
-   * abstract), so the write projects exactly whatever the key's norm. */
+   * abstract), so the write projects exactly whatever the key's norm.
+   * Not for RWKV6 or GDN-2 (DL_ERR_ARG). */
   DL_FLAG_KLA = 4,
   /* int8 base quantized once per window ("LeapQuant" abstract: the state
    * is quantized only at the end of a window of tokens, and outputs inside
@@ -166,10 +173,12 @@ int dl_state_load_seqs(dl_state* st, int n, const int32_t* seqs, const float* S,
  *   q: q_t (r_t for RWKV6)  [B, H, d_k] in_dtype
  *   k: k_t                  [B, H, d_k] in_dtype
  *   v: v_t                  [B, H, d_v] in_dtype
- *   decay: fp32, GDN alpha_t [B, H]; KDA alpha_t [B, H, d_k];
+ *   decay: fp32, GDN alpha_t [B, H]; KDA and GDN-2 alpha_t [B, H, d_k];
  *          RWKV6 w_t [B, H, d_k]; every value in (0, 1]
- *   beta: fp32 [B, H] for GDN/KDA; ignored (may be NULL) for RWKV6
- *   bonus: fp32 [H, d_k] RWKV6 u; ignored (may be NULL) otherwise
+ *   beta: fp32 [B, H] for GDN/KDA; GDN-2: the erase gate e_t [B, H, d_k];
+ *         ignored (may be NULL) for RWKV6
+ *   bonus: fp32 [H, d_k] RWKV6 u; GDN-2: the write gate w_t [B, H, d_v];
+ *          ignored (may be NULL) otherwise
  *   o: fp32 [B, H, d_v] output o_t
  * All pointers 16-byte aligned device addresses.  Without
  * DL_FLAG_FUSED_MERGE, returns DL_ERR_LOG_FULL (enqueuing nothing) when

@@ -74,21 +74,23 @@ bool head_size_ok(int d) { return d == 64 || d == 128; }
 // Shape checks shared by every call.  `need_L`: whether L matters.
 int check_config(const dl_config* c, bool need_L) {
   if (c == nullptr) return DL_ERR_ARG;
-  if (c->variant < DL_GDN || c->variant > DL_RWKV6) return DL_ERR_ARG;
+  if (c->variant < DL_GDN || c->variant > DL_GDN2) return DL_ERR_ARG;
   if (c->B < 1 || c->H < 1 || c->d_k < 1 || c->d_v < 1) return DL_ERR_ARG;
   if (c->in_dtype != DL_F32 && c->in_dtype != DL_BF16) return DL_ERR_ARG;
   if (need_L && (c->L < 1 || c->L > 64)) return DL_ERR_ARG;
   if ((c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_PERSISTENT | DL_FLAG_KLA |
                            DL_FLAG_BASE_Q8)) != 0)
     return DL_ERR_ARG;
-  if ((c->flags & DL_FLAG_KLA) && (c->variant == DL_RWKV6 || !(c->kla_eps >= 0.f)))
+  if ((c->flags & DL_FLAG_KLA) &&
+      (c->variant == DL_RWKV6 || c->variant == DL_GDN2 || !(c->kla_eps >= 0.f)))
     return DL_ERR_ARG;
   const uint64_t bh = uint64_t(c->B) * uint64_t(c->H);
   if (bh > 0x7fffffffull) return DL_ERR_ARG;  // one CTA per head in a 1-D grid
   if (bh * uint64_t(c->d_v) * uint64_t(c->d_k) >= (1ull << 40)) return DL_ERR_ARG;
   if (!head_size_ok(c->d_k) || !head_size_ok(c->d_v)) return DL_ERR_UNSUPPORTED;
   if (c->step_split != 0 && !dl::split_ok(c->d_v, c->step_split)) return DL_ERR_ARG;
-  if ((c->flags & DL_FLAG_BASE_Q8) && (c->flags & DL_FLAG_PERSISTENT)) return DL_ERR_UNSUPPORTED;
+  if ((c->flags & DL_FLAG_PERSISTENT) && ((c->flags & DL_FLAG_BASE_Q8) || c->variant == DL_GDN2))
+    return DL_ERR_UNSUPPORTED;
   return DL_OK;
 }
 
@@ -106,12 +108,14 @@ cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, const dl::F
     switch (c.variant) {
       case DL_GDN: return dl::launch_step<dl::kVarGDN, int8_t>(sh, fused, p, fp, n, s);
       case DL_KDA: return dl::launch_step<dl::kVarKDA, int8_t>(sh, fused, p, fp, n, s);
+      case DL_GDN2: return dl::launch_step<dl::kVarGDN2, int8_t>(sh, fused, p, fp, n, s);
       default: return dl::launch_step<dl::kVarRWKV6, int8_t>(sh, fused, p, fp, n, s);
     }
   }
   switch (c.variant) {
     case DL_GDN: return dl::launch_step<dl::kVarGDN, float>(sh, fused, p, fp, n, s);
     case DL_KDA: return dl::launch_step<dl::kVarKDA, float>(sh, fused, p, fp, n, s);
+    case DL_GDN2: return dl::launch_step<dl::kVarGDN2, float>(sh, fused, p, fp, n, s);
     default: return dl::launch_step<dl::kVarRWKV6, float>(sh, fused, p, fp, n, s);
   }
 }
@@ -124,12 +128,14 @@ cudaError_t launch_merge(const dl_config& c, const dl::MergeParams& p, const dl:
     switch (c.variant) {
       case DL_GDN: return dl::launch_merge<dl::kVarGDN, int8_t>(sh, p, list, nctas, s);
       case DL_KDA: return dl::launch_merge<dl::kVarKDA, int8_t>(sh, p, list, nctas, s);
+      case DL_GDN2: return dl::launch_merge<dl::kVarGDN2, int8_t>(sh, p, list, nctas, s);
       default: return dl::launch_merge<dl::kVarRWKV6, int8_t>(sh, p, list, nctas, s);
     }
   }
   switch (c.variant) {
     case DL_GDN: return dl::launch_merge<dl::kVarGDN, float>(sh, p, list, nctas, s);
     case DL_KDA: return dl::launch_merge<dl::kVarKDA, float>(sh, p, list, nctas, s);
+    case DL_GDN2: return dl::launch_merge<dl::kVarGDN2, float>(sh, p, list, nctas, s);
     default: return dl::launch_merge<dl::kVarRWKV6, float>(sh, p, list, nctas, s);
   }
 }
@@ -148,12 +154,14 @@ size_t smem_need(const dl_config& c) {
     switch (c.variant) {
       case DL_GDN: return smem_need<dl::kVarGDN, int8_t>(sh, c.L);
       case DL_KDA: return smem_need<dl::kVarKDA, int8_t>(sh, c.L);
+      case DL_GDN2: return smem_need<dl::kVarGDN2, int8_t>(sh, c.L);
       default: return smem_need<dl::kVarRWKV6, int8_t>(sh, c.L);
     }
   }
   switch (c.variant) {
     case DL_GDN: return smem_need<dl::kVarGDN, float>(sh, c.L);
     case DL_KDA: return smem_need<dl::kVarKDA, float>(sh, c.L);
+    case DL_GDN2: return smem_need<dl::kVarGDN2, float>(sh, c.L);
     default: return smem_need<dl::kVarRWKV6, float>(sh, c.L);
   }
 }
@@ -163,6 +171,7 @@ cudaError_t launch_eager(const dl_config& c, const dl::EagerParams& p, cudaStrea
   switch (c.variant) {
     case DL_GDN: return dl::launch_eager<dl::kVarGDN>(shape_of(c), p, n, s);
     case DL_KDA: return dl::launch_eager<dl::kVarKDA>(shape_of(c), p, n, s);
+    case DL_GDN2: return dl::launch_eager<dl::kVarGDN2>(shape_of(c), p, n, s);
     default: return dl::launch_eager<dl::kVarRWKV6>(shape_of(c), p, n, s);
   }
 }
@@ -184,11 +193,13 @@ int* global_err_word() {
 int check_step_args(const dl_config& c, const void* q, const void* k, const void* v,
                     const float* decay, const float* beta, const float* bonus, const float* o) {
   if (!q || !k || !v || !decay || !o) return DL_ERR_ARG;
-  if (c.variant == DL_RWKV6 ? (bonus == nullptr) : (beta == nullptr)) return DL_ERR_ARG;
+  const bool need_bonus = c.variant == DL_RWKV6 || c.variant == DL_GDN2;
+  const bool need_beta = c.variant != DL_RWKV6;
+  if ((need_bonus && bonus == nullptr) || (need_beta && beta == nullptr)) return DL_ERR_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(decay, 16) ||
       !aligned(o, 16))
     return DL_ERR_ALIGN;
-  if (c.variant == DL_RWKV6 ? !aligned(bonus, 16) : !aligned(beta, 16)) return DL_ERR_ALIGN;
+  if ((need_bonus && !aligned(bonus, 16)) || (need_beta && !aligned(beta, 16))) return DL_ERR_ALIGN;
   return DL_OK;
 }
 

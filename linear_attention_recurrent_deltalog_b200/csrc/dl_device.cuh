@@ -16,6 +16,7 @@ namespace dl {
 constexpr int kVarGDN = 0;
 constexpr int kVarKDA = 1;
 constexpr int kVarRWKV6 = 2;
+constexpr int kVarGDN2 = 3;  // GDN-2: KDA's log and decay, separate erase / write gates
 
 // Device error codes written to the error word.
 constexpr int kDevErrTimeout = 1;   // a bounded mbarrier wait gave up

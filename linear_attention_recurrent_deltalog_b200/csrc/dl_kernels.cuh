@@ -156,19 +156,26 @@ __device__ __forceinline__ uint32_t g_copy_bytes(int f) {
 template <int VAR, int DK, typename TK, typename TIn>
 __device__ __forceinline__ void entry_weights(int f, int warp, int nwarps, int lane, const TK* kin,
                                               const TK* qin, const TIn* sK, const float* sG,
-                                              const float* dec, float* sW, float* sZ) {
+                                              const float* dec, float* sW, float* sZ,
+                                              const float* kgate = nullptr) {
   constexpr int CPE = DK / 8;  // channels per lane
   const int slot = lane >> 3;
   const int c0 = (lane & 7) * CPE;
   float kl[CPE], ql[CPE], gl[CPE];
   load_f<CPE>(kin + c0, kl);
   load_f<CPE>(qin + c0, ql);
+  if (VAR == kVarGDN2) {  // GDN-2 reads through the gated key b o k
+    float bg[CPE];
+    load_f<CPE>(kgate + c0, bg);
+#pragma unroll
+    for (int c = 0; c < CPE; ++c) kl[c] *= bg[c];
+  }
   float gt0 = 0.f;
   if (VAR == kVarGDN) {
     gt0 = sG[f - 1] + logf(dec[0]);
   } else {
     load_f<CPE>(sG + size_t(f - 1) * DK + c0, gl);
-    if (VAR == kVarKDA) {
+    if (VAR == kVarKDA || VAR == kVarGDN2) {
       float dl[CPE];
       load_f<CPE>(dec + c0, dl);
 #pragma unroll
@@ -254,6 +261,7 @@ __device__ __forceinline__ void rows_gemv(const float* sS, int j0, int lane, con
 //   sums each for instruction-level parallelism), then
 //   GDN  : u = beta (v - gamma a - ck),  o = gamma b + cq + (k.q) u
 //   KDA  : u = beta (v - a - ck),        o = b + cq + (k.q) u
+//   GDN-2: u = (w o v) - a - ck,         o = b + cq + (k.q) u  (vj is w_j v_j)
 //   RWKV6: u = v,                        o = b + cq + bonus v
 // sScal: [0] k.q or the RWKV6 bonus, [1] beta, [2] gamma = e^{g_t} (GDN).
 template <int VAR, typename TU>
@@ -286,6 +294,9 @@ __device__ __forceinline__ void row_update(const TU* sU, int jl, int f, int L, c
     o = gamma * b + cq + sdot * u;
   } else if (VAR == kVarKDA) {
     u = sScal[1] * (vj - a - ck);
+    o = b + cq + sdot * u;
+  } else if (VAR == kVarGDN2) {
+    u = vj - a - ck;
     o = b + cq + sdot * u;
   } else {
     u = vj;
@@ -601,7 +612,7 @@ struct StepLayout {
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
   static constexpr bool Q8 = std::is_same<TB, int8_t>::value;
   size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offBonus,
-      offScale, offVecH, offDecF, offKt, offBar, total;
+      offWg, offScale, offVecH, offDecF, offKt, offBar, total;
   __host__ __device__ explicit StepLayout(int L) {
     offU = Tile<DK, ROWS, TB>::kTileBytes;
     offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
@@ -617,8 +628,11 @@ struct StepLayout {
     offScal = offZ + align_up(size_t(L) * 4, 16);
     // int8 base: the CTA's row scales, the GEMV's fp16 vectors [4][DK], the
     // base decay [DK] and, for the fused merge, the staged key fragments
+    // RWKV6: the bonus u [DK]; GDN-2: the erase gate b [DK] and this CTA's
+    // rows of the write gate w [ROWS]
     offBonus = offScal + 64;
-    offScale = offBonus + (VAR == kVarRWKV6 ? align_up(size_t(DK) * 4, 128) : 0);
+    offWg = offBonus + ((VAR == kVarRWKV6 || VAR == kVarGDN2) ? align_up(size_t(DK) * 4, 128) : 0);
+    offScale = offWg + (VAR == kVarGDN2 ? align_up(size_t(ROWS) * 4, 128) : 0);
     offVecH = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
     offDecF = offVecH + (Q8 ? align_up(size_t(4) * kVecHStride<DK> * 2, 128) : 0);
     offKt = offDecF + (Q8 ? align_up(size_t(DK) * 4, 128) : 0);
@@ -673,7 +687,8 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   float* sZ = reinterpret_cast<float*>(smem + lay.offZ);      // per-entry weights on q / r
   float* sScal = reinterpret_cast<float*>(smem + lay.offScal);  // [0] k.q / bonus [1] beta
                                                                 // [2] e^{g_t}
-  float* sBonus = reinterpret_cast<float*>(smem + lay.offBonus);  // RWKV6: u [DK]
+  float* sBonus = reinterpret_cast<float*>(smem + lay.offBonus);  // RWKV6: u; GDN-2: b [DK]
+  float* sWg = reinterpret_cast<float*>(smem + lay.offWg);        // GDN-2: w, this CTA's rows
   float* sScale = reinterpret_cast<float*>(smem + lay.offScale);  // int8 base: row scales
   __half* sVecH = reinterpret_cast<__half*>(smem + lay.offVecH);  // GEMV vectors, fp16 hi/lo
   float* sDecF = reinterpret_cast<float*>(smem + lay.offDecF);    // fused merge: base decay
@@ -706,7 +721,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   // scalars no bulk copy can carry (GDN's decay, beta) into registers, so
   // no barrier waits on those loads.
   const float dec_s = (GW == 1) ? __ldg(p.decay + head) : 0.f;
-  const float beta_s = (VAR == kVarRWKV6) ? 0.f : __ldg(p.beta + head);
+  const float beta_s = (VAR == kVarRWKV6 || VAR == kVarGDN2) ? 0.f : __ldg(p.beta + head);
   if (warp == 0 && lane == 0) {
 #pragma unroll
     for (int c = 0; c < Tl::kChunks; ++c) mbar_init(&bars[c], 1);
@@ -727,11 +742,16 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
     const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
     const uint32_t bs = Q8 ? ROWS * 4u : 0u;
-    const uint32_t bb = (VAR == kVarRWKV6) ? DK * 4u : 0u;
+    const uint32_t bb = (VAR == kVarRWKV6 || VAR == kVarGDN2) ? DK * 4u : 0u;
+    const uint32_t bw = (VAR == kVarGDN2) ? ROWS * 4u : 0u;
     mbar_arrive_expect_tx(barLog,
-                          2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg + bs + bb);
+                          2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg + bs + bb + bw);
     if (Q8) tma_load_1d(sScale, p.scale + head * DV + r0, bs, barLog);
     if (VAR == kVarRWKV6) tma_load_1d(sBonus, p.bonus + size_t(h) * DK, bb, barLog);
+    if (VAR == kVarGDN2) {
+      tma_load_1d(sBonus, p.beta + head * DK, bb, barLog);        // erase gate b_t
+      tma_load_1d(sWg, p.bonus + head * DV + r0, bw, barLog);      // write gate w_t rows
+    }
     tma_load_1d(sQr, static_cast<const TIn*>(p.q) + head * DK, bq, barLog);
     tma_load_1d(sKr, static_cast<const TIn*>(p.k) + head * DK, bq, barLog);
     tma_load_1d(sVr, static_cast<const TIn*>(p.v) + head * DV + r0, bv, barLog);
@@ -760,9 +780,9 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       const float gt = gp + logf(sDecV[c]);
       sGp[c] = gp;
       sGt[c] = gt;
-      if (VAR == kVarKDA) {
+      if (VAR == kVarKDA || VAR == kVarGDN2) {
         const float e = expf(gt);
-        sKh[c] = e * kc;
+        sKh[c] = (VAR == kVarGDN2) ? e * (sBonus[c] * kc) : e * kc;
         sQh[c] = e * qc;
       } else {  // RWKV6 reads S_{t-1}: decay up to the previous step
         sQh[c] = expf(gp) * qc;
@@ -774,7 +794,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     else if (appender)
       gK[size_t(f) * DK + c] = kraw;
     if constexpr (Q8) {  // the GEMV's B columns: k-hat and q-hat as fp16 hi/lo pairs
-      const float va = (VAR == kVarGDN) ? kc : (VAR == kVarKDA ? sKh[c] : 0.f);
+      const float va = (VAR == kVarGDN) ? kc : (VAR == kVarRWKV6 ? 0.f : sKh[c]);
       const float vb = (VAR == kVarGDN) ? qc : sQh[c];
       uint32_t hi, lo;
       split_h2(va, vb, hi, lo);
@@ -796,7 +816,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   }
   if (f > 0)
     entry_weights<VAR, DK, TIn, TIn>(f, warp, NW, lane, sKr, sQr, sK, sG,
-                                     (GW == 1) ? &dec_s : sDecV, sW, sZ);
+                                     (GW == 1) ? &dec_s : sDecV, sW, sZ, sBonus);
   if (warp == NW - 1) {
     // GDN/KDA: k_t . q_t (the current entry's own weight on q) and, for the
     // KLA step size, |k_t|^2; RWKV6: the bonus sum_c r_c u_c k_c.
@@ -844,7 +864,8 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     owner = (lane & 1) == 0;
   }
   float u, o;
-  row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, to_f(sVr[jl]), a, b, u, o);
+  const float vj = (VAR == kVarGDN2) ? sWg[jl] * to_f(sVr[jl]) : to_f(sVr[jl]);
+  row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, vj, a, b, u, o);
   if (owner) {
     p.o[head * DV + r0 + jl] = o;
     if (merge_now)
@@ -1125,8 +1146,8 @@ dl_eager_kernel(const EagerParams p) {
     sk[c] = kc;
     sq[c] = qc;
     sDec[c] = dc;
-    if (VAR == kVarKDA) {  // S Diag(alpha) k and S Diag(alpha) q
-      sKh[c] = dc * kc;
+    if (VAR == kVarKDA || VAR == kVarGDN2) {  // S Diag(alpha) k and S Diag(alpha) q
+      sKh[c] = (VAR == kVarGDN2) ? dc * (p.beta[head * DK + c] * kc) : dc * kc;  // GDN-2: b o k
       sQh[c] = dc * qc;
     } else {               // GDN scales after the GEMV; RWKV6 reads S_{t-1}
       sKh[c] = kc;
@@ -1135,7 +1156,7 @@ dl_eager_kernel(const EagerParams p) {
   }
   for (int j = tid - 32; j < DV; j += NT - 32) {
     if (j < 0) break;
-    sV[j] = to_f(gv[j]);
+    sV[j] = (VAR == kVarGDN2) ? p.bonus[head * DV + j] * to_f(gv[j]) : to_f(gv[j]);  // GDN-2: w o v
   }
   __syncthreads();
   if (warp == NW - 1) {
@@ -1151,7 +1172,7 @@ dl_eager_kernel(const EagerParams p) {
     if (VAR != kVarRWKV6 && p.kla) kk = warp_sum(kk);
     if (lane == 0) {
       sScal[0] = x;
-      sScal[1] = (VAR == kVarRWKV6) ? 0.f
+      sScal[1] = (VAR == kVarRWKV6 || VAR == kVarGDN2) ? 0.f
                  : (p.kla ? p.beta[head] / (kk + p.kla_eps) : p.beta[head]);
       sScal[2] = (VAR == kVarGDN) ? p.decay[head] : 1.f;
     }
@@ -1176,6 +1197,9 @@ dl_eager_kernel(const EagerParams p) {
     o = alpha * b + sdot * u;
   } else if (VAR == kVarKDA) {
     u = sScal[1] * (vj - a);
+    o = b + sdot * u;
+  } else if (VAR == kVarGDN2) {  // vj is w_j v_j
+    u = vj - a;
     o = b + sdot * u;
   } else {
     u = vj;

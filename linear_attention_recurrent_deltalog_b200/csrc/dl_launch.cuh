@@ -146,6 +146,7 @@ size_t merge_smem_bytes(const Shape& sh, int L);
 DL_DECLARE_VARIANT_LAUNCHERS(kVarGDN)
 DL_DECLARE_VARIANT_LAUNCHERS(kVarKDA)
 DL_DECLARE_VARIANT_LAUNCHERS(kVarRWKV6)
+DL_DECLARE_VARIANT_LAUNCHERS(kVarGDN2)
 
 // Functors the shape dispatch calls (namespace scope: local classes cannot
 // have member templates).
@@ -203,7 +204,7 @@ cudaError_t launch_step_persistent_t(const StepParams& p, const FillParam& fp, u
 template <int VAR, int DK, int DV, int ROWS, typename T, typename TB, bool FUSED>
 cudaError_t launch_step_rows(bool persistent, const StepParams& p, const FillParam& fp, unsigned n,
                              cudaStream_t s) {
-  if constexpr (std::is_same<TB, float>::value) {
+  if constexpr (std::is_same<TB, float>::value && VAR != kVarGDN2) {
     if (persistent) {
       const cudaError_t e = launch_step_persistent_t<VAR, DK, DV, ROWS, T, FUSED>(p, fp, n, s);
       if (e != cudaErrorNotSupported) return e;

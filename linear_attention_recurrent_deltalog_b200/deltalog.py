@@ -25,7 +25,7 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdeltalog.so")
 
 # enums (mirror deltalog.h)
-DL_GDN, DL_KDA, DL_RWKV6 = 0, 1, 2
+DL_GDN, DL_KDA, DL_RWKV6, DL_GDN2 = 0, 1, 2, 3
 DL_F32, DL_BF16 = 0, 1
 DL_OK = 0
 DL_ERR_ARG, DL_ERR_ALIGN, DL_ERR_LOG_FULL = -1, -2, -3
@@ -36,7 +36,7 @@ DL_FLAG_PERSISTENT = 2
 DL_FLAG_KLA = 4
 DL_FLAG_BASE_Q8 = 8
 
-VARIANT_IDS = {"gdn": DL_GDN, "kda": DL_KDA, "rwkv6": DL_RWKV6}
+VARIANT_IDS = {"gdn": DL_GDN, "kda": DL_KDA, "rwkv6": DL_RWKV6, "gdn2": DL_GDN2}
 DTYPE_IDS = {"f32": DL_F32, "bf16": DL_BF16}
 _TORCH_IN = {DL_F32: torch.float32, DL_BF16: torch.bfloat16}
 
@@ -197,10 +197,13 @@ def _check_step_tensors(cfg: Config, q, k, v, decay, beta, bonus, o) -> None:
     _need(k, "k", BH * dk, tin)
     _need(v, "v", BH * dv, tin)
     _need(decay, "decay", BH * (1 if cfg.variant == "gdn" else dk), torch.float32)
-    if cfg.variant != "rwkv6":
-        _need(beta, "beta", BH, torch.float32)
-    else:
+    if cfg.variant == "rwkv6":
         _need(bonus, "bonus", cfg.H * dk, torch.float32)
+    elif cfg.variant == "gdn2":           # beta: erase gate; bonus: write gate
+        _need(beta, "beta", BH * dk, torch.float32)
+        _need(bonus, "bonus", BH * dv, torch.float32)
+    else:
+        _need(beta, "beta", BH, torch.float32)
     _need(o, "o", BH * dv, torch.float32)
 
 

@@ -49,6 +49,14 @@ def step_to_device(s: wl.StepInputs, dev):
     return q, k, v, dec, beta
 
 
+def step_bonus(s: wl.StepInputs, dev, fixed=None):
+    """The step's `bonus` argument: GDN-2's write gate for this step, else the
+    fixed RWKV6 bonus (or None)."""
+    if s.wgate is not None:
+        return host_to_device(s.wgate, dev).reshape(-1)
+    return fixed
+
+
 @dataclasses.dataclass
 class ArmResult:
     state_err: float
@@ -114,13 +122,14 @@ def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence
     S_out = torch.empty(BH * dv * dk, dtype=torch.float32, device=device)
     for s in wl.StepStream(w, T, workers=workers):
         q, k, v, dec, beta = step_to_device(s, device)
+        bon_s = step_bonus(s, device, bonus_d)
         n = s.t + 1
         for arm in arms:
             if arm == "eager":
-                dlb.dl_eager_step(cfg_e, dense[arm], q, k, v, dec, beta, bonus_d, o)
+                dlb.dl_eager_step(cfg_e, dense[arm], q, k, v, dec, beta, bon_s, o)
             else:
                 st = states[arm]
-                st.step(q, k, v, dec, beta, bonus_d, o)
+                st.step(q, k, v, dec, beta, bon_s, o)
                 if arm == "log":
                     st.merge(dlb.DL_MERGE_FULL)
                 if n in merge_all_at:
@@ -136,7 +145,8 @@ def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence
                                     .astype(np.float64))
         flat = lambda x: None if x is None else x.reshape((BH,) + x.shape[2:])[heads][:, None]
         recs.append(types.SimpleNamespace(q=flat(s.q), k=flat(s.k), v=flat(s.v),
-                                          decay=flat(s.decay), beta=flat(s.beta)))
+                                          decay=flat(s.decay), beta=flat(s.beta),
+                                          wgate=flat(s.wgate)))
     torch.cuda.synchronize()
     for arm, st in states.items():
         code, head = st.device_error()
@@ -237,7 +247,7 @@ def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Seque
     for s in wl.StepStream(w, T, workers=workers):
         q, k, v, dec, beta = step_to_device(s, device)
         n = s.t + 1
-        st.step(q, k, v, dec, beta, bonus_d, o)
+        st.step(q, k, v, dec, beta, step_bonus(s, device, bonus_d), o)
         if not fused:
             st.merge(dlb.DL_MERGE_FULL)
         if n in forced:
@@ -245,7 +255,7 @@ def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Seque
         o_gpu = o.view(BH, dv).index_select(0, heads_t).cpu().numpy().astype(np.float64)
         flat = lambda x: None if x is None else x.reshape((BH,) + x.shape[2:])[heads][:, None]
         step = types.SimpleNamespace(q=flat(s.q), k=flat(s.k), v=flat(s.v), decay=flat(s.decay),
-                                     beta=flat(s.beta))
+                                     beta=flat(s.beta), wgate=flat(s.wgate))
         res = oracle.run_eager(w.variant, S, [step], bonus=bon, kla_eps=w.kla_eps)
         S = res.S
         out_err = max(out_err, _rel(o_gpu, res.outputs[0]))

@@ -60,6 +60,8 @@ def test_state_bytes_layout():
     assert nl_kda == pad(BH * 16 * 128 * 4) + pad(BH * 16 * 128 * 2) + pad(BH * 16 * 128 * 4)
     _, nl_rw, _ = dlb.dl_state_bytes(cfg(variant="rwkv6", d_k=64, d_v=64, L=32))
     assert nl_rw == pad(BH * 32 * 64 * 2) + pad(BH * 32 * 64 * 2) + pad(BH * 32 * 64 * 4)
+    # GDN-2 keeps KDA's log
+    assert dlb.dl_state_bytes(cfg(variant="gdn2")) == dlb.dl_state_bytes(cfg(variant="kda"))
     # int8 base: codes, then the fp32 row scales at the next 256-B boundary;
     # the log and meta buffers do not change
     nbq, nlq, nmq = dlb.dl_state_bytes(cfg(base="q8"))
@@ -108,6 +110,17 @@ def test_bad_enums_rejected():
     c = cfg(variant="rwkv6", d_k=64, d_v=64, kla_eps=1e-6).c()
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
     c = cfg(kla_eps=-1.0).c()
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+    # GDN-2: built for both bases; no KLA step size, no persistent kernel
+    for base in ("f32", "q8"):
+        c = cfg(variant="gdn2", base=base).c()
+        assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_OK
+    c = cfg(variant="gdn2", kla_eps=1e-6).c()
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
+    c = cfg(variant="gdn2", persistent=True).c()
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_UNSUPPORTED
+    c = cfg().c()
+    c.variant = 4
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
 
 
@@ -181,6 +194,16 @@ def test_binding_rejects_undersized_tensors():
     with pytest.raises(TypeError):
         dlb._check_step_tensors(c, torch.zeros(512), torch.zeros(512), torch.zeros(512),
                                 torch.zeros(4), torch.zeros(4), None, torch.zeros(512))
+    # GDN-2: beta carries the erase gate [B,H,d_k], bonus the write gate [B,H,d_v]
+    g = cfg(variant="gdn2", B=2, H=2, in_dtype="f32")
+    ok = dict(q=torch.zeros(512), k=torch.zeros(512), v=torch.zeros(512), decay=torch.zeros(512),
+              beta=torch.zeros(512), bonus=torch.zeros(512), o=torch.zeros(512))
+    dlb._check_step_tensors(g, **ok)
+    for name in ("beta", "bonus", "decay"):
+        bad = dict(ok)
+        bad[name] = torch.zeros(4)
+        with pytest.raises(ValueError):
+            dlb._check_step_tensors(g, **bad)
 
 
 def test_load_seqs_checks_indices_on_the_host():

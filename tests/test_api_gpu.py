@@ -88,13 +88,13 @@ def test_python_binding_refuses_small_buffers_before_launch():
 
 
 @pytest.mark.parametrize("fused", [True, False])
-@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
+@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6", "gdn2"])
 def test_slot_admission_matches_oracle(name, fused):
     # Sequences 1 and 4 get new dense states mid-stream (different fill
     # phases), sequence 2 a zero state later; the others run on untouched.
     import types
     import oracle
-    from tests.parity import OUT_TOL, STATE_TOL, host_to_device
+    from tests.parity import OUT_TOL, STATE_TOL, host_to_device, step_bonus
     w = wl.WORKLOADS[name].replace(B=6, H=3, L=5, T=20, ragged=True)
     BH, dk, dv = w.heads, w.d_k, w.d_v
     cfg = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype, fused_merge=fused)
@@ -126,13 +126,14 @@ def test_slot_admission_matches_oracle(name, fused):
         q, k, v = (host_to_device(s.device_array(n), "cuda").reshape(-1) for n in ("q", "k", "v"))
         dec = host_to_device(s.decay, "cuda").reshape(-1)
         beta = None if s.beta is None else host_to_device(s.beta, "cuda").reshape(-1)
-        st.step(q, k, v, dec, beta, bonus_d, o)
+        st.step(q, k, v, dec, beta, step_bonus(s, "cuda", bonus_d), o)
         if not fused:
             st.merge(dlb.DL_MERGE_FULL)
         flat = lambda x: None if x is None else x.reshape((BH,) + x.shape[2:])
         step = types.SimpleNamespace(q=flat(s.q)[:, None], k=flat(s.k)[:, None], v=flat(s.v)[:, None],
                                      decay=flat(s.decay)[:, None],
-                                     beta=None if s.beta is None else flat(s.beta)[:, None])
+                                     beta=None if s.beta is None else flat(s.beta)[:, None],
+                                     wgate=None if s.wgate is None else flat(s.wgate)[:, None])
         res = oracle.run_eager(w.variant, S_or, [step],
                                bonus=None if bonus is None else bonus[np.arange(BH) % w.H])
         S_or = res.S

@@ -131,3 +131,31 @@ def test_kla_step_size(name, persistent):
     _check(run_parity(w, snap_every=9, workers=0, persistent=persistent))
     w = wl.WORKLOADS[name].replace(kla_eps=1e-3)
     _check(run_parity(w, T=40, heads=wl.sample_heads(w, 24), arms=("fused", "eager")))
+
+
+# ---------------------------------------------------------------- GDN-2
+
+def test_gdn2_full_workload():
+    # B=128 H=32 d=128 L=16: erase and write gates per channel, every step
+    w = wl.WORKLOADS["gdn2"]
+    _check(run_parity(w, heads=wl.sample_heads(w, 48)))
+
+
+@pytest.mark.parametrize("split", [1, 2, 4])
+@pytest.mark.parametrize("dk,dv,dtype", [(128, 128, "bf16"), (64, 128, "f32"), (128, 64, "bf16"),
+                                         (64, 64, "f32")])
+def test_gdn2_shapes_splits(dk, dv, dtype, split):
+    if dv // split < 32:
+        pytest.skip("d_v / split < 32 is not built")
+    w = wl.WORKLOADS["gdn2"].replace(B=5, H=3, d_k=dk, d_v=dv, in_dtype=dtype, L=6, T=29,
+                                     ragged=True)
+    _check(run_parity(w, snap_every=7, workers=0, split=split))
+
+
+def test_gdn2_log_lengths_and_forced_merges():
+    for L in (1, 2, 64):
+        w = wl.WORKLOADS["gdn2"].replace(B=3, H=4, L=L, T=max(3 * L, 12) + 1, ragged=True)
+        _check(run_parity(w, snap_every=max(L, 4), workers=0))
+    w = wl.WORKLOADS["gdn2"].replace(B=4, H=3, L=16, T=40, ragged=True)
+    _check(run_parity(w, snap_every=5, merge_all_at=(3, 7, 20, 21), workers=0,
+                      arms=("log", "fused")))

@@ -52,7 +52,7 @@ def test_q8_tiny_all_heads(fused):
 
 
 @pytest.mark.parametrize("fused", [True, False])
-@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
+@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6", "gdn2"])
 def test_q8_workloads(name, fused):
     w = wl.WORKLOADS[name].replace(ragged=True)
     heads = heads_covering_phases(w, 24)
@@ -73,11 +73,12 @@ def test_q8_serving_full_batch():
 @pytest.mark.parametrize("variant,dk,dv,dtype", [
     ("gdn", 64, 128, "bf16"), ("kda", 128, 64, "f32"), ("rwkv6", 64, 64, "f32"),
     ("gdn", 128, 128, "f32"), ("kda", 64, 64, "bf16"), ("rwkv6", 128, 128, "bf16"),
+    ("gdn2", 64, 128, "bf16"), ("gdn2", 128, 128, "f32"),
 ])
 def test_q8_shapes_dtypes_splits(variant, dk, dv, dtype, split):
     if dv // split < 32:
         pytest.skip("work items hold at least 32 rows")
-    base = {"gdn": "gdn_qwen", "kda": "kda", "rwkv6": "rwkv6"}[variant]
+    base = {"gdn": "gdn_qwen", "kda": "kda", "rwkv6": "rwkv6", "gdn2": "gdn2"}[variant]
     w = wl.WORKLOADS[base].replace(B=6, H=3, d_k=dk, d_v=dv, in_dtype=dtype, L=5, ragged=True,
                                    seed=31 + split)
     for fused in (True, False):
