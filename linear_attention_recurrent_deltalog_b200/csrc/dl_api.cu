@@ -249,7 +249,7 @@ dl_quantize_kernel(int8_t* codes, float* scales, int* fill, const float* S, cons
     if (m >= dl::kTinyAmax) {
       const float inv = __fdiv_rn(127.0f, m);
       for (int e = 0; e < per; ++e)
-        w |= (uint32_t(__float2int_rn(__fmul_rn(x[e], inv))) & 0xffu) << (8 * e);
+        w |= (dl::round_code_bits(x[e], inv) & 0xffu) << (8 * e);
       sc = __fdiv_rn(m, 127.0f);
     }
     // the lane's `per` codes stay contiguous inside one 16-byte chunk of the

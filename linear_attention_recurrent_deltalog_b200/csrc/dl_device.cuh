@@ -260,73 +260,23 @@ struct Tile {
 // ------------------------------------------------------ int8 base rows
 //
 // A quantized base row holds d_k int8 codes and one fp32 scale per value
-// row (the scale multiplies a finished row dot product).  A warp covers 16
-// rows with 16 consecutive codes (one 16-byte shared-memory load) per lane:
-// QL lanes per row, 32/QL rows per warp instruction, QNV rows per lane.
-
-template <int DK>
-struct QRows {
-  static constexpr int kCodes = 16;          // codes per lane per row
-  static constexpr int kLPR = DK / kCodes;   // lanes per row
-  static constexpr int kRPI = 32 / kLPR;     // rows per warp instruction
-  static constexpr int kNV = 16 / kRPI;      // rows per lane
-  static_assert(kLPR == 2 * kNV, "row reduction layout");
-};
-
-// Four int8 codes packed in a word -> exact fp32 values.  IEEE-754 single
-// precision has 23 fraction bits, so 2^23 + n for n in [0, 255] is exact and
-// its low fraction byte is n.  Flipping each code's sign bit gives n = code +
-// 128; a byte permute builds the word (0x4B, 0, 0, n) = 2^23 + n and one
-// subtraction of 2^23 + 128 leaves the code, with no integer-to-float
-// conversion instruction.
-__device__ __forceinline__ void codes4_to_f(uint32_t w, float* f) {
-  const uint32_t u = w ^ 0x80808080u;
-  constexpr float kBias = 8388736.0f;  // 2^23 + 128
-  f[0] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)) - kBias;
-  f[1] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541)) - kBias;
-  f[2] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)) - kBias;
-  f[3] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543)) - kBias;
-}
-
-// Sixteen codes (16-byte aligned) -> fp32.
-__device__ __forceinline__ void codes16_to_f(const int8_t* p, float (&f)[16]) {
-  const uint4 w = *reinterpret_cast<const uint4*>(p);
-  codes4_to_f(w.x, f);
-  codes4_to_f(w.y, f + 4);
-  codes4_to_f(w.z, f + 8);
-  codes4_to_f(w.w, f + 12);
-}
+// row: code = round-half-even(x * inv), inv = 127 / amax, scale = amax / 127.
 
 // Rows whose absolute maximum is below this are stored as zero (127/amax
 // would overflow fp32 near the bottom of its range).
 constexpr float kTinyAmax = 7.52316384526264e-37f;  // 2^-120
 
-// Quantizes this lane's 16 values of a row whose absolute maximum is amax
-// (the same in every lane of the row): code = round-half-even(x * inv),
-// inv = 127 / amax, each one correctly rounded fp32 operation.  Returns the
-// codes packed for one 16-byte store; *scale = amax / 127.
-__device__ __forceinline__ uint4 quantize16(const float (&x)[16], float amax, float* scale) {
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
-  if (amax >= kTinyAmax) {
-    const float inv = __fdiv_rn(127.0f, amax);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c = __float2int_rn(__fmul_rn(x[i], inv));
-      w[i >> 2] |= (uint32_t(c) & 0xffu) << (8 * (i & 3));
-    }
-    *scale = __fdiv_rn(amax, 127.0f);
-  } else {
-    *scale = 0.f;
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+// round-half-even(fl32(x * inv)) as the low byte of a float: the product is
+// rounded once (__fmul_rn, never fused), and adding 1.5 * 2^23 in
+// round-to-nearest-even leaves, for |x * inv| < 2^22, exactly that integer
+// in the low mantissa bits (its low byte is the int8 code, two's complement).
+__device__ __forceinline__ uint32_t round_code_bits(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));
 }
 
-// Maximum over the kLPR lanes of a row (lanes differing in their low bits).
-template <int LPR>
-__device__ __forceinline__ float row_max(float x) {
-#pragma unroll
-  for (int o = 1; o < LPR; o <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
+// Four rounded values (from round_code_bits) -> one word of int8 codes.
+__device__ __forceinline__ uint32_t pack_codes4(uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  return __byte_perm(__byte_perm(r0, r1, 0x0040), __byte_perm(r2, r3, 0x0040), 0x5410);
 }
 
 // ------------------------------------------- int8 codes on the tensor cores
@@ -373,13 +323,6 @@ __device__ __forceinline__ void codes4_to_h2(uint32_t w, uint32_t& h01, uint32_t
   const __half2 bias = bits_h2(0x64806480u);  // (1152, 1152)
   h01 = h2_bits(__hsub2(bits_h2(__byte_perm(u, 0x64646464u, 0x4140)), bias));
   h23 = h2_bits(__hsub2(bits_h2(__byte_perm(u, 0x64646464u, 0x4342)), bias));
-}
-
-// Two int8 codes (low half of a word) -> fp32, exactly.
-__device__ __forceinline__ float2 codes2_to_f(uint32_t w) {
-  uint32_t h01, h23;
-  codes4_to_h2(w, h01, h23);
-  return __half22float2(bits_h2(h01));
 }
 
 // D += A B for one m16n8k16 tile (fp16 inputs, fp32 accumulators).

@@ -571,15 +571,11 @@ __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sSca
     const float inv = (m >= kTinyAmax) ? __fdiv_rn(127.0f, m) : 0.f;
     uint32_t w[WORDS];
 #pragma unroll
-    for (int v = 0; v < WORDS; ++v) {
-      const float x[4] = {acc[2 * v][2 * half], acc[2 * v][2 * half + 1], acc[2 * v + 1][2 * half],
-                          acc[2 * v + 1][2 * half + 1]};
-      uint32_t word = 0u;
-#pragma unroll
-      for (int b = 0; b < 4; ++b)
-        word |= (uint32_t(__float2int_rn(__fmul_rn(x[b], inv))) & 0xffu) << (8 * b);
-      w[v] = word;
-    }
+    for (int v = 0; v < WORDS; ++v)
+      w[v] = pack_codes4(round_code_bits(acc[2 * v][2 * half], inv),
+                         round_code_bits(acc[2 * v][2 * half + 1], inv),
+                         round_code_bits(acc[2 * v + 1][2 * half], inv),
+                         round_code_bits(acc[2 * v + 1][2 * half + 1], inv));
 #pragma unroll
     for (int v = 0; v < WORDS / 4; ++v)
       *reinterpret_cast<uint4*>(gCodes + q8_off<DK>(r, cbase + 16 * v)) =
@@ -606,7 +602,8 @@ __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sSca
 // log-decay bookkeeping and the per-entry weights are computed together, a
 // second barrier publishes them, and each warp streams its rows.
 
-template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB = float>
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB = float,
+          bool FUSED = true>
 struct StepLayout {
   using TU = typename LogU<VAR, TIn>::type;
   static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
@@ -626,17 +623,18 @@ struct StepLayout {
     offW = offVec + align_up(size_t(4 * DK + 2 * GW) * 4, 128);
     offZ = offW + align_up(size_t(L) * 4, 16);
     offScal = offZ + align_up(size_t(L) * 4, 16);
-    // int8 base: the CTA's row scales, the GEMV's fp16 vectors [4][DK], the
-    // base decay [DK] and, for the fused merge, the staged key fragments
     // RWKV6: the bonus u [DK]; GDN-2: the erase gate b [DK] and this CTA's
     // rows of the write gate w [ROWS]
     offBonus = offScal + 64;
     offWg = offBonus + ((VAR == kVarRWKV6 || VAR == kVarGDN2) ? align_up(size_t(DK) * 4, 128) : 0);
+    // int8 base: the CTA's row scales, the GEMV's fp16 vectors [4][DK] and,
+    // for the fused merge only, the base decay [DK] and the staged key
+    // fragments
     offScale = offWg + (VAR == kVarGDN2 ? align_up(size_t(ROWS) * 4, 128) : 0);
     offVecH = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
     offDecF = offVecH + (Q8 ? align_up(size_t(4) * kVecHStride<DK> * 2, 128) : 0);
-    offKt = offDecF + (Q8 ? align_up(size_t(DK) * 4, 128) : 0);
-    offBar = offKt + (Q8 ? size_t(q8_chunks(L)) * DK * 64 : 0);
+    offKt = offDecF + ((Q8 && FUSED) ? align_up(size_t(DK) * 4, 128) : 0);
+    offBar = offKt + ((Q8 && FUSED) ? size_t(q8_chunks(L)) * DK * 64 : 0);
     total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
   }
 };
@@ -658,7 +656,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   using TU = typename LogU<VAR, TIn>::type;
   constexpr bool Q8 = std::is_same<TB, int8_t>::value;
   constexpr int SPLIT = DV / ROWS;
-  constexpr int GW = StepLayout<VAR, DK, DV, ROWS, TIn, TB>::GW;
+  constexpr int GW = StepLayout<VAR, DK, DV, ROWS, TIn, TB, FUSED>::GW;
   constexpr int NT = Tl::kThreads;
   constexpr int NW = Tl::kWarps;
   constexpr int CPL = Tl::kCPL;
@@ -668,7 +666,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int L = p.L;
   const int GS = g_stride(VAR, L, DK);
-  const StepLayout<VAR, DK, DV, ROWS, TIn, TB> lay(L);
+  const StepLayout<VAR, DK, DV, ROWS, TIn, TB, FUSED> lay(L);
   TB* sS = reinterpret_cast<TB*>(smem);                       // [ROWS][DK]
   TU* sU = reinterpret_cast<TU*>(smem + lay.offU);            // [ROWS/32][L][32]
   TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);          // [L][DK]

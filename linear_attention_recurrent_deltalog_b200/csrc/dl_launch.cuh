@@ -54,7 +54,7 @@ cudaError_t launch_step_t(const StepParams& p, const FillParam& fp, unsigned nhe
   auto kern = dl_step_kernel<VAR, DK, DV, ROWS, TIn, TB, FUSED>;
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
-  const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn, TB>(p.L).total;
+  const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn, TB, FUSED>(p.L).total;
   kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p, fp);
   return cudaGetLastError();
 }
