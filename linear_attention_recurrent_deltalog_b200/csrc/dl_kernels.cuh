@@ -479,16 +479,24 @@ __device__ __forceinline__ void stage_kt_frags(const TIn* sK, const float* sG, c
   }
 }
 
+// Index of key channel c in the fold's padded decay array: 16 bytes of
+// padding after every 32 channels put the four lanes of a row group (which
+// read their 32 channels each as float4s) in different bank groups.
+__host__ __device__ constexpr int dec_pad(int c) { return c + ((c >> 5) << 2); }
+template <int DK>
+constexpr int kDecPadLen = DK + DK / 8;
+
 // Folds nent log entries into the warp's 16 rows of an int8 base on the
 // tensor cores, in one pass:
 //   x = deq(code) * dec + U Kt,   deq(code) = code * scale,
 // U = the rows' u values (A, split hi/lo in registers), Kt = the staged B
-// fragments.  Lane 4g + t holds rows j0+g and j0+g+8 over the key channels
+// fragments, sDec the base decay at dec_pad indices (SDEC: one scalar decay,
+// any entry).  Lane 4g + t holds rows j0+g and j0+g+8 over the key channels
 // [DK/4 t, DK/4 (t+1)) (fold_channel).  With gOut the rows are written to it
 // as fp32 (unswizzled); otherwise each row's absolute maximum is reduced
 // over its four lanes and the row is requantized straight from the
 // accumulators into gCodes (swizzled order) and gScale.
-template <int DK, typename TU>
+template <int DK, typename TU, bool SDEC>
 __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sScale, const TU* sU,
                                              const uint32_t* sB, const float* sDec, int nent,
                                              int nchunks, int L, int j0, int lane, int8_t* gCodes,
@@ -515,17 +523,25 @@ __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sSca
       w[4 * v + 2] = q.z;
       w[4 * v + 3] = q.w;
     }
+    const float sd = SDEC ? s * sDec[0] : 0.f;
 #pragma unroll
     for (int v = 0; v < WORDS; ++v) {
       uint32_t h01, h23;
       codes4_to_h2(w[v], h01, h23);
       const float2 c01 = __half22float2(bits_h2(h01));
       const float2 c23 = __half22float2(bits_h2(h23));
-      const float4 d4 = *reinterpret_cast<const float4*>(sDec + cbase + 4 * v);
-      acc[2 * v][2 * half] = (c01.x * s) * d4.x;
-      acc[2 * v][2 * half + 1] = (c01.y * s) * d4.y;
-      acc[2 * v + 1][2 * half] = (c23.x * s) * d4.z;
-      acc[2 * v + 1][2 * half + 1] = (c23.y * s) * d4.w;
+      if (SDEC) {
+        acc[2 * v][2 * half] = c01.x * sd;
+        acc[2 * v][2 * half + 1] = c01.y * sd;
+        acc[2 * v + 1][2 * half] = c23.x * sd;
+        acc[2 * v + 1][2 * half + 1] = c23.y * sd;
+      } else {
+        const float4 d4 = *reinterpret_cast<const float4*>(sDec + dec_pad(cbase + 4 * v));
+        acc[2 * v][2 * half] = (c01.x * s) * d4.x;
+        acc[2 * v][2 * half + 1] = (c01.y * s) * d4.y;
+        acc[2 * v + 1][2 * half] = (c23.x * s) * d4.z;
+        acc[2 * v + 1][2 * half + 1] = (c23.y * s) * d4.w;
+      }
     }
   }
   const uint4* sB4 = reinterpret_cast<const uint4*>(sB);
@@ -633,7 +649,7 @@ struct StepLayout {
     offScale = offWg + (VAR == kVarGDN2 ? align_up(size_t(ROWS) * 4, 128) : 0);
     offVecH = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
     offDecF = offVecH + (Q8 ? align_up(size_t(4) * kVecHStride<DK> * 2, 128) : 0);
-    offKt = offDecF + ((Q8 && FUSED) ? align_up(size_t(DK) * 4, 128) : 0);
+    offKt = offDecF + ((Q8 && FUSED) ? align_up(size_t(kDecPadLen<DK>) * 4, 128) : 0);
     offBar = offKt + ((Q8 && FUSED) ? size_t(q8_chunks(L)) * DK * 64 : 0);
     total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
   }
@@ -881,9 +897,9 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       __syncthreads();
     }
     stage_kt_frags<VAR, DK, TIn>(sK, sG, sGt, sW, f, f + 1, q8_chunks(f + 1), sB, tid, NT);
-    for (int c = tid; c < DK; c += NT) sDecF[c] = (GW == 1) ? sScal[2] : expf(sGt[c]);
+    for (int c = tid; c < DK; c += NT) sDecF[dec_pad(c)] = (GW == 1) ? sScal[2] : expf(sGt[c]);
     __syncthreads();
-    fold_rows_q8<DK, TU>(sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L, j0, lane,
+    fold_rows_q8<DK, TU, GW == 1>(sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L, j0, lane,
                          static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
                          p.scale + head * size_t(DV) + r0, nullptr);
   } else {
@@ -908,7 +924,8 @@ struct MergeLayout {
     // fp32 decayed keys [L][DK], or (int8 base) their staged fp16 fragments
     offG = offKt + align_up(Q8 ? size_t(q8_chunks(L)) * DK * 64 : size_t(L) * DK * 4, 128);
     offDec = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
-    offScale = offDec + align_up(size_t(DK + (Q8 ? 64 : 0)) * 4, 128);  // + GDN entry factors
+    // int8: the decay at dec_pad indices, then GDN's per-entry factors
+    offScale = offDec + align_up(size_t(Q8 ? kDecPadLen<DK> + 64 : DK) * 4, 128);
     offBar = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
     total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
   }
@@ -918,9 +935,14 @@ struct MergeLayout {
 // DV / ROWS CTAs, as in the step).  With a list, the fills come from the
 // list and only part 0 empties the log, so split CTAs never race on it;
 // without a list the kernel runs unsplit and reads the device fill.
+// The int8 merge folds every CTA: compiled for 640 threads per SM (about
+// 100 registers, no spills).
+template <typename TB, int THREADS>
+constexpr int kMergeMinBlocks = std::is_same<TB, int8_t>::value ? 640 / THREADS : 1;
+
 template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB>
 __global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads,
-                                  kMinBlocks<TB, Tile<DK, ROWS, TB>::kThreads, true>)
+                                  kMergeMinBlocks<TB, Tile<DK, ROWS, TB>::kThreads>)
 dl_merge_kernel(const MergeParams p, const SeqList list) {
   using Tl = Tile<DK, ROWS, TB>;
   using TU = typename LogU<VAR, TIn>::type;
@@ -1006,10 +1028,10 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
   // decay of the base and decayed keys k-tilde_i = k_i o e^{g_last - g_i},
   // one (entry, channel) pair per thread
   for (int c = tid; c < DK; c += NT)
-    sDec[c] = expf((f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f);
+    sDec[Q8 ? dec_pad(c) : c] = expf((f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f);
   if constexpr (Q8) {
     if (f > 0) {
-      float* sFac = sDec + DK;  // GDN: e^{g_last - g_i} per entry
+      float* sFac = sDec + kDecPadLen<DK>;  // GDN: e^{g_last - g_i} per entry
       if (GW == 1) {
         for (int e = tid; e < f; e += NT) sFac[e] = expf(sG[f - 1] - sG[e]);
         __syncthreads();
@@ -1040,7 +1062,7 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
   }
   if constexpr (Q8) {
     const bool to_fp32 = (p.mode == 2);
-    fold_rows_q8<DK, TU>(sS, sScale, sU, reinterpret_cast<const uint32_t*>(sKt), sDec, f,
+    fold_rows_q8<DK, TU, GW == 1>(sS, sScale, sU, reinterpret_cast<const uint32_t*>(sKt), sDec, f,
                          q8_chunks(f), L, j0, lane,
                          static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
                          p.scale + head * size_t(DV) + r0,
