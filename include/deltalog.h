@@ -112,7 +112,8 @@ enum dl_flags {
 /* Layer configuration.  d_k, d_v in {64, 128}; 1 <= L <= 64; B, H >= 1 and
  * B*H*d_v*d_k < 2^40.  `flags` is a bitwise OR of dl_flags.  `step_split`
  * is into how many work items (of d_v / step_split rows) the step kernel
- * cuts one head: 0 picks the library's default, otherwise 1, 2 or 4 with
+ * cuts one head: 0 picks the library's default (2 for GDN at d_v = 128,
+ * else 1), otherwise 1, 2 or 4 with
  * d_v / step_split >= 32 (a performance knob only: results do not depend
  * on it). */
 typedef struct dl_config {

@@ -37,8 +37,13 @@ struct Layout {
 
 bool is_q8(const dl_config& c) { return (c.flags & DL_FLAG_BASE_Q8) != 0; }
 
-// Default work items per head for the step kernel: 64-row items.
-int default_split(const dl_config& c) { return c.d_v >= 128 ? 2 : 1; }
+// Default work items per head for the step kernel (measured on B200): GDN
+// cuts a d_v = 128 head into two 64-row items; the vector-decay variants
+// (KDA, GDN-2, RWKV6), whose per-head log-decay block and entry weights every
+// item would stage again, keep one item per head (fp32 and int8 base alike).
+int default_split(const dl_config& c) {
+  return (c.variant == DL_GDN && c.d_v >= 128) ? 2 : 1;
+}
 int split_of(const dl_config& c) { return c.step_split == 0 ? default_split(c) : c.step_split; }
 
 int u_elem_size(const dl_config& c) {
