@@ -187,3 +187,15 @@ def test_q8_free_run_error_matches_oracle():
     d_go = np.max(np.abs(np.stack(outs) - np.stack(windowed.outputs)))
     assert d_go <= 8 * np.max(np.abs(np.stack(windowed.outputs) - np.stack(exact.outputs))) + 1e-6
     st.close()
+
+
+@pytest.mark.parametrize("L", [4, 32, 64])
+def test_q8_serving_L_sweep(L):
+    # B=512 with ragged fills: every sequence ends at least two windows at its
+    # own phase, separate and fused merge
+    w = wl.WORKLOADS["gdn_serving"].replace(L=L)
+    heads = heads_covering_phases(w, 16)
+    for fused in (True, False):
+        r = run_parity_q8(w, T=2 * L + 5, heads=heads, fused=fused, snap_every=max(L // 2, 4),
+                          workers=None)
+        _check(r)
