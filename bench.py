@@ -403,10 +403,8 @@ def run_ours(args, world, rank, local):
     step_bytes_avg = (rd + wr) / args.steps
     achieved = step_bytes_avg / step_avg / 1e9
     traffic = None
-    for tname in ("step_kernel_traffic.json", "step_kernel_traffic_q8.json"):
-        tfile = os.path.join(ROOT, "profiles", tname)
-        if not os.path.exists(tfile):
-            continue
+    import glob
+    for tfile in sorted(glob.glob(os.path.join(ROOT, "profiles", "step_kernel_traffic*.json"))):
         try:
             t = json.load(open(tfile))
         except Exception:
@@ -737,7 +735,9 @@ def main():
                     help="CTAs per head in the step kernel (0 = library default)")
     ap.add_argument("--only-step", action="store_true",
                     help="time the DeltaLog step only (profiling); not a bench line")
-    ap.add_argument("--merge", choices=("fused", "separate"), default="fused")
+    ap.add_argument("--merge", choices=("fused", "separate"), default=None,
+                    help="merge mode (default: fused for the fp32 base, separate for the int8 "
+                         "base, the faster mode of each)")
     ap.add_argument("--base", choices=("f32", "q8"), default="f32",
                     help="base storage: fp32, or int8 codes + row scales requantized per window")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
@@ -751,6 +751,8 @@ def main():
     ap.add_argument("--admit-every", type=int, default=8,
                     help="--serving: admit B/64 new sequences every this many steps (0: never)")
     args = ap.parse_args()
+    if args.merge is None:
+        args.merge = "separate" if args.base == "q8" else "fused"
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
