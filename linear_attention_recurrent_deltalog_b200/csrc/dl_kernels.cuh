@@ -159,6 +159,7 @@ __device__ __forceinline__ void entry_weights(int f, int warp, int nwarps, int l
                                               const float* dec, float* sW, float* sZ,
                                               const float* kgate = nullptr) {
   constexpr int CPE = DK / 8;  // channels per lane
+  if (warp * 4 >= f) return;   // no entry for this warp
   const int slot = lane >> 3;
   const int c0 = (lane & 7) * CPE;
   float kl[CPE], ql[CPE], gl[CPE];
