@@ -83,6 +83,35 @@ __device__ __forceinline__ void load_f(const __nv_bfloat16* p, float (&out)[N]) 
   }
 }
 
+// N in {2, 4, 8, 16} consecutive elements as fp32 (p aligned to the size
+// of the load: N elements).
+template <int N>
+__device__ __forceinline__ void load_small(const float* p, float (&out)[N]) {
+  if constexpr (N == 2) {
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    out[0] = v.x;
+    out[1] = v.y;
+  } else {
+    load_f<N>(p, out);
+  }
+}
+template <int N>
+__device__ __forceinline__ void load_small(const __nv_bfloat16* p, float (&out)[N]) {
+  if constexpr (N == 2) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    out[0] = __uint_as_float(w << 16);
+    out[1] = __uint_as_float(w & 0xffff0000u);
+  } else if constexpr (N == 4) {
+    const float4 v = load4(p);
+    out[0] = v.x;
+    out[1] = v.y;
+    out[2] = v.z;
+    out[3] = v.w;
+  } else {
+    load_f<N>(p, out);
+  }
+}
+
 __device__ __forceinline__ float dot4(float4 a, float4 b) {
   return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }

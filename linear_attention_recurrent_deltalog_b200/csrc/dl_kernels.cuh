@@ -144,30 +144,33 @@ __device__ __forceinline__ uint32_t g_copy_bytes(int f) {
 }
 
 // Per-entry weights of the log correction for the f entries of one head,
-// computed entry-parallel: eight lanes share an entry (d_k/8 key channels
-// each), so a warp covers four entries per pass and each sum needs a 3-level
-// shuffle reduction rather than a full 5-level one per entry.
+// computed entry-parallel: LPE lanes share an entry (d_k / LPE key channels
+// each) and a warp covers 32 / LPE entries per pass; each sum is a
+// log2(LPE)-level shuffle reduction inside the lane group.
 //   GDN  : W_i = e^{g_t - g_i} (k_i . k_t),  Z_i = e^{g_t - g_i} (k_i . q_t)
 //   KDA  : W_i = sum_c k_i[c] k_t[c] e^{g_t[c] - g_i[c]},  Z_i the same with q_t
+//   GDN-2: as KDA, with k_t replaced by the gated key kgate o k_t in W_i
 //   RWKV6: Z_i = sum_c k_i[c] r_t[c] e^{g_{t-1}[c] - g_i[c]}
 // kin, qin: k_t and q_t (r_t) in shared memory (fp32 or the input type);
 // sK: the staged log keys [f][DK]; sG: the staged log-decay; dec: the
 // step's decay (one scalar for GDN, d_k values otherwise).  Requires f > 0.
-template <int VAR, int DK, typename TK, typename TIn>
-__device__ __forceinline__ void entry_weights(int f, int warp, int nwarps, int lane, const TK* kin,
-                                              const TK* qin, const TIn* sK, const float* sG,
-                                              const float* dec, float* sW, float* sZ,
-                                              const float* kgate = nullptr) {
-  constexpr int CPE = DK / 8;  // channels per lane
-  if (warp * 4 >= f) return;   // no entry for this warp
-  const int slot = lane >> 3;
-  const int c0 = (lane & 7) * CPE;
+// Warps with no entry return at once.
+template <int VAR, int DK, typename TK, typename TIn, int LPE>
+__device__ __forceinline__ void entry_weights_lpe(int f, int warp, int nwarps, int lane,
+                                                  const TK* kin, const TK* qin, const TIn* sK,
+                                                  const float* sG, const float* dec, float* sW,
+                                                  float* sZ, const float* kgate) {
+  constexpr int CPE = DK / LPE;  // channels per lane
+  constexpr int EPW = 32 / LPE;  // entries per warp per pass
+  if (warp * EPW >= f) return;
+  const int slot = lane / LPE;
+  const int c0 = (lane % LPE) * CPE;
   float kl[CPE], ql[CPE], gl[CPE];
-  load_f<CPE>(kin + c0, kl);
-  load_f<CPE>(qin + c0, ql);
+  load_small<CPE>(kin + c0, kl);
+  load_small<CPE>(qin + c0, ql);
   if (VAR == kVarGDN2) {  // GDN-2 reads through the gated key b o k
     float bg[CPE];
-    load_f<CPE>(kgate + c0, bg);
+    load_small<CPE>(kgate + c0, bg);
 #pragma unroll
     for (int c = 0; c < CPE; ++c) kl[c] *= bg[c];
   }
@@ -175,23 +178,23 @@ __device__ __forceinline__ void entry_weights(int f, int warp, int nwarps, int l
   if (VAR == kVarGDN) {
     gt0 = sG[f - 1] + logf(dec[0]);
   } else {
-    load_f<CPE>(sG + size_t(f - 1) * DK + c0, gl);
+    load_small<CPE>(sG + size_t(f - 1) * DK + c0, gl);
     if (VAR == kVarKDA || VAR == kVarGDN2) {
       float dl[CPE];
-      load_f<CPE>(dec + c0, dl);
+      load_small<CPE>(dec + c0, dl);
 #pragma unroll
       for (int c = 0; c < CPE; ++c) gl[c] += logf(dl[c]);
     }
   }
-  for (int base = warp * 4; base < f; base += nwarps * 4) {
+  for (int base = warp * EPW; base < f; base += nwarps * EPW) {
     const int i = base + slot;
     float x = 0.f, y = 0.f;
     if (i < f) {
       float ki[CPE];
-      load_f<CPE>(sK + size_t(i) * DK + c0, ki);
+      load_small<CPE>(sK + size_t(i) * DK + c0, ki);
       if (VAR != kVarGDN) {
         float gi[CPE];
-        load_f<CPE>(sG + size_t(i) * DK + c0, gi);
+        load_small<CPE>(sG + size_t(i) * DK + c0, gi);
 #pragma unroll
         for (int c = 0; c < CPE; ++c) ki[c] *= expf(gl[c] - gi[c]);
       }
@@ -202,17 +205,41 @@ __device__ __forceinline__ void entry_weights(int f, int warp, int nwarps, int l
       }
     }
 #pragma unroll
-    for (int o = 4; o > 0; o >>= 1) {
+    for (int o = LPE / 2; o > 0; o >>= 1) {
       if (VAR != kVarRWKV6) x += __shfl_xor_sync(0xffffffffu, x, o);
       y += __shfl_xor_sync(0xffffffffu, y, o);
     }
-    if (i < f && (lane & 7) == 0) {
+    if (i < f && (lane % LPE) == 0) {
       float e = 1.f;
       if (VAR == kVarGDN) e = expf(gt0 - sG[i]);
       sW[i] = x * e;
       sZ[i] = y * e;
     }
   }
+}
+
+// Picks the lanes per entry so that the f entries spread over every warp:
+// 32 when there are at most as many entries as warps, 16 up to two per
+// warp, 8 otherwise.  That shortens the phase for the latency-bound kernels;
+// an issue-bound caller (SPREAD = false) keeps 8 lanes per entry, which
+// issues the fewest instructions.
+template <int VAR, int DK, typename TK, typename TIn, bool SPREAD = true>
+__device__ __forceinline__ void entry_weights(int f, int warp, int nwarps, int lane, const TK* kin,
+                                              const TK* qin, const TIn* sK, const float* sG,
+                                              const float* dec, float* sW, float* sZ,
+                                              const float* kgate = nullptr) {
+  if (!SPREAD)
+    entry_weights_lpe<VAR, DK, TK, TIn, 8>(f, warp, nwarps, lane, kin, qin, sK, sG, dec, sW, sZ,
+                                           kgate);
+  else if (f <= nwarps)
+    entry_weights_lpe<VAR, DK, TK, TIn, 32>(f, warp, nwarps, lane, kin, qin, sK, sG, dec, sW, sZ,
+                                            kgate);
+  else if (f <= 2 * nwarps)
+    entry_weights_lpe<VAR, DK, TK, TIn, 16>(f, warp, nwarps, lane, kin, qin, sK, sG, dec, sW, sZ,
+                                            kgate);
+  else
+    entry_weights_lpe<VAR, DK, TK, TIn, 8>(f, warp, nwarps, lane, kin, qin, sK, sG, dec, sW, sZ,
+                                           kgate);
 }
 
 // The 16 staged u values of rows j0 .. j0+15 (one 32-row block) of entry i.
@@ -830,8 +857,10 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     if (appender) gG[f] = gt;
   }
   if (f > 0)
-    entry_weights<VAR, DK, TIn, TIn>(f, warp, NW, lane, sKr, sQr, sK, sG,
-                                     (GW == 1) ? &dec_s : sDecV, sW, sZ, sBonus);
+    // the int8 GDN step is issue-bound: fewest instructions (8 lanes per entry)
+    entry_weights<VAR, DK, TIn, TIn, !(Q8 && VAR == kVarGDN)>(f, warp, NW, lane, sKr, sQr, sK, sG,
+                                                              (GW == 1) ? &dec_s : sDecV, sW, sZ,
+                                                              sBonus);
   if (warp == NW - 1) {
     // GDN/KDA: k_t . q_t (the current entry's own weight on q) and, for the
     // KLA step size, |k_t|^2; RWKV6: the bonus sum_c r_c u_c k_c.
