@@ -87,8 +87,10 @@ def _rel(a: np.ndarray, ref: np.ndarray) -> float:
 def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence[int]] = None,
                arms=("log", "fused", "eager"), snap_every: int = 64, L: Optional[int] = None,
                merge_all_at: Sequence[int] = (), workers: Optional[int] = None,
-               split: int = 0, persistent: bool = False, device="cuda") -> Dict[str, ArmResult]:
-    """Runs the given arms and the oracle; returns per-arm errors."""
+               split: int = 0, persistent: bool = False, device="cuda",
+               edit=None) -> Dict[str, ArmResult]:
+    """Runs the given arms and the oracle; returns per-arm errors.  ``edit``
+    (optional) maps each drawn StepInputs to the one both sides receive."""
     if L is not None:
         w = w.replace(L=L)
     T = w.T if T is None else T
@@ -121,6 +123,8 @@ def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence
     o = torch.empty(BH * dv, dtype=torch.float32, device=device)
     S_out = torch.empty(BH * dv * dk, dtype=torch.float32, device=device)
     for s in wl.StepStream(w, T, workers=workers):
+        if edit is not None:
+            s = edit(s)
         q, k, v, dec, beta = step_to_device(s, device)
         bon_s = step_bonus(s, device, bonus_d)
         n = s.t + 1
@@ -206,7 +210,7 @@ def _lib_rows(S, rec):
 def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence[int]] = None,
                   fused: bool = True, split: int = 0, merge_all_at: Sequence[int] = (),
                   resync: bool = True, snap_every: int = 8, workers: Optional[int] = 0,
-                  device="cuda") -> Q8Result:
+                  device="cuda", edit=None) -> Q8Result:
     """The int8-base path against the windowed oracle (oracle.run_windowed's
     definition, stepped here one step at a time for the sampled heads).
 
@@ -216,7 +220,8 @@ def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Seque
     and amax may differ from the oracle's by the state tolerance).  With
     ``resync`` the oracle's codes and scales are then written into the GPU
     base for those heads, so every window starts from identical values and
-    outputs and states are held to the fp32 tolerances."""
+    outputs and states are held to the fp32 tolerances.  ``edit`` as in
+    run_parity."""
     T = w.T if T is None else T
     BH, dk, dv, H, L = w.heads, w.d_k, w.d_v, w.H, w.L
     rec = w.variant == wl.RWKV6
@@ -245,6 +250,8 @@ def run_parity_q8(w: wl.Workload, T: Optional[int] = None, heads: Optional[Seque
     mismatches = total = windows = 0
     forced = set(int(x) for x in merge_all_at)
     for s in wl.StepStream(w, T, workers=workers):
+        if edit is not None:
+            s = edit(s)
         q, k, v, dec, beta = step_to_device(s, device)
         n = s.t + 1
         st.step(q, k, v, dec, beta, step_bonus(s, device, bonus_d), o)
