@@ -90,7 +90,9 @@ enum dl_flags {
    * step carries the gate eta_t and the kernels use
    * beta_t = eta_t / (|k_t|_2^2 + kla_eps) ("Kaczmarz Linear Attention"
    * abstract), so the write projects exactly whatever the key's norm.
-   * Not for RWKV6 or GDN-2 (DL_ERR_ARG). */
+   * With kla_eps = 0 a zero key gives an infinite beta_t, and the outputs
+   * are NaN exactly as the formula's are: use kla_eps > 0 where keys may
+   * vanish.  Not for RWKV6 or GDN-2 (DL_ERR_ARG). */
   DL_FLAG_KLA = 4,
   /* int8 base quantized once per window ("LeapQuant" abstract: the state
    * is quantized only at the end of a window of tokens, and outputs inside
