@@ -690,6 +690,31 @@ def oracle_tokens_per_s(w, target_s: float = 0.0, seqs: int = 2, steps: int = 0,
     return seqs * done / el, done, el, threads
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and logical core count (for the CPU baseline)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+def oracle_single_core(w, target_s: float):
+    """oracle_tokens_per_s with the numerical libraries held to one thread."""
+    try:
+        import threadpoolctl
+        with threadpoolctl.threadpool_limits(1):
+            v, steps, el, _ = oracle_tokens_per_s(w, target_s=target_s, warmup=1)
+    except Exception as e:  # a reported figure only: never fail the line for it
+        return {"unavailable": f"{type(e).__name__}: {e}"}
+    return {"value": round(v, 3), "cores": 1, "sample": cpu_sample_desc(w, steps, el)}
+
+
 def cpu_sample_desc(w, steps, el, seqs=2):
     n = min(seqs, w.B)
     return (f"first {n} of {w.B} sequences ({n * w.H} heads), {steps} steps, "
@@ -713,7 +738,7 @@ def run_reference(args, world, rank):
         "config": {"workload": workload_desc(w, args.merge) + " (oracle: eager fp64)",
                    "name": w.name, "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "L": w.L},
         "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": cpu_sample_desc(w, steps, el, seqs)},
+                         "sample": cpu_sample_desc(w, steps, el, seqs), **host_cpu()},
         "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -774,7 +799,8 @@ def main():
             w = w.replace(L=args.L or w.L, B=args.B or w.B)
             v, steps, el, threads = oracle_tokens_per_s(w, target_s=args.cpu_seconds, warmup=1)
             line["cpu_baseline"] = {"value": round(v, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": cpu_sample_desc(w, steps, el)}
+                                    "sample": cpu_sample_desc(w, steps, el), **host_cpu(),
+                                    "single_core": oracle_single_core(w, args.cpu_seconds / 2)}
         if rank == 0:
             print(json.dumps(line), flush=True)
         if args.sweep:

@@ -61,5 +61,13 @@ def test_reference_arm_prints_the_contract_line():
         assert key in line, key
     assert line["steps"] == 2 and line["warmup"] == 3 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["nproc"] >= 1 and "cpu_model" in line["cpu_baseline"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["metric"] == bench.METRIC and line["unit"] == "tokens/s"
+
+
+def test_single_core_oracle_sample():
+    # the single-core figure of the CPU baseline: the oracle with one thread
+    w = bench.wl.WORKLOADS["gdn_tiny"]
+    r = bench.oracle_single_core(w, target_s=0.05)
+    assert r["cores"] == 1 and r["value"] > 0 and "sequences" in r["sample"]
