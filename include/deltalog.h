@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-/* Recurrence family ("We implement DeltaLog for GDN, KDA, and RWKV6"), plus
+/* Recurrence family (the DeltaLog page builds it for GDN, KDA and RWKV6), plus
  * GDN-2 (Gated DeltaNet-2 abstract: separate channel-wise erase and write
  * gates; KDA when both are the same scalar). */
 enum dl_variant { DL_GDN = 0, DL_KDA = 1, DL_RWKV6 = 2, DL_GDN2 = 3 };

@@ -14,8 +14,9 @@ recurrence exactly as written, forming the matrices the formula names
       o_t = S_t q_t,
   with S of shape d_v x d_k, alpha_t and beta_t scalars per head.
 
-* KDA (the same delta rule with channel-wise decay; Gated DeltaNet-2
-  abstract: "KDA sharpens forgetting with channel-wise decay"):
+* KDA (the same delta rule with channel-wise decay; the Gated DeltaNet-2
+  abstract credits KDA with a decay per key channel, which makes its
+  forgetting finer than GDN's one scalar):
       S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
       o_t = S_t q_t,
   alpha_t a vector over the d_k key channels.  The decay acts on the key
