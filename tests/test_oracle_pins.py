@@ -11,8 +11,8 @@ hold independently of it:
   orthonormal keys; the Frobenius norm never grows when v = 0, |k| = 1,
   beta in [0, 1], alpha <= 1;
 * a special case that reduces to another routine: KDA with a constant decay
-  vector is GDN ("KDA sharpens forgetting with channel-wise decay", Gated
-  DeltaNet-2 abstract);
+  vector is GDN (the Gated DeltaNet-2 abstract describes KDA as GDN with a
+  decay per key channel);
 * brute force: DeltaLog's log form in exact rationals (tests/logform_exact.py)
   equals the oracle for several L and fill offsets, and L = 1 (merge after
   every step) as well.
