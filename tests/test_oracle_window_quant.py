@@ -189,9 +189,50 @@ def pin_long_window_is_eager(wq):
     assert res.ends == []
 
 
+def pin_row_inverse_hand(wq):
+    # inv_j = 127 / amax_j in fp32 (amax over |x|), exact on these rows;
+    # zero rows and rows below 2^-120 give 0, a row at exactly 2^-120 is live
+    X = np.array([[127.0, -3.0, 5.0],
+                  [-254.0, 3.0, 0.0],
+                  [1.0, -0.5, 0.25],
+                  [0.0, 0.0, 0.0],
+                  [2.0 ** -121, -(2.0 ** -122), 0.0],
+                  [2.0 ** -120, 0.0, 0.0]])
+    inv = wq.row_inverse(X)
+    assert inv.dtype == np.float32 and inv.shape == (6,)
+    assert inv[:4].tolist() == [1.0, 0.5, 127.0, 0.0]
+    assert inv[4] == 0.0
+    assert inv[5] == np.float32(127.0 * 2.0 ** 120)  # exact: 127 * 2^120 is an fp32 value
+
+
+def pin_row_inverse_fp32(wq):
+    # 127/3 rounded once to fp32 has the bits 0x42295555 (binary expansion
+    # 101010.0101..., cut at 24 significant bits, next bit 0); the product with
+    # the element of pin_decision_in_fp32 is then exactly 10.5 in fp32
+    x = np.array([0x3E7DFBF8], dtype=np.uint32).view(np.float32)[0]
+    inv = wq.row_inverse(np.array([[3.0, float(x)], [-3.0, 1.0]]))
+    assert inv.dtype == np.float32
+    assert inv.view(np.uint32).tolist() == [0x42295555, 0x42295555]
+    assert np.float32(x) * inv[0] == np.float32(10.5)
+
+
+def pin_row_inverse_drives_codes(wq):
+    # the quantizer's codes are rint(fl32(x * inv)) clipped to +-127 with the
+    # same inv, on random rows of many magnitudes (ties the inverse to the
+    # hand-pinned codes above)
+    rng = np.random.default_rng(16)
+    X = rng.standard_normal((3, 12, 32)) * (10.0 ** rng.uniform(-6, 6, (3, 12, 1)))
+    X[0, 0] = 0.0
+    codes, _ = wq.quantize_rows(X)
+    inv = wq.row_inverse(X)
+    prod = (X.astype(np.float32) * inv[..., None]).astype(np.float32)
+    assert np.array_equal(codes.astype(np.int64), np.clip(np.rint(prod), -127, 127).astype(np.int64))
+
+
 WQ_PINS = [pin_hand_rows, pin_decision_in_fp32, pin_per_row_scale, pin_roundtrip_exact,
            pin_error_bound, pin_window_timing, pin_forced_merge_timing, pin_initial_quantization,
-           pin_rwkv6_orientation, pin_long_window_is_eager]
+           pin_rwkv6_orientation, pin_long_window_is_eager, pin_row_inverse_hand,
+           pin_row_inverse_fp32, pin_row_inverse_drives_codes]
 
 
 @pytest.mark.parametrize("pin", WQ_PINS, ids=lambda p: p.__name__)
@@ -283,20 +324,45 @@ Q_MUTANTS = {
     "scale_per_key_column": _quantizer(axis="col"),
     "scale_per_matrix": _quantizer(axis="all"),
 }
+def _inverse(qmax=127.0, fp32=True, cutoff="ge", absval=True):
+    """A copy of row_inverse with one planted mistake."""
+    def inv(X):
+        x = np.asarray(X).astype(np.float32 if fp32 else np.float64)
+        amax = np.max(np.abs(x) if absval else x, axis=-1)
+        tiny = wq_mod.TINY_AMAX
+        live = {"ge": amax >= tiny, "gt": amax > tiny, "none": amax > 0}[cutoff]
+        safe = np.where(live, amax, 1.0).astype(x.dtype)
+        return np.where(live, x.dtype.type(qmax) / safe, 0.0).astype(x.dtype)
+    return inv
+
+
+INV_MUTANTS = {
+    "inverse_128": _inverse(qmax=128.0),
+    "inverse_in_fp64": _inverse(fp32=False),
+    "inverse_no_tiny_cutoff": _inverse(cutoff="none"),
+    "inverse_strict_cutoff": _inverse(cutoff="gt"),
+    "inverse_signed_max": _inverse(absval=False),
+}
 W_MUTANTS = ["never", "late", "early", "no_forced", "no_initial", "key_rows"]
 
 
-@pytest.mark.parametrize("name", sorted(Q_MUTANTS) + ["window_" + k for k in W_MUTANTS])
+@pytest.mark.parametrize("name", sorted(Q_MUTANTS) + sorted(INV_MUTANTS)
+                         + ["window_" + k for k in W_MUTANTS])
 def test_window_quant_mutant_is_caught(name, monkeypatch):
     if name.startswith("window_"):
         mutant = _windowed_mutant(name[len("window_"):])
         impl = types.SimpleNamespace(quantize_rows=wq_mod.quantize_rows,
-                                     dequantize_rows=wq_mod.dequantize_rows, run_windowed=mutant)
+                                     dequantize_rows=wq_mod.dequantize_rows, run_windowed=mutant,
+                                     row_inverse=wq_mod.row_inverse)
+    elif name in INV_MUTANTS:
+        impl = types.SimpleNamespace(quantize_rows=wq_mod.quantize_rows,
+                                     dequantize_rows=wq_mod.dequantize_rows,
+                                     run_windowed=wq_mod.run_windowed, row_inverse=INV_MUTANTS[name])
     else:
         monkeypatch.setattr(wq_mod, "quantize_rows", Q_MUTANTS[name])
         impl = types.SimpleNamespace(quantize_rows=wq_mod.quantize_rows,
                                      dequantize_rows=wq_mod.dequantize_rows,
-                                     run_windowed=wq_mod.run_windowed)
+                                     run_windowed=wq_mod.run_windowed, row_inverse=wq_mod.row_inverse)
     failed = []
     for pin in WQ_PINS:
         try:
