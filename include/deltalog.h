@@ -80,12 +80,7 @@ enum dl_flags {
    * log writes the merged base instead and leaves an empty log, so the log
    * is never full and dl_merge(DL_MERGE_FULL) has nothing to do. */
   DL_FLAG_FUSED_MERGE = 1,
-  /* Run the step as a persistent warp-specialised kernel (one CTA per SM, a
-   * producer lane streaming work items through a ring of shared-memory
-   * stages) when its ring fits, instead of one CTA per work item.  A
-   * performance choice only; on B200 the default measured faster.  fp32
-   * base and GDN / KDA / RWKV6 only (else DL_ERR_UNSUPPORTED). */
-  DL_FLAG_PERSISTENT = 2,
+  /* Bit 2 is reserved (DL_ERR_ARG if set). */
   /* Kaczmarz step size (KLA, GDN and KDA only): the `beta` argument of a
    * step carries the gate eta_t and the kernels use
    * beta_t = eta_t / (|k_t|_2^2 + kla_eps) ("Kaczmarz Linear Attention"
@@ -106,8 +101,7 @@ enum dl_flags {
    * zero codes and scale 0); the base value is code_jc * scale_j.  Every
    * merge (DL_MERGE_FULL, DL_MERGE_ALL, the fused merge) folds the log in
    * fp32 and requantizes the rows it writes; dl_state_reset and
-   * dl_state_load_seqs quantize the states they load.  Not combinable with
-   * DL_FLAG_PERSISTENT (DL_ERR_UNSUPPORTED). */
+   * dl_state_load_seqs quantize the states they load. */
   DL_FLAG_BASE_Q8 = 8
 };
 
@@ -172,7 +166,9 @@ int dl_state_reset(dl_state* st, const float* S0, const int32_t* fill0, void* st
  * Errors: DL_ERR_ARG (bad or repeated index, n < 0), DL_ERR_ALIGN. */
 int dl_state_load_seqs(dl_state* st, int n, const int32_t* seqs, const float* S, void* stream);
 
-/* One decode step for all B*H heads (one kernel launch).
+/* One decode step for all B*H heads (one kernel launch).  Defines: the
+ * DeltaLog page, Abstract -- a decode step reads the base and the log and
+ * appends compact update factors instead of writing the full state back.
  *   q: q_t (r_t for RWKV6)  [B, H, d_k] in_dtype
  *   k: k_t                  [B, H, d_k] in_dtype
  *   v: v_t                  [B, H, d_v] in_dtype
@@ -194,21 +190,25 @@ int dl_decode_step(dl_state* st, const void* q, const void* k, const void* v,
                    float* o, void* stream);
 
 /* Folds logs into the base: S_b <- S_b Diag(gamma) + sum_i u_i (k_i o
- * gamma / gamma_i)^T, then empties those logs.  mode DL_MERGE_FULL folds
- * the sequences whose log holds L entries, DL_MERGE_ALL every non-empty
- * log.  Enqueues nothing when no sequence qualifies.  Like
+ * gamma / gamma_i)^T, then empties those logs.  Defines: the DeltaLog page,
+ * Abstract -- periodic merge steps fold the log back into the dense base.
+ * mode DL_MERGE_FULL folds the sequences whose log holds L entries,
+ * DL_MERGE_ALL every non-empty log.  Enqueues nothing when no sequence qualifies.  Like
  * dl_decode_step, the launch carries the qualifying sequences and their
  * fills by value (do not capture it in a CUDA graph). */
 int dl_merge(dl_state* st, int mode, void* stream);
 
 /* Writes the dense state S_t = base folded with the log to S_out (fp32
  * [B, H, d_v, d_k], 16-B aligned, must not alias the base) without changing
- * the state.  An int8 base is dequantized (code * scale) before the fold. */
+ * the state.  An int8 base is dequantized (code * scale) before the fold.
+ * Defines: the DeltaLog page, Abstract -- the model observes the same dense
+ * state as in eager decoding; this call produces that state on demand. */
 int dl_materialize(const dl_state* st, float* S_out, void* stream);
 
 /* Eager dense step, the comparison point: reads and writes the whole fp32
  * state S [B, H, d_v, d_k] (16-B aligned) in place, same recurrence and
- * arguments as dl_decode_step.  cfg->L and every flag but DL_FLAG_KLA are
+ * arguments as dl_decode_step.  Defines: the DeltaLog page, Abstract --
+ * eager decoding writes the full recurrent state back after every token.  cfg->L and every flag but DL_FLAG_KLA are
  * ignored (the state is always fp32). */
 int dl_eager_step(const dl_config* cfg, float* S, const void* q, const void* k,
                   const void* v, const float* decay, const float* beta,
@@ -222,8 +222,16 @@ int dl_state_destroy(dl_state* st);
 
 /* Reads and optionally clears the device error word that kernels set when
  * a bounded wait gives up or a device-side check fails (code 0 = none;
- * *head = first failing head).  `st` NULL reads the word the eager kernel
- * uses on the current device.  Synchronizes `stream`. */
+ * *head = first failing head).  Synchronizes `stream`.
+ *   - A state has its own word (in its meta buffer).  A nonzero code after a
+ *     step or a merge means some head's work was skipped part-way (a step
+ *     may already have advanced that head's fill, a merge may have folded
+ *     only some rows): the state is invalid until dl_state_reset.
+ *   - `st` NULL reads the one word per device that every dl_eager_step call
+ *     and dl_selftest_wait_timeout share: the first error recorded wins, so
+ *     with overlapping eager calls the head index may belong to either, and
+ *     the self-test clears the word (erasing what an earlier eager call
+ *     recorded). */
 int dl_device_error(dl_state* st, int32_t* code, int32_t* head, int clear, void* stream);
 
 /* Exercises the kernels' failure path on the current device without a

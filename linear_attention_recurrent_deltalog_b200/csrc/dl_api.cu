@@ -83,8 +83,7 @@ int check_config(const dl_config* c, bool need_L) {
   if (c->B < 1 || c->H < 1 || c->d_k < 1 || c->d_v < 1) return DL_ERR_ARG;
   if (c->in_dtype != DL_F32 && c->in_dtype != DL_BF16) return DL_ERR_ARG;
   if (need_L && (c->L < 1 || c->L > 64)) return DL_ERR_ARG;
-  if ((c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_PERSISTENT | DL_FLAG_KLA |
-                           DL_FLAG_BASE_Q8)) != 0)
+  if ((c->flags & ~int32_t(DL_FLAG_FUSED_MERGE | DL_FLAG_KLA | DL_FLAG_BASE_Q8)) != 0)
     return DL_ERR_ARG;
   if ((c->flags & DL_FLAG_KLA) &&
       (c->variant == DL_RWKV6 || c->variant == DL_GDN2 || !(c->kla_eps >= 0.f)))
@@ -94,14 +93,11 @@ int check_config(const dl_config* c, bool need_L) {
   if (bh * uint64_t(c->d_v) * uint64_t(c->d_k) >= (1ull << 40)) return DL_ERR_ARG;
   if (!head_size_ok(c->d_k) || !head_size_ok(c->d_v)) return DL_ERR_UNSUPPORTED;
   if (c->step_split != 0 && !dl::split_ok(c->d_v, c->step_split)) return DL_ERR_ARG;
-  if ((c->flags & DL_FLAG_PERSISTENT) && ((c->flags & DL_FLAG_BASE_Q8) || c->variant == DL_GDN2))
-    return DL_ERR_UNSUPPORTED;
   return DL_OK;
 }
 
 Shape shape_of(const dl_config& c) {
-  return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0, split_of(c),
-               (c.flags & DL_FLAG_PERSISTENT) ? 1 : 0};
+  return Shape{c.d_k, c.d_v, c.in_dtype == DL_BF16 ? 1 : 0, split_of(c)};
 }
 
 cudaError_t launch_step(const dl_config& c, const dl::StepParams& p, const dl::FillParam& fp,

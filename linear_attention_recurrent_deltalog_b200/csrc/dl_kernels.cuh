@@ -58,7 +58,6 @@ struct StepParams {
   float* o;
   int H;
   int L;
-  int nitems;    // work items (head rows) of a persistent launch
   int fills_in_param;  // 1: read fills from the FillParam argument
   int kla;       // 1: beta carries the KLA gate eta; beta = eta / (|k|^2 + kla_eps)
   float kla_eps;
@@ -1077,12 +1076,14 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
       sKt[x] = to_f(sK[x]) * expf(gl - sG[size_t(i) * GW + (GW > 1 ? c : 0)]);
     }
   }
-  if (tid == 0 && part == 0 && p.mode != 2) p.fill[head] = 0;
   if (!__syncthreads_and(ok)) {
     if (log_copies) mbar_wait(barLog, 0, nullptr, 0);
     for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
     return;
   }
+  // the log is emptied only once its entries are staged (a wait that gave
+  // up leaves the fill, and the error word says the state is invalid)
+  if (tid == 0 && part == 0 && p.mode != 2) p.fill[head] = 0;
 
   const int j0 = warp * Tl::kRowsPerWarp;
   uint64_t* barMine = &bars[j0 / Tl::kChunkRows];

@@ -9,7 +9,6 @@
 #include <cstdlib>
 
 #include "dl_kernels.cuh"
-#include "dl_step_persistent.cuh"
 
 namespace dl {
 
@@ -19,7 +18,6 @@ struct Shape {
   int dv;
   int bf16;        // 1: q/k/v are bf16, 0: fp32
   int split;       // step kernel: work items per head (1, 2 or 4; d_v / split >= 32)
-  int persistent;  // 1: persistent warp-specialised step kernel when its ring fits (fp32 base)
 };
 
 inline bool split_ok(int dv, int split) {
@@ -150,80 +148,15 @@ DL_DECLARE_VARIANT_LAUNCHERS(kVarGDN2)
 
 // Functors the shape dispatch calls (namespace scope: local classes cannot
 // have member templates).
-// Ring stages of the persistent step kernel that fit in shared memory
-// (capped by DELTALOG_MAX_STAGES, default 8).
-inline int max_stages() {
-  static const int m = [] {
-    const char* e = std::getenv("DELTALOG_MAX_STAGES");
-    const int v = (e && *e) ? std::atoi(e) : 8;
-    return v < 2 ? 2 : (v > 8 ? 8 : v);
-  }();
-  return m;
-}
-
-inline int sm_count() {
-  static std::atomic<int> cache[kMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-  int v = cache[dev].load(std::memory_order_relaxed);
-  if (v > 0) return v;
-  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  cache[dev].store(v, std::memory_order_relaxed);
-  return v;
-}
-
-template <int VAR, int DK, int DV, int ROWS, typename TIn>
-int persistent_stages(int L) {
-  const size_t stage = PStage<VAR, DK, DV, ROWS, TIn>(L).bytes + 16;
-  const int n = int((size_t(kMaxSmemOptIn) - 256) / stage);
-  return n < max_stages() ? n : max_stages();
-}
-
-// Persistent launch: one CTA per SM (or per item when there are fewer).
-// Returns cudaErrorNotSupported when its ring would have fewer than 2 stages.
-template <int VAR, int DK, int DV, int ROWS, typename TIn, bool FUSED>
-cudaError_t launch_step_persistent_t(const StepParams& p, const FillParam& fp, unsigned nheads,
-                                     cudaStream_t s) {
-  const int nst = persistent_stages<VAR, DK, DV, ROWS, TIn>(p.L);
-  if (nst < 2) return cudaErrorNotSupported;
-  static std::atomic<unsigned long long> done{0};
-  auto kern = dl_step_persistent_kernel<VAR, DK, DV, ROWS, TIn, FUSED>;
-  cudaError_t e = prepare_kernel(kern, done);
-  if (e != cudaSuccess) return e;
-  const size_t smem = size_t(nst) * PStage<VAR, DK, DV, ROWS, TIn>(p.L).bytes + 16 * size_t(nst);
-  const unsigned nitems = nheads * unsigned(DV / ROWS);
-  const int sms = sm_count();
-  if (sms <= 0) return cudaErrorInvalidDevice;
-  const unsigned grid = nitems < unsigned(sms) ? nitems : unsigned(sms);
-  StepParams q = p;
-  q.nitems = int(nitems);
-  kern<<<grid, PGeom<ROWS>::kThreads, smem, s>>>(q, nst, fp);
-  return cudaGetLastError();
-}
-
-template <int VAR, int DK, int DV, int ROWS, typename T, typename TB, bool FUSED>
-cudaError_t launch_step_rows(bool persistent, const StepParams& p, const FillParam& fp, unsigned n,
-                             cudaStream_t s) {
-  if constexpr (std::is_same<TB, float>::value && VAR != kVarGDN2) {
-    if (persistent) {
-      const cudaError_t e = launch_step_persistent_t<VAR, DK, DV, ROWS, T, FUSED>(p, fp, n, s);
-      if (e != cudaErrorNotSupported) return e;
-    }
-  }
-  return launch_step_t<VAR, DK, DV, ROWS, T, TB, FUSED>(p, fp, n, s);
-}
-
 template <int VAR, int DK, int DV, typename T, typename TB, bool FUSED>
-cudaError_t launch_step_split(int split, bool persistent, const StepParams& p, const FillParam& fp,
-                              unsigned n, cudaStream_t s) {
-  if (split == 1) return launch_step_rows<VAR, DK, DV, DV, T, TB, FUSED>(persistent, p, fp, n, s);
+cudaError_t launch_step_split(int split, const StepParams& p, const FillParam& fp, unsigned n,
+                              cudaStream_t s) {
+  if (split == 1) return launch_step_t<VAR, DK, DV, DV, T, TB, FUSED>(p, fp, n, s);
   if constexpr (DV / 2 >= 32) {
-    if (split == 2)
-      return launch_step_rows<VAR, DK, DV, DV / 2, T, TB, FUSED>(persistent, p, fp, n, s);
+    if (split == 2) return launch_step_t<VAR, DK, DV, DV / 2, T, TB, FUSED>(p, fp, n, s);
   }
   if constexpr (DV / 4 >= 32) {
-    if (split == 4)
-      return launch_step_rows<VAR, DK, DV, DV / 4, T, TB, FUSED>(persistent, p, fp, n, s);
+    if (split == 4) return launch_step_t<VAR, DK, DV, DV / 4, T, TB, FUSED>(p, fp, n, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -236,11 +169,10 @@ struct StepRun {
   cudaStream_t s;
   bool fused;
   int split;
-  bool persistent;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    return fused ? launch_step_split<VAR, DK, DV, T, TB, true>(split, persistent, p, fp, n, s)
-                 : launch_step_split<VAR, DK, DV, T, TB, false>(split, persistent, p, fp, n, s);
+    return fused ? launch_step_split<VAR, DK, DV, T, TB, true>(split, p, fp, n, s)
+                 : launch_step_split<VAR, DK, DV, T, TB, false>(split, p, fp, n, s);
   }
 };
 template <int VAR, typename TB>
@@ -297,7 +229,7 @@ struct MergeSmem {
   template <>                                                                              \
   cudaError_t launch_step<VAR, TB>(const Shape& sh, bool fused, const StepParams& p,       \
                                    const FillParam& fp, unsigned nheads, cudaStream_t s) { \
-    StepRun<VAR, TB> f{p, fp, nheads, s, fused, sh.split, sh.persistent != 0};              \
+    StepRun<VAR, TB> f{p, fp, nheads, s, fused, sh.split};              \
     return dispatch_shape(sh, f);                                                          \
   }                                                                                        \
   template <>                                                                              \

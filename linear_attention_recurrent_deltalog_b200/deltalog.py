@@ -32,7 +32,6 @@ DL_ERR_ARG, DL_ERR_ALIGN, DL_ERR_LOG_FULL = -1, -2, -3
 DL_ERR_CUDA, DL_ERR_UNSUPPORTED, DL_ERR_DEVICE = -4, -5, -6
 DL_MERGE_FULL, DL_MERGE_ALL = 0, 1
 DL_FLAG_FUSED_MERGE = 1
-DL_FLAG_PERSISTENT = 2
 DL_FLAG_KLA = 4
 DL_FLAG_BASE_Q8 = 8
 
@@ -132,7 +131,6 @@ class Config:
     in_dtype: str = "bf16"
     fused_merge: bool = False
     step_split: int = 0
-    persistent: bool = False
     kla_eps: Optional[float] = None  # set: beta carries the KLA gate eta
     base: str = "f32"                # "f32", or "q8": int8 codes + row scales
 
@@ -140,7 +138,6 @@ class Config:
         if self.base not in ("f32", "q8"):
             raise ValueError(f"base must be 'f32' or 'q8', not {self.base!r}")
         flags = (DL_FLAG_FUSED_MERGE if self.fused_merge else 0) | \
-            (DL_FLAG_PERSISTENT if self.persistent else 0) | \
             (DL_FLAG_KLA if self.kla_eps is not None else 0) | \
             (DL_FLAG_BASE_Q8 if self.base == "q8" else 0)
         return dl_config(VARIANT_IDS[self.variant], self.B, self.H, self.d_k, self.d_v, self.L,

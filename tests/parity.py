@@ -87,7 +87,7 @@ def _rel(a: np.ndarray, ref: np.ndarray) -> float:
 def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence[int]] = None,
                arms=("log", "fused", "eager"), snap_every: int = 64, L: Optional[int] = None,
                merge_all_at: Sequence[int] = (), workers: Optional[int] = None,
-               split: int = 0, persistent: bool = False, device="cuda",
+               split: int = 0, device="cuda",
                edit=None) -> Dict[str, ArmResult]:
     """Runs the given arms and the oracle; returns per-arm errors.  ``edit``
     (optional) maps each drawn StepInputs to the one both sides receive."""
@@ -111,7 +111,7 @@ def run_parity(w: wl.Workload, T: Optional[int] = None, heads: Optional[Sequence
             dense[arm] = S0_d.clone()
         else:
             cfg = dlb.Config(w.variant, w.B, w.H, dk, dv, w.L, w.in_dtype,
-                             fused_merge=(arm == "fused"), step_split=split, persistent=persistent,
+                             fused_merge=(arm == "fused"), step_split=split,
                              kla_eps=w.kla_eps)
             st = dlb.DeltaLogState(cfg, device=device)
             st.reset(S0_d, fill0.tolist())

@@ -97,11 +97,12 @@ def test_bad_enums_rejected():
     c = cfg().c()
     c.flags = 16
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
-    # the int8 base does not combine with the persistent step kernel
+    # bit 2 is reserved
+    c = cfg().c()
+    c.flags = 2
+    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
     c = cfg(base="q8").c()
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_OK
-    c = cfg(base="q8", persistent=True).c()
-    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_UNSUPPORTED
     with pytest.raises(ValueError):
         cfg(base="q4").c()
     # the KLA step size applies to GDN and KDA, with a non-negative epsilon
@@ -111,14 +112,12 @@ def test_bad_enums_rejected():
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
     c = cfg(kla_eps=-1.0).c()
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
-    # GDN-2: built for both bases; no KLA step size, no persistent kernel
+    # GDN-2: built for both bases; no KLA step size
     for base in ("f32", "q8"):
         c = cfg(variant="gdn2", base=base).c()
         assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_OK
     c = cfg(variant="gdn2", kla_eps=1e-6).c()
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG
-    c = cfg(variant="gdn2", persistent=True).c()
-    assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_UNSUPPORTED
     c = cfg().c()
     c.variant = 4
     assert dlb._lib.dl_state_bytes(ctypes.byref(c), None, None, None) == dlb.DL_ERR_ARG

@@ -59,3 +59,36 @@ def test_single_rank_helpers():
     import bench
     assert bench.max_over_ranks(1.5, 1, "cpu") == 1.5
     assert bench.aggregate_value(1000, 1, 0.5) == 2000
+
+
+def test_world_plan():
+    import bench
+    assert bench.world_plan(1, {}) == "run"
+    assert bench.world_plan(4, {}) == "spawn"
+    assert bench.world_plan(2, {"WORLD_SIZE": "2"}) == "run"
+    with pytest.raises(SystemExit):
+        bench.world_plan(8, {"WORLD_SIZE": "1"})
+    with pytest.raises(SystemExit):
+        bench.world_plan(0, {})
+    cmd = bench.spawn_command(2, ["--gpus", "2"], 29999)
+    assert "--nproc-per-node=2" in cmd and cmd[-2:] == ["--gpus", "2"]
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    # --gpus 2 with no launcher: bench.py starts 2 local ranks itself.  The
+    # oracle arm runs on CPU (gloo), so the launched world size shows in its
+    # line without a GPU.
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    env["DL_BENCH_BACKEND"] = "gloo"
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--impl",
+                          "reference", "--workload", "gdn_tiny", "--steps", "2", "--warmup", "3"],
+                         env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"

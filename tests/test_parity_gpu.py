@@ -68,28 +68,18 @@ def test_shapes_and_dtypes(variant, dk, dv, dtype):
     w = wl.WORKLOADS[base].replace(B=5, H=3, d_k=dk, d_v=dv, in_dtype=dtype, L=6, T=29,
                                    ragged=True)
     for split in (1, dv // 32):
-        for persistent in (True, False):
-            _check(run_parity(w, snap_every=7, workers=0, split=split, persistent=persistent))
+        _check(run_parity(w, snap_every=7, workers=0, split=split))
 
 
-@pytest.mark.parametrize("persistent", [True, False])
 @pytest.mark.parametrize("split", [1, 2, 4])
 @pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
-def test_step_split(name, split, persistent):
-    # a head cut into 1, 2 or 4 work items, persistent or one CTA per item
+def test_step_split(name, split):
+    # a head cut into 1, 2 or 4 work items
     w = wl.WORKLOADS[name]
     if w.d_v // split < 32:
         pytest.skip("d_v / split < 32 is not built")
     w = w.replace(B=6, H=5, L=8, T=27, ragged=True)
-    _check(run_parity(w, snap_every=9, workers=0, split=split, persistent=persistent,
-                      arms=("log", "fused")))
-
-
-@pytest.mark.parametrize("name", ["gdn_qwen", "kda", "rwkv6"])
-def test_persistent_full_workload(name):
-    w = wl.WORKLOADS[name]
-    res = run_parity(w, T=64, heads=wl.sample_heads(w, 24), persistent=True, arms=("fused",))
-    _check(res)
+    _check(run_parity(w, snap_every=9, workers=0, split=split, arms=("log", "fused")))
 
 
 @pytest.mark.parametrize("L", [1, 2, 64])
@@ -123,12 +113,11 @@ def test_large_batch_fallbacks(B):
                       arms=("log", "fused")))
 
 
-@pytest.mark.parametrize("persistent", [False, True])
 @pytest.mark.parametrize("name", ["gdn_qwen", "kda"])
-def test_kla_step_size(name, persistent):
+def test_kla_step_size(name):
     # beta = eta / (|k|^2 + eps) formed in the kernels, unnormalised keys
     w = wl.WORKLOADS[name].replace(B=6, H=5, L=8, T=27, ragged=True, kla_eps=1e-6)
-    _check(run_parity(w, snap_every=9, workers=0, persistent=persistent))
+    _check(run_parity(w, snap_every=9, workers=0))
     w = wl.WORKLOADS[name].replace(kla_eps=1e-3)
     _check(run_parity(w, T=40, heads=wl.sample_heads(w, 24), arms=("fused", "eager")))
 
