@@ -50,18 +50,49 @@ RING = 16
 L2_BYTES = 126 * 2**20
 FALLBACK_HBM_GBS = 6650.0
 
-# Step kernel source files: a traffic figure taken by ncu is reported only
-# while these are unchanged.
-KERNEL_SOURCES = ("linear_attention_recurrent_deltalog_b200/csrc/dl_kernels.cuh",
-                  "linear_attention_recurrent_deltalog_b200/csrc/dl_device.cuh")
+# Sources of each kernel: a DRAM traffic figure taken by ncu (a JSON record
+# under profiles/) is reported only while the sources it was taken from are
+# unchanged.
+_CSRC = "linear_attention_recurrent_deltalog_b200/csrc/"
+KERNEL_SOURCES = {
+    "dl_step_kernel": ("dl_device.cuh", "dl_common.cuh", "dl_q8.cuh", "dl_step.cuh"),
+    "dl_merge_kernel": ("dl_device.cuh", "dl_common.cuh", "dl_q8.cuh", "dl_merge.cuh"),
+    "dl_eager_kernel": ("dl_device.cuh", "dl_common.cuh", "dl_eager.cuh"),
+}
 
 
-def kernel_hash() -> str:
+def kernel_hash(kernel: str = "dl_step_kernel") -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, p), "rb") as f:
+    for p in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, _CSRC, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def traffic_record(kernel: str, **match):
+    """The committed ncu traffic record of `kernel` for this workload (every
+    key in `match` equal), taken from the current sources; None if there is
+    none."""
+    import glob
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*traffic*.json"))):
+        try:
+            with open(path) as f:
+                t = json.load(f)
+        except Exception:
+            continue
+        if not str(t.get("kernel", "")).startswith(kernel):
+            continue
+        if t.get("kernel_hash") != kernel_hash(kernel):
+            continue
+        if all(t.get(k, "f32" if k == "base" else None) == v for k, v in match.items()):
+            return t
+    return None
+
+
+def mean_dram(t, key):
+    """Mean per-launch DRAM bytes (`dram_read` or `dram_write`) of a record."""
+    xs = [float(x[key]) for x in t.get("launches", [])]
+    return sum(xs) / len(xs) if xs else None
 
 
 def hbm_peak():
@@ -506,17 +537,9 @@ def run_ours(args, world, rank, local):
     step_avg = step_kernel_s / args.steps
     step_bytes_avg = (rd + wr) / args.steps
     achieved = step_bytes_avg / step_avg / 1e9
-    traffic = None
-    import glob
-    for tfile in sorted(glob.glob(os.path.join(ROOT, "profiles", "step_kernel_traffic*.json"))):
-        try:
-            t = json.load(open(tfile))
-        except Exception:
-            continue
-        if (t.get("kernel_hash") == kernel_hash() and t.get("L") == w.L and t.get("merge") == args.merge
-                and t.get("workload") == w.name and t.get("B") == w.B
-                and t.get("base", "f32") == args.base):
-            traffic = t.get("bytes_per_launch")
+    rec = traffic_record("dl_step_kernel", workload=w.name, B=w.B, L=w.L, merge=args.merge,
+                         base=args.base)
+    traffic = rec.get("bytes_per_launch") if rec else None
 
     if args.only_step:
         st.close()
@@ -681,9 +704,7 @@ def run_ours(args, world, rank, local):
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "clocks": clk.summary(),
         "hbm_gbs_step_plus_merge": round(((rd + wr + mrd + mwr) / args.steps) / (max_elapsed / args.steps) / 1e9, 1),
-        "write_bytes_per_token": {"deltalog": round((wr + mwr) / args.steps / w.B, 1),
-                                  "eager": round(ewr / w.B, 1),
-                                  "reduction": round(ewr / ((wr + mwr) / args.steps), 3)},
+        "write_bytes_per_token": write_bytes_line(w, args, wr + mwr, ewr, rec),
         "merge_kernel": merge_k,
         "materialize_kernel": mat_k,
         "eager": {"value": round(aggregate_value(tokens, 1, eager_s), 1), "unit": UNIT,
@@ -692,6 +713,27 @@ def run_ours(args, world, rank, local):
                   "speedup_of_deltalog": round(eager_s / elapsed, 3)},
     }
     return line
+
+
+def write_bytes_line(w, args, dl_write_total, eager_write, step_rec):
+    """State write bytes per token: algorithmic (DeltaLog's timed steps and
+    the eager step), and measured (DRAM writes per launch from the committed
+    ncu records of the step and eager kernels at this batch, while both
+    kernels' sources are unchanged)."""
+    out = {"deltalog": round(dl_write_total / args.steps / w.B, 1),
+           "eager": round(eager_write / w.B, 1),
+           "reduction": round(eager_write / (dl_write_total / args.steps), 3)}
+    eager_rec = traffic_record("dl_eager_kernel", workload=w.name, B=w.B)
+    sw = mean_dram(step_rec, "dram_write") if step_rec and args.merge == "fused" else None
+    ew = mean_dram(eager_rec, "dram_write") if eager_rec else None
+    if sw and ew:
+        out["measured"] = {"deltalog_dram_write_per_token": round(sw / w.B, 1),
+                           "eager_dram_write_per_token": round(ew / w.B, 1),
+                           "measured_reduction": round(ew / sw, 3),
+                           "source": "profiles/ ncu records (dram__bytes_write.sum per launch)"}
+    else:
+        out["measured"] = None
+    return out
 
 
 # ------------------------------------------------------------ serving loop

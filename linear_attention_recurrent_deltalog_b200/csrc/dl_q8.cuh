@@ -1,0 +1,252 @@
+// dl_q8.cuh -- per-warp operations on an int8 base (codes + row scales) on the
+// tensor cores: the base GEMV and the fold of the log into requantized rows.
+#pragma once
+
+#include "dl_common.cuh"
+
+namespace dl {
+
+// ---------------------------------------------------- int8 base rows
+//
+// The same per-warp operations on an int8 base, on the tensor cores (see
+// dl_device.cuh): a warp's 16 rows are one m16 tile.  Codes sit in shared
+// memory in the swizzled order of q8_off.
+
+// Number of 16-entry chunks the fold's k dimension is cut into.
+__host__ __device__ constexpr int q8_chunks(int L) { return (L + 15) / 16; }
+
+// Row stride (in halves) of the GEMV's fp16 vectors: 32 bytes of padding put
+// the four rows (read together by lanes 4g + t, g < 4) in different banks.
+template <int DK>
+constexpr int kVecHStride = DK + 16;
+
+// Base GEMV on the tensor cores: A = the warp's 16 rows of codes, B = the
+// four fp16 vectors of sVecH [4][kVecHStride] (columns: k-hat hi, k-hat lo, q-hat hi,
+// q-hat lo; the other four columns are zero), so D's columns 0+1 hold S k-hat
+// and 2+3 hold S q-hat.  Inside each 16-channel k-step, logical k (2t, 2t+1,
+// 2t+8, 2t+9) is channel (4t .. 4t+3): A and B agree, so the dot products
+// are unchanged.  Lane 4g + t with t < 2 finishes row jl = j0 + g (t = 0) or
+// j0 + g + 8 (t = 1), scaled by its row scale; `owner` is false elsewhere.
+template <int DK>
+__device__ __forceinline__ void rows_gemv_q8(const int8_t* sQ, const float* sScale, int j0, int lane,
+                                             const __half* sVecH, float& a, float& b, int& jl,
+                                             bool& owner) {
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  const int m = lane >> 3;                       // ldmatrix: which matrix this lane addresses
+  const int arow = j0 + (lane & 7) + 8 * (m & 1);
+#pragma unroll
+  for (int kk = 0; kk < DK / 16; kk += 2) {
+    uint32_t w[4];
+    ldmatrix_x4(w, sQ + q8_off<DK>(arow, 16 * (kk + (m >> 1))));
+    uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+    codes4_to_h2(w[0], a0, a2);  // row g,   channels 16 kk + 4t ..
+    codes4_to_h2(w[1], a1, a3);  // row g+8
+    codes4_to_h2(w[2], c0, c2);  // row g,   next k-step
+    codes4_to_h2(w[3], c1, c3);  // row g+8, next k-step
+    uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
+    if (g < 4) {
+      b0 = *reinterpret_cast<const uint2*>(sVecH + g * kVecHStride<DK> + 16 * kk + 4 * t);
+      b1 = *reinterpret_cast<const uint2*>(sVecH + g * kVecHStride<DK> + 16 * (kk + 1) + 4 * t);
+    }
+    mma_16816(d, a0, a1, a2, a3, b0.x, b0.y);
+    mma_16816(d, c0, c1, c2, c3, b1.x, b1.y);
+  }
+  // t = 0 holds S k-hat (rows g, g+8), t = 1 holds S q-hat; trade halves
+  const float send = (t == 0) ? d[2] + d[3] : d[0] + d[1];
+  const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+  owner = t < 2;
+  jl = j0 + g + ((t == 1) ? 8 : 0);
+  const float own = (t == 1) ? d[2] + d[3] : d[0] + d[1];
+  a = (t == 0) ? own : recv;
+  b = (t == 0) ? recv : own;
+  const float sc = sScale[jl];
+  a *= sc;
+  b *= sc;
+}
+
+// Key channel of column j (0..7) of n-tile n in the fold's MMAs.  The fold
+// permutes the N dimension so that lane 4g + t, whose accumulators hold
+// columns 2t and 2t+1 of every n-tile, owns the DK/4 contiguous channels
+// [DK/4 t, DK/4 (t+1)) of its two rows: whole 16-byte groups of codes to
+// load and store.
+template <int DK>
+__host__ __device__ constexpr int fold_channel(int n, int j) {
+  return (DK / 4) * (j >> 1) + 2 * n + (j & 1);
+}
+
+// Slot of lane l's 16-byte B fragment for n-tile n in the staged array: the
+// lane index is XOR-ed with n mod 8, which leaves the fold's loads (one
+// n-tile, 32 lanes) conflict-free and spreads the staging stores over all
+// bank groups.
+__host__ __device__ constexpr int kt_slot(int kc, int ntiles, int n, int l) {
+  return (kc * ntiles + n) * 32 + (l ^ (n & 7));
+}
+
+// Stages the decayed keys kt_e[c] = k_e[c] e^{gLast[c] - g_e[c]} (factor 1
+// for entries e >= nlog, 0 for e >= nent) as fp16 hi/lo B fragments of the
+// fold: for 16-entry chunk kc and n-tile n, lane l's 16 bytes {b0 hi, b1 hi,
+// b0 lo, b1 lo} sit at kt_slot (column l/4 of the n-tile is key channel
+// fold_channel(n, l/4)).  A thread takes one key channel of one chunk: it
+// reads the chunk's 16 keys of that channel (consecutive threads read
+// consecutive channels) and writes the four lanes' fragments that carry
+// them.  GDN's decay is one factor per entry, from sFac (filled by the
+// caller); the vector decays take it per channel.  All threads of the CTA
+// take part; the caller synchronises afterwards.
+template <int VAR, int DK, typename TIn>
+__device__ __forceinline__ void stage_kt_frags(const TIn* sK, const float* sG, const float* gLast,
+                                               const float* sFac, int nlog, int nent, int nchunks,
+                                               uint32_t* sB, int tid, int nt) {
+  constexpr int NTILE = DK / 8;
+  constexpr int CPL = DK / 4;
+  for (int idx = tid; idx < nchunks * DK; idx += nt) {
+    const int c = idx % DK;
+    const int kc = idx / DK;
+    // inverse of fold_channel: c = CPL (j / 2) + 2 n + (j mod 2)
+    const int n = (c % CPL) >> 1;
+    const int j = 2 * (c / CPL) + (c & 1);
+    float x[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int e = 16 * kc + q;
+      float v = 0.f;
+      if (e < nent) {
+        v = to_f(sK[size_t(e) * DK + c]);
+        if (e < nlog)
+          v *= (VAR == kVarGDN) ? sFac[e] : expf(gLast[c] - sG[size_t(e) * DK + c]);
+      }
+      x[q] = v;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      uint4 w;
+      split_h2(x[2 * t], x[2 * t + 1], w.x, w.z);          // b0: entries 2t, 2t+1
+      split_h2(x[2 * t + 8], x[2 * t + 9], w.y, w.w);      // b1: entries 2t+8, 2t+9
+      reinterpret_cast<uint4*>(sB)[kt_slot(kc, NTILE, n, 4 * j + t)] = w;
+    }
+  }
+}
+
+// Index of key channel c in the fold's padded decay array: 16 bytes of
+// padding after every 32 channels put the four lanes of a row group (which
+// read their 32 channels each as float4s) in different bank groups.
+__host__ __device__ constexpr int dec_pad(int c) { return c + ((c >> 5) << 2); }
+template <int DK>
+constexpr int kDecPadLen = DK + DK / 8;
+
+// Folds nent log entries into the warp's 16 rows of an int8 base on the
+// tensor cores, in one pass:
+//   x = deq(code) * dec + U Kt,   deq(code) = code * scale,
+// U = the rows' u values (A, split hi/lo in registers), Kt = the staged B
+// fragments, sDec the base decay at dec_pad indices (SDEC: one scalar decay,
+// any entry).  Lane 4g + t holds rows j0+g and j0+g+8 over the key channels
+// [DK/4 t, DK/4 (t+1)) (fold_channel).  With gOut the rows are written to it
+// as fp32 (unswizzled); otherwise each row's absolute maximum is reduced
+// over its four lanes and the row is requantized straight from the
+// accumulators into gCodes (swizzled order) and gScale.
+template <int DK, typename TU, bool SDEC>
+__device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sScale, const TU* sU,
+                                             const uint32_t* sB, const float* sDec, int nent,
+                                             int nchunks, int L, int j0, int lane, int8_t* gCodes,
+                                             float* gScale, float* gOut) {
+  constexpr int NTILE = DK / 8;      // n-tiles; lane holds 2 channels of each
+  constexpr int CPL = DK / 4;        // contiguous channels per lane
+  constexpr int WORDS = CPL / 4;     // 4-code words per lane per row
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int cbase = CPL * t;
+  const int rows[2] = {j0 + g, j0 + g + 8};
+  // acc[n][0..1]: row g, channels cbase + 2n, +1; acc[n][2..3]: row g+8
+  float acc[NTILE][4];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int r = rows[half];
+    const float s = sScale[r];
+    uint32_t w[WORDS];
+#pragma unroll
+    for (int v = 0; v < WORDS / 4; ++v) {
+      const uint4 q = *reinterpret_cast<const uint4*>(sQ + q8_off<DK>(r, cbase + 16 * v));
+      w[4 * v] = q.x;
+      w[4 * v + 1] = q.y;
+      w[4 * v + 2] = q.z;
+      w[4 * v + 3] = q.w;
+    }
+    const float sd = SDEC ? s * sDec[0] : 0.f;
+#pragma unroll
+    for (int v = 0; v < WORDS; ++v) {
+      uint32_t h01, h23;
+      codes4_to_h2(w[v], h01, h23);
+      const float2 c01 = __half22float2(bits_h2(h01));
+      const float2 c23 = __half22float2(bits_h2(h23));
+      if (SDEC) {
+        acc[2 * v][2 * half] = c01.x * sd;
+        acc[2 * v][2 * half + 1] = c01.y * sd;
+        acc[2 * v + 1][2 * half] = c23.x * sd;
+        acc[2 * v + 1][2 * half + 1] = c23.y * sd;
+      } else {
+        const float4 d4 = *reinterpret_cast<const float4*>(sDec + dec_pad(cbase + 4 * v));
+        acc[2 * v][2 * half] = (c01.x * s) * d4.x;
+        acc[2 * v][2 * half + 1] = (c01.y * s) * d4.y;
+        acc[2 * v + 1][2 * half] = (c23.x * s) * d4.z;
+        acc[2 * v + 1][2 * half + 1] = (c23.y * s) * d4.w;
+      }
+    }
+  }
+  const uint4* sB4 = reinterpret_cast<const uint4*>(sB);
+  for (int kc = 0; kc < nchunks; ++kc) {
+    const int e0 = 16 * kc + 2 * t;
+    float u[8];  // (g, e0), (g, e0+1), (g+8, e0), (g+8, e0+1), then the same at e0+8
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = e0 + (q & 1) + ((q & 4) ? 8 : 0);
+      u[q] = (e < nent) ? to_f(sU[su_offset(rows[(q >> 1) & 1], e, L)]) : 0.f;
+    }
+    uint32_t ah[4], al[4];
+    split_h2(u[0], u[1], ah[0], al[0]);  // a0: row g,   k 2t..
+    split_h2(u[2], u[3], ah[1], al[1]);  // a1: row g+8
+    split_h2(u[4], u[5], ah[2], al[2]);  // a2: row g,   k 2t+8..
+    split_h2(u[6], u[7], ah[3], al[3]);  // a3: row g+8
+#pragma unroll
+    for (int n = 0; n < NTILE; ++n) {
+      const uint4 bf = sB4[kt_slot(kc, NTILE, n, lane)];
+      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.x, bf.y);
+      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.z, bf.w);
+      mma_16816(acc[n], al[0], al[1], al[2], al[3], bf.x, bf.y);
+    }
+  }
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int r = rows[half];
+    if (gOut != nullptr) {
+      float4* o = reinterpret_cast<float4*>(gOut + size_t(r) * DK + cbase);
+#pragma unroll
+      for (int v = 0; v < WORDS; ++v)
+        o[v] = make_float4(acc[2 * v][2 * half], acc[2 * v][2 * half + 1], acc[2 * v + 1][2 * half],
+                           acc[2 * v + 1][2 * half + 1]);
+      continue;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int n = 0; n < NTILE; ++n)
+      m = fmaxf(m, fmaxf(fabsf(acc[n][2 * half]), fabsf(acc[n][2 * half + 1])));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    // rows below the tiny threshold store zero codes (inv = 0) and scale 0
+    const float inv = (m >= kTinyAmax) ? __fdiv_rn(127.0f, m) : 0.f;
+    uint32_t w[WORDS];
+#pragma unroll
+    for (int v = 0; v < WORDS; ++v)
+      w[v] = pack_codes4(round_code_bits(acc[2 * v][2 * half], inv),
+                         round_code_bits(acc[2 * v][2 * half + 1], inv),
+                         round_code_bits(acc[2 * v + 1][2 * half], inv),
+                         round_code_bits(acc[2 * v + 1][2 * half + 1], inv));
+#pragma unroll
+    for (int v = 0; v < WORDS / 4; ++v)
+      *reinterpret_cast<uint4*>(gCodes + q8_off<DK>(r, cbase + 16 * v)) =
+          make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    if (t == 0) gScale[r] = (m >= kTinyAmax) ? __fdiv_rn(m, 127.0f) : 0.f;
+  }
+}
+
+}  // namespace dl

@@ -1,0 +1,320 @@
+// dl_step.cuh -- the DeltaLog decode step kernel.
+#pragma once
+
+#include "dl_common.cuh"
+#include "dl_q8.cuh"
+
+namespace dl {
+
+// ------------------------------------------------------------------ step
+//
+// A head's rows may be split over SPLIT = DV / ROWS CTAs (blockIdx.x =
+// head * SPLIT + part).  Rows are independent in the GEMV, the correction
+// and the readout; every part recomputes the per-head scalars (cheap) and
+// stages all f log keys but only its own rows of the log's u vectors.  The
+// smaller shared-memory footprint lets more CTAs -- and more bytes in
+// flight -- sit on each SM.  Part 0 appends k_t and g_t and advances the
+// fill; fills are double-buffered by step parity (read fill_in, write
+// fill_out), so no CTA ever reads a counter another CTA of the same launch
+// writes.
+//
+// Order inside a CTA: the tile's bulk copies go out first (they do not
+// depend on anything), then the fill is read and the log's copies go out;
+// the per-head vectors are loaded meanwhile.  After one barrier, the
+// log-decay bookkeeping and the per-entry weights are computed together, a
+// second barrier publishes them, and each warp streams its rows.
+
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB = float,
+          bool FUSED = true>
+struct StepLayout {
+  using TU = typename LogU<VAR, TIn>::type;
+  static constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
+  static constexpr bool Q8 = std::is_same<TB, int8_t>::value;
+  size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offBonus,
+      offWg, offScale, offVecH, offDecF, offKt, offBar, total;
+  __host__ __device__ explicit StepLayout(int L) {
+    offU = Tile<DK, ROWS, TB>::kTileBytes;
+    offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
+    offG = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
+    offQr = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
+    offKr = offQr + align_up(size_t(DK) * sizeof(TIn), 128);
+    offVr = offKr + align_up(size_t(DK) * sizeof(TIn), 128);
+    offDecV = offVr + align_up(size_t(ROWS) * sizeof(TIn), 128);
+    offVec = offDecV + align_up(size_t(GW) * 4, 128);
+    // fp32 k, q, k-hat, q-hat [DK] each; g_t, g_{t-1} [GW]
+    offW = offVec + align_up(size_t(4 * DK + 2 * GW) * 4, 128);
+    offZ = offW + align_up(size_t(L) * 4, 16);
+    offScal = offZ + align_up(size_t(L) * 4, 16);
+    // RWKV6: the bonus u [DK]; GDN-2: the erase gate b [DK] and this CTA's
+    // rows of the write gate w [ROWS]
+    offBonus = offScal + 64;
+    offWg = offBonus + ((VAR == kVarRWKV6 || VAR == kVarGDN2) ? align_up(size_t(DK) * 4, 128) : 0);
+    // int8 base: the CTA's row scales, the GEMV's fp16 vectors [4][DK] and,
+    // for the fused merge only, the base decay [DK] and the staged key
+    // fragments
+    offScale = offWg + (VAR == kVarGDN2 ? align_up(size_t(ROWS) * 4, 128) : 0);
+    offVecH = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
+    offDecF = offVecH + (Q8 ? align_up(size_t(4) * kVecHStride<DK> * 2, 128) : 0);
+    offKt = offDecF + ((Q8 && FUSED) ? align_up(size_t(kDecPadLen<DK>) * 4, 128) : 0);
+    offBar = offKt + ((Q8 && FUSED) ? size_t(q8_chunks(L)) * DK * 64 : 0);
+    total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
+  }
+};
+
+// Resident CTAs per SM the int8 kernels are compiled for: the plain step
+// 1152 threads per SM (56 registers a thread), the step with the fused merge
+// and the merge 768 (80 registers; the fold's accumulators may spill a
+// little), so the rare fold does not set the occupancy of every step.  The
+// fp32 kernels keep the compiler's choice.
+template <typename TB, int THREADS, bool FOLDS>
+constexpr int kMinBlocks =
+    std::is_same<TB, int8_t>::value ? (FOLDS ? 768 : 1152) / THREADS : 1;
+
+template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB, bool FUSED>
+__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads,
+                                  kMinBlocks<TB, Tile<DK, ROWS, TB>::kThreads, FUSED>)
+dl_step_kernel(const StepParams p, const FillParam fp) {
+  using Tl = Tile<DK, ROWS, TB>;
+  using TU = typename LogU<VAR, TIn>::type;
+  constexpr bool Q8 = std::is_same<TB, int8_t>::value;
+  constexpr int SPLIT = DV / ROWS;
+  constexpr int GW = StepLayout<VAR, DK, DV, ROWS, TIn, TB, FUSED>::GW;
+  constexpr int NT = Tl::kThreads;
+  constexpr int NW = Tl::kWarps;
+  constexpr int CPL = Tl::kCPL;
+  static_assert(DV % ROWS == 0, "rows split evenly");
+  static_assert(NW >= 2, "one warp issues the tile copies, another the small ones");
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int L = p.L;
+  const int GS = g_stride(VAR, L, DK);
+  const StepLayout<VAR, DK, DV, ROWS, TIn, TB, FUSED> lay(L);
+  TB* sS = reinterpret_cast<TB*>(smem);                       // [ROWS][DK]
+  TU* sU = reinterpret_cast<TU*>(smem + lay.offU);            // [ROWS/32][L][32]
+  TIn* sK = reinterpret_cast<TIn*>(smem + lay.offK);          // [L][DK]
+  float* sG = reinterpret_cast<float*>(smem + lay.offG);      // [L][GW]
+  TIn* sQr = reinterpret_cast<TIn*>(smem + lay.offQr);        // q_t (r_t) as given
+  TIn* sKr = reinterpret_cast<TIn*>(smem + lay.offKr);        // k_t as given
+  TIn* sVr = reinterpret_cast<TIn*>(smem + lay.offVr);        // this part's rows of v_t
+  float* sDecV = reinterpret_cast<float*>(smem + lay.offDecV);  // decay_t (vector variants)
+  float* sk = reinterpret_cast<float*>(smem + lay.offVec);    // k_t (fp32)
+  float* sq = sk + DK;                                        // q_t / r_t (fp32)
+  float* sKh = sq + DK;                                       // GEMV vector for a
+  float* sQh = sKh + DK;                                      // GEMV vector for b
+  float* sGt = sQh + DK;                                      // g_t
+  float* sGp = sGt + GW;                                      // g_{t-1}
+  float* sW = reinterpret_cast<float*>(smem + lay.offW);      // per-entry weights on k
+  float* sZ = reinterpret_cast<float*>(smem + lay.offZ);      // per-entry weights on q / r
+  float* sScal = reinterpret_cast<float*>(smem + lay.offScal);  // [0] k.q / bonus [1] beta
+                                                                // [2] e^{g_t}
+  float* sBonus = reinterpret_cast<float*>(smem + lay.offBonus);  // RWKV6: u; GDN-2: b [DK]
+  float* sWg = reinterpret_cast<float*>(smem + lay.offWg);        // GDN-2: w, this CTA's rows
+  float* sScale = reinterpret_cast<float*>(smem + lay.offScale);  // int8 base: row scales
+  __half* sVecH = reinterpret_cast<__half*>(smem + lay.offVecH);  // GEMV vectors, fp16 hi/lo
+  float* sDecF = reinterpret_cast<float*>(smem + lay.offDecF);    // fused merge: base decay
+  uint32_t* sB = reinterpret_cast<uint32_t*>(smem + lay.offKt);   // fused merge: key fragments
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + lay.offBar);
+  uint64_t* barLog = &bars[Tl::kChunks];
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const size_t head = blockIdx.x / SPLIT;
+  const int part = static_cast<int>(blockIdx.x % SPLIT);
+  const int r0 = part * ROWS;  // first value row of this CTA
+  const int h = static_cast<int>(head % static_cast<size_t>(p.H));
+  const int f = step_fill(p, fp, head);
+  if (f < 0 || f >= L) {  // the host never launches a step on a full log
+    if (tid == 0 && p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
+    return;
+  }
+  const bool merge_now = FUSED && (f + 1 == L);
+  const bool appender = (part == 0) && !merge_now;
+
+  const TB* gS = static_cast<const TB*>(p.base) + (head * size_t(DV) + r0) * DK;
+  TU* gU = static_cast<TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
+  TIn* gK = static_cast<TIn*>(p.logK) + head * size_t(L) * DK;
+  float* gG = p.logG + head * size_t(GS);
+
+  // Warp 0 streams the tile; warp 1 fetches everything small (the step's
+  // vectors and the f log entries).  Each thread reads the two per-head
+  // scalars no bulk copy can carry (GDN's decay, beta) into registers, so
+  // no barrier waits on those loads.
+  const float dec_s = (GW == 1) ? __ldg(p.decay + head) : 0.f;
+  const float beta_s = (VAR == kVarRWKV6 || VAR == kVarGDN2) ? 0.f : __ldg(p.beta + head);
+  if (warp == 0 && lane == 0) {
+#pragma unroll
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_init(&bars[c], 1);
+    fence_mbar_init();
+#pragma unroll
+    for (int c = 0; c < Tl::kChunks; ++c) {
+      mbar_arrive_expect_tx(&bars[c], Tl::kChunkBytes);
+      tma_load_1d_stream(sS + size_t(c) * Tl::kChunkRows * DK, gS + size_t(c) * Tl::kChunkRows * DK,
+                         Tl::kChunkBytes, &bars[c]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    mbar_init(barLog, 1);
+    fence_mbar_init();
+    const uint32_t bq = DK * sizeof(TIn);
+    const uint32_t bv = ROWS * sizeof(TIn);
+    const uint32_t bd = (GW > 1) ? DK * 4u : 0u;
+    const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one row block
+    const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
+    const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
+    const uint32_t bs = Q8 ? ROWS * 4u : 0u;
+    const uint32_t bb = (VAR == kVarRWKV6 || VAR == kVarGDN2) ? DK * 4u : 0u;
+    const uint32_t bw = (VAR == kVarGDN2) ? ROWS * 4u : 0u;
+    mbar_arrive_expect_tx(barLog,
+                          2 * bq + bv + bd + bu * uint32_t(ROWS / kURows) + bk + bg + bs + bb + bw);
+    if (Q8) tma_load_1d(sScale, p.scale + head * DV + r0, bs, barLog);
+    if (VAR == kVarRWKV6) tma_load_1d(sBonus, p.bonus + size_t(h) * DK, bb, barLog);
+    if (VAR == kVarGDN2) {
+      tma_load_1d(sBonus, p.beta + head * DK, bb, barLog);        // erase gate b_t
+      tma_load_1d(sWg, p.bonus + head * DV + r0, bw, barLog);      // write gate w_t rows
+    }
+    tma_load_1d(sQr, static_cast<const TIn*>(p.q) + head * DK, bq, barLog);
+    tma_load_1d(sKr, static_cast<const TIn*>(p.k) + head * DK, bq, barLog);
+    tma_load_1d(sVr, static_cast<const TIn*>(p.v) + head * DV + r0, bv, barLog);
+    if (GW > 1) tma_load_1d(sDecV, p.decay + head * DK, bd, barLog);
+    if (f > 0) {
+      tma_load_1d(sK, gK, bk, barLog);
+      tma_load_1d(sG, gG, bg, barLog);
+      for (int rb = 0; rb < ROWS / kURows; ++rb)
+        tma_load_1d(sU + size_t(rb) * L * kURows, gU + u_offset(0, r0 + rb * kURows, 0, L, DV), bu,
+                    barLog);
+    }
+    if (part == 0) p.fill_out[head] = merge_now ? 0 : f + 1;
+  }
+  __syncthreads();
+
+  // ---- decay bookkeeping, appends of k and g, per-entry weights
+  const bool ok = mbar_wait(barLog, 0, p.err, int(head));
+  for (int c = tid; c < DK; c += NT) {
+    const TIn kraw = sKr[c];
+    const float kc = to_f(kraw);
+    const float qc = to_f(sQr[c]);
+    sk[c] = kc;
+    sq[c] = qc;
+    if (GW > 1) {
+      const float gp = (f > 0) ? sG[size_t(f - 1) * DK + c] : 0.f;
+      const float gt = gp + logf(sDecV[c]);
+      sGp[c] = gp;
+      sGt[c] = gt;
+      if (VAR == kVarKDA || VAR == kVarGDN2) {
+        const float e = expf(gt);
+        sKh[c] = (VAR == kVarGDN2) ? e * (sBonus[c] * kc) : e * kc;
+        sQh[c] = e * qc;
+      } else {  // RWKV6 reads S_{t-1}: decay up to the previous step
+        sQh[c] = expf(gp) * qc;
+      }
+      if (appender) gG[size_t(f) * DK + c] = gt;
+    }
+    if (merge_now)
+      sK[size_t(f) * DK + c] = kraw;
+    else if (appender)
+      gK[size_t(f) * DK + c] = kraw;
+    if constexpr (Q8) {  // the GEMV's B columns: k-hat and q-hat as fp16 hi/lo pairs
+      const float va = (VAR == kVarGDN) ? kc : (VAR == kVarRWKV6 ? 0.f : sKh[c]);
+      const float vb = (VAR == kVarGDN) ? qc : sQh[c];
+      uint32_t hi, lo;
+      split_h2(va, vb, hi, lo);
+      const __half2 h = bits_h2(hi), l = bits_h2(lo);
+      constexpr int VS = kVecHStride<DK>;
+      sVecH[c] = __low2half(h);
+      sVecH[VS + c] = __low2half(l);
+      sVecH[2 * VS + c] = __high2half(h);
+      sVecH[3 * VS + c] = __high2half(l);
+    }
+  }
+  if (GW == 1 && tid == NT - 1) {
+    const float gp = (f > 0) ? sG[f - 1] : 0.f;
+    const float gt = gp + logf(dec_s);
+    sGp[0] = gp;
+    sGt[0] = gt;
+    sScal[2] = expf(gt);
+    if (appender) gG[f] = gt;
+  }
+  if (f > 0)
+    // the int8 GDN step is issue-bound: fewest instructions (8 lanes per entry)
+    entry_weights<VAR, DK, TIn, TIn, !(Q8 && VAR == kVarGDN)>(f, warp, NW, lane, sKr, sQr, sK, sG,
+                                                              (GW == 1) ? &dec_s : sDecV, sW, sZ,
+                                                              sBonus);
+  if (warp == NW - 1) {
+    // GDN/KDA: k_t . q_t (the current entry's own weight on q) and, for the
+    // KLA step size, |k_t|^2; RWKV6: the bonus sum_c r_c u_c k_c.
+    float x = 0.f, kk = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) {
+      const int c = lane * CPL + cc;
+      const float kc = to_f(sKr[c]);
+      const float qc = to_f(sQr[c]);
+      x = (VAR == kVarRWKV6) ? fmaf(qc * sBonus[c], kc, x) : fmaf(kc, qc, x);
+      kk = fmaf(kc, kc, kk);
+    }
+    x = warp_sum(x);
+    if (VAR != kVarRWKV6 && p.kla) kk = warp_sum(kk);
+    if (lane == 0) {
+      sScal[0] = x;
+      sScal[1] = (VAR != kVarRWKV6 && p.kla) ? beta_s / (kk + p.kla_eps) : beta_s;  // eta -> beta
+    }
+  }
+  if (!__syncthreads_and(ok)) {
+    mbar_wait(barLog, 0, nullptr, 0);
+    for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
+    return;
+  }
+
+  // ---- one pass over this warp's 16 rows of S_b
+  const int j0 = warp * Tl::kRowsPerWarp;  // local row index
+  uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
+  const bool mine = mbar_wait(barMine, 0, p.err, int(head));
+  // the int8 fused merge synchronises the whole CTA below, so there every
+  // warp has to know whether all tile chunks arrived
+  const bool all_in = (Q8 && merge_now) ? __syncthreads_and(mine) : mine;
+  if (!all_in) {
+    mbar_wait(barMine, 0, nullptr, 0);
+    return;
+  }
+  float a, b;
+  int jl;  // local row this lane finishes
+  bool owner;  // the one lane that writes row jl
+  if constexpr (Q8) {
+    rows_gemv_q8<DK>(sS, sScale, j0, lane, sVecH, a, b, jl, owner);
+  } else {
+    rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
+                                    (VAR == kVarGDN) ? sq : sQh, a, b, jl);
+    owner = (lane & 1) == 0;
+  }
+  float u, o;
+  const float vj = (VAR == kVarGDN2) ? sWg[jl] * to_f(sVr[jl]) : to_f(sVr[jl]);
+  row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, vj, a, b, u, o);
+  if (owner) {
+    p.o[head * DV + r0 + jl] = o;
+    if (merge_now)
+      sU[su_offset(jl, f, L)] = Elem<TU>::from_f(u);
+    else
+      gU[u_offset(0, r0 + jl, f, L, DV)] = Elem<TU>::from_f(u);
+  }
+  if (!merge_now) return;
+  if constexpr (Q8) {
+    // every warp's u_t rows are in slot f; stage the decayed keys of the
+    // L entries and the base decay once for the CTA, then fold and requantize
+    __syncthreads();
+    if (GW == 1) {  // GDN: one decay factor per entry (sW's weights are no longer needed)
+      for (int e = tid; e < f; e += NT) sW[e] = expf(sGt[0] - sG[e]);
+      __syncthreads();
+    }
+    stage_kt_frags<VAR, DK, TIn>(sK, sG, sGt, sW, f, f + 1, q8_chunks(f + 1), sB, tid, NT);
+    for (int c = tid; c < DK; c += NT) sDecF[dec_pad(c)] = (GW == 1) ? sScal[2] : expf(sGt[c]);
+    __syncthreads();
+    fold_rows_q8<DK, TU, GW == 1>(sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L, j0, lane,
+                         static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
+                         p.scale + head * size_t(DV) + r0, nullptr);
+  } else {
+    __syncwarp();
+    merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,
+                                       static_cast<float*>(p.base) + (head * size_t(DV) + r0) * DK);
+  }
+}
+
+}  // namespace dl
