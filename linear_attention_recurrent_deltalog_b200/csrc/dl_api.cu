@@ -37,12 +37,15 @@ struct Layout {
 
 bool is_q8(const dl_config& c) { return (c.flags & DL_FLAG_BASE_Q8) != 0; }
 
-// Default work items per head for the step kernel (measured on B200): GDN
-// cuts a d_v = 128 head into two 64-row items; the vector-decay variants
-// (KDA, GDN-2, RWKV6), whose per-head log-decay block and entry weights every
-// item would stage again, keep one item per head (fp32 and int8 base alike).
+// Default work items per head for the step kernel (measured on B200): with
+// an fp32 base GDN cuts a d_v = 128 head into two 64-row items; the
+// vector-decay variants (KDA, GDN-2, RWKV6), whose per-head log-decay block
+// and entry weights every item would stage again, keep one item per head,
+// and so does every int8 base (a quarter of the bytes per row, so one
+// 128-row head per CTA still leaves 6 CTAs per SM and forms the per-entry
+// weights once).
 int default_split(const dl_config& c) {
-  return (c.variant == DL_GDN && c.d_v >= 128) ? 2 : 1;
+  return (c.variant == DL_GDN && c.d_v >= 128 && !is_q8(c)) ? 2 : 1;
 }
 int split_of(const dl_config& c) { return c.step_split == 0 ? default_split(c) : c.step_split; }
 
@@ -92,7 +95,9 @@ int check_config(const dl_config* c, bool need_L) {
   if (bh > 0x7fffffffull) return DL_ERR_ARG;  // one CTA per head in a 1-D grid
   if (bh * uint64_t(c->d_v) * uint64_t(c->d_k) >= (1ull << 40)) return DL_ERR_ARG;
   if (!head_size_ok(c->d_k) || !head_size_ok(c->d_v)) return DL_ERR_UNSUPPORTED;
-  if (c->step_split != 0 && !dl::split_ok(c->d_v, c->step_split)) return DL_ERR_ARG;
+  if (c->step_split != 0 &&
+      !dl::split_ok(c->d_v, c->step_split, (c->flags & DL_FLAG_BASE_Q8) != 0))
+    return DL_ERR_ARG;
   return DL_OK;
 }
 

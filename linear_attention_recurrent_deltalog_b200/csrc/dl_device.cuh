@@ -286,6 +286,28 @@ struct Tile {
   static_assert(kLPR == 2 * kNV, "row reduction layout");
 };
 
+// Step geometry of an int8 base: a warp owns 32 rows (two m16 tiles of the
+// tensor-core GEMV, which share its B fragments), so after the GEMV each of
+// its 32 lanes finishes one row; one bulk copy per warp's rows.
+template <int DK, int ROWS>
+struct TileQ8 {
+  static_assert(DK == 64 || DK == 128, "d_k in {64,128}");
+  static_assert(ROWS == 64 || ROWS == 128, "rows per CTA in {64,128}");
+  static constexpr int kWarps = ROWS / 32;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kRowsPerWarp = 32;
+  static constexpr int kChunkRows = 32;
+  static constexpr int kChunks = ROWS / kChunkRows;
+  static constexpr uint32_t kChunkBytes = kChunkRows * DK;
+  static constexpr size_t kTileBytes = size_t(ROWS) * DK;
+  static constexpr int kCPL = DK / 32;
+};
+
+// The step kernel's tile geometry for a base of element type TB.
+template <int DK, int ROWS, typename TB>
+using StepTile = typename std::conditional<std::is_same<TB, int8_t>::value, TileQ8<DK, ROWS>,
+                                           Tile<DK, ROWS, TB>>::type;
+
 // ------------------------------------------------------ int8 base rows
 //
 // A quantized base row holds d_k int8 codes and one fp32 scale per value

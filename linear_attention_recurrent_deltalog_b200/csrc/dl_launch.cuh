@@ -20,8 +20,14 @@ struct Shape {
   int split;       // step kernel: work items per head (1, 2 or 4; d_v / split >= 32)
 };
 
-inline bool split_ok(int dv, int split) {
-  return (split == 1 || split == 2 || split == 4) && dv % split == 0 && dv / split >= 32;
+// Smallest work item (rows) the step kernel is built for: 32 rows for an
+// fp32 base, 64 for an int8 base (32 rows per warp, at least two warps).
+template <typename TB>
+constexpr int kMinItemRows = std::is_same<TB, int8_t>::value ? 64 : 32;
+
+inline bool split_ok(int dv, int split, bool q8) {
+  return (split == 1 || split == 2 || split == 4) && dv % split == 0 &&
+         dv / split >= (q8 ? 64 : 32);
 }
 
 // Dynamic shared memory each kernel may use; set once per device.
@@ -53,7 +59,7 @@ cudaError_t launch_step_t(const StepParams& p, const FillParam& fp, unsigned nhe
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
   const size_t smem = StepLayout<VAR, DK, DV, ROWS, TIn, TB, FUSED>(p.L).total;
-  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p, fp);
+  kern<<<nheads * unsigned(DV / ROWS), StepTile<DK, ROWS, TB>::kThreads, smem, s>>>(p, fp);
   return cudaGetLastError();
 }
 
@@ -65,7 +71,7 @@ cudaError_t launch_merge_rows(const MergeParams& p, const SeqList& list, unsigne
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
   const size_t smem = MergeLayout<VAR, DK, DV, ROWS, TIn, TB>(p.L).total;
-  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS>::kThreads, smem, s>>>(p, list);
+  kern<<<nheads * unsigned(DV / ROWS), Tile<DK, ROWS, TB>::kThreads, smem, s>>>(p, list);
   return cudaGetLastError();
 }
 
@@ -152,10 +158,10 @@ template <int VAR, int DK, int DV, typename T, typename TB, bool FUSED>
 cudaError_t launch_step_split(int split, const StepParams& p, const FillParam& fp, unsigned n,
                               cudaStream_t s) {
   if (split == 1) return launch_step_t<VAR, DK, DV, DV, T, TB, FUSED>(p, fp, n, s);
-  if constexpr (DV / 2 >= 32) {
+  if constexpr (DV / 2 >= kMinItemRows<TB>) {
     if (split == 2) return launch_step_t<VAR, DK, DV, DV / 2, T, TB, FUSED>(p, fp, n, s);
   }
-  if constexpr (DV / 4 >= 32) {
+  if constexpr (DV / 4 >= kMinItemRows<TB>) {
     if (split == 4) return launch_step_t<VAR, DK, DV, DV / 4, T, TB, FUSED>(p, fp, n, s);
   }
   return cudaErrorInvalidValue;
@@ -201,10 +207,10 @@ struct StepSmem {
   cudaError_t run() {
     out = 0;
     if (split == 1) out = need<DK, DV, DV, T>();
-    if constexpr (DV / 2 >= 32) {
+    if constexpr (DV / 2 >= kMinItemRows<TB>) {
       if (split == 2) out = need<DK, DV, DV / 2, T>();
     }
-    if constexpr (DV / 4 >= 32) {
+    if constexpr (DV / 4 >= kMinItemRows<TB>) {
       if (split == 4) out = need<DK, DV, DV / 4, T>();
     }
     return out ? cudaSuccess : cudaErrorInvalidValue;

@@ -20,47 +20,64 @@ __host__ __device__ constexpr int q8_chunks(int L) { return (L + 15) / 16; }
 template <int DK>
 constexpr int kVecHStride = DK + 16;
 
-// Base GEMV on the tensor cores: A = the warp's 16 rows of codes, B = the
-// four fp16 vectors of sVecH [4][kVecHStride] (columns: k-hat hi, k-hat lo, q-hat hi,
-// q-hat lo; the other four columns are zero), so D's columns 0+1 hold S k-hat
-// and 2+3 hold S q-hat.  Inside each 16-channel k-step, logical k (2t, 2t+1,
-// 2t+8, 2t+9) is channel (4t .. 4t+3): A and B agree, so the dot products
-// are unchanged.  Lane 4g + t with t < 2 finishes row jl = j0 + g (t = 0) or
-// j0 + g + 8 (t = 1), scaled by its row scale; `owner` is false elsewhere.
+// Two k-steps (16 channels each) of one m16 tile of the base GEMV: A = the
+// tile's codes (ldmatrix from the swizzled tile, rows `arow` of this lane's
+// matrix), B = the shared fragments b0 / b1 of the two k-steps.
+template <int DK>
+__device__ __forceinline__ void gemv_q8_ksteps(const int8_t* sQ, int arow, int kk, int m,
+                                               uint2 b0, uint2 b1, float (&d)[4]) {
+  uint32_t w[4];
+  ldmatrix_x4(w, sQ + q8_off<DK>(arow, 16 * (kk + (m >> 1))));
+  uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
+  codes4_to_h2(w[0], a0, a2);  // row g,   channels 16 kk + 4t ..
+  codes4_to_h2(w[1], a1, a3);  // row g+8
+  codes4_to_h2(w[2], c0, c2);  // row g,   next k-step
+  codes4_to_h2(w[3], c1, c3);  // row g+8, next k-step
+  mma_16816(d, a0, a1, a2, a3, b0.x, b0.y);
+  mma_16816(d, c0, c1, c2, c3, b1.x, b1.y);
+}
+
+// Base GEMV of a warp's 32 rows j0 .. j0+31 (two m16 tiles) on the tensor
+// cores: A = the codes, B = the four fp16 vectors of sVecH [4][kVecHStride]
+// (columns: k-hat hi, k-hat lo, q-hat hi, q-hat lo; the other four columns
+// are zero), shared by both tiles, so D's columns 0+1 hold S k-hat and 2+3
+// hold S q-hat.  Inside each 16-channel k-step, logical k (2t, 2t+1, 2t+8,
+// 2t+9) is channel (4t .. 4t+3): A and B agree, so the dot products are
+// unchanged.  Three shuffles then hand every lane one finished row:
+// lane 4g + t ends with row jl = j0 + g + 8t, scaled by its row scale.
 template <int DK>
 __device__ __forceinline__ void rows_gemv_q8(const int8_t* sQ, const float* sScale, int j0, int lane,
-                                             const __half* sVecH, float& a, float& b, int& jl,
-                                             bool& owner) {
+                                             const __half* sVecH, float& a, float& b, int& jl) {
   const int g = lane >> 2;
   const int t = lane & 3;
-  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
   const int m = lane >> 3;                       // ldmatrix: which matrix this lane addresses
   const int arow = j0 + (lane & 7) + 8 * (m & 1);
 #pragma unroll
   for (int kk = 0; kk < DK / 16; kk += 2) {
-    uint32_t w[4];
-    ldmatrix_x4(w, sQ + q8_off<DK>(arow, 16 * (kk + (m >> 1))));
-    uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-    codes4_to_h2(w[0], a0, a2);  // row g,   channels 16 kk + 4t ..
-    codes4_to_h2(w[1], a1, a3);  // row g+8
-    codes4_to_h2(w[2], c0, c2);  // row g,   next k-step
-    codes4_to_h2(w[3], c1, c3);  // row g+8, next k-step
     uint2 b0 = make_uint2(0u, 0u), b1 = make_uint2(0u, 0u);
     if (g < 4) {
       b0 = *reinterpret_cast<const uint2*>(sVecH + g * kVecHStride<DK> + 16 * kk + 4 * t);
       b1 = *reinterpret_cast<const uint2*>(sVecH + g * kVecHStride<DK> + 16 * (kk + 1) + 4 * t);
     }
-    mma_16816(d, a0, a1, a2, a3, b0.x, b0.y);
-    mma_16816(d, c0, c1, c2, c3, b1.x, b1.y);
+    gemv_q8_ksteps<DK>(sQ, arow, kk, m, b0, b1, d0);
+    gemv_q8_ksteps<DK>(sQ, arow + 16, kk, m, b0, b1, d1);
   }
-  // t = 0 holds S k-hat (rows g, g+8), t = 1 holds S q-hat; trade halves
-  const float send = (t == 0) ? d[2] + d[3] : d[0] + d[1];
-  const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-  owner = t < 2;
-  jl = j0 + g + ((t == 1) ? 8 : 0);
-  const float own = (t == 1) ? d[2] + d[3] : d[0] + d[1];
-  a = (t == 0) ? own : recv;
-  b = (t == 0) ? recv : own;
+  // lane (g, t<2) holds, per tile, column pair t (t = 0: S k-hat, t = 1:
+  // S q-hat) of rows g (x) and g+8 (y); lanes t >= 2 hold zero columns.
+  // First lanes t >= 2 take tile 1's sums from lane t-2, then each pair
+  // (t even, t odd) trades halves so the even lane owns the pair's first
+  // row and the odd lane its second.
+  const float x1 = d1[0] + d1[1], y1 = d1[2] + d1[3];
+  const float rx = __shfl_xor_sync(0xffffffffu, x1, 2);
+  const float ry = __shfl_xor_sync(0xffffffffu, y1, 2);
+  const float x = (t < 2) ? d0[0] + d0[1] : rx;
+  const float y = (t < 2) ? d0[2] + d0[3] : ry;
+  const bool even = (t & 1) == 0;
+  const float recv = __shfl_xor_sync(0xffffffffu, even ? y : x, 1);
+  a = even ? x : recv;
+  b = even ? recv : y;
+  jl = j0 + g + 8 * t;
   const float sc = sScale[jl];
   a *= sc;
   b *= sc;

@@ -33,7 +33,7 @@ struct StepLayout {
   size_t offU, offK, offG, offQr, offKr, offVr, offDecV, offVec, offW, offZ, offScal, offBonus,
       offWg, offScale, offVecH, offDecF, offKt, offBar, total;
   __host__ __device__ explicit StepLayout(int L) {
-    offU = Tile<DK, ROWS, TB>::kTileBytes;
+    offU = StepTile<DK, ROWS, TB>::kTileBytes;
     offK = offU + align_up(size_t(L) * ROWS * sizeof(TU), 128);
     offG = offK + align_up(size_t(L) * DK * sizeof(TIn), 128);
     offQr = offG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128);
@@ -57,24 +57,22 @@ struct StepLayout {
     offDecF = offVecH + (Q8 ? align_up(size_t(4) * kVecHStride<DK> * 2, 128) : 0);
     offKt = offDecF + ((Q8 && FUSED) ? align_up(size_t(kDecPadLen<DK>) * 4, 128) : 0);
     offBar = offKt + ((Q8 && FUSED) ? size_t(q8_chunks(L)) * DK * 64 : 0);
-    total = offBar + 8 * (Tile<DK, ROWS, TB>::kChunks + 1);
+    total = offBar + 8 * (StepTile<DK, ROWS, TB>::kChunks + 1);
   }
 };
 
-// Resident CTAs per SM the int8 kernels are compiled for: the plain step
-// 1152 threads per SM (56 registers a thread), the step with the fused merge
-// and the merge 768 (80 registers; the fold's accumulators may spill a
-// little), so the rare fold does not set the occupancy of every step.  The
-// fp32 kernels keep the compiler's choice.
+// Resident threads per SM the int8 step is compiled for: 768 (up to 85
+// registers a thread), which the ~34 KB of shared memory of a 128-row head
+// allows anyway; the fold of the fused merge runs one 16-row tile at a time
+// so it needs no more.  The fp32 kernels keep the compiler's choice.
 template <typename TB, int THREADS, bool FOLDS>
-constexpr int kMinBlocks =
-    std::is_same<TB, int8_t>::value ? (FOLDS ? 768 : 1152) / THREADS : 1;
+constexpr int kMinBlocks = std::is_same<TB, int8_t>::value ? 768 / THREADS : 1;
 
 template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB, bool FUSED>
-__global__ void __launch_bounds__(Tile<DK, ROWS, TB>::kThreads,
-                                  kMinBlocks<TB, Tile<DK, ROWS, TB>::kThreads, FUSED>)
+__global__ void __launch_bounds__(StepTile<DK, ROWS, TB>::kThreads,
+                                  kMinBlocks<TB, StepTile<DK, ROWS, TB>::kThreads, FUSED>)
 dl_step_kernel(const StepParams p, const FillParam fp) {
-  using Tl = Tile<DK, ROWS, TB>;
+  using Tl = StepTile<DK, ROWS, TB>;
   using TU = typename LogU<VAR, TIn>::type;
   constexpr bool Q8 = std::is_same<TB, int8_t>::value;
   constexpr int SPLIT = DV / ROWS;
@@ -264,7 +262,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     return;
   }
 
-  // ---- one pass over this warp's 16 rows of S_b
+  // ---- one pass over this warp's rows of S_b (16 fp32 rows, or 32 int8 rows)
   const int j0 = warp * Tl::kRowsPerWarp;  // local row index
   uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
   const bool mine = mbar_wait(barMine, 0, p.err, int(head));
@@ -277,9 +275,9 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   }
   float a, b;
   int jl;  // local row this lane finishes
-  bool owner;  // the one lane that writes row jl
+  bool owner = true;  // the one lane that writes row jl (every lane for an int8 base)
   if constexpr (Q8) {
-    rows_gemv_q8<DK>(sS, sScale, j0, lane, sVecH, a, b, jl, owner);
+    rows_gemv_q8<DK>(sS, sScale, j0, lane, sVecH, a, b, jl);
   } else {
     rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
                                     (VAR == kVarGDN) ? sq : sQh, a, b, jl);
@@ -307,9 +305,12 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
     stage_kt_frags<VAR, DK, TIn>(sK, sG, sGt, sW, f, f + 1, q8_chunks(f + 1), sB, tid, NT);
     for (int c = tid; c < DK; c += NT) sDecF[dec_pad(c)] = (GW == 1) ? sScal[2] : expf(sGt[c]);
     __syncthreads();
-    fold_rows_q8<DK, TU, GW == 1>(sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L, j0, lane,
-                         static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
-                         p.scale + head * size_t(DV) + r0, nullptr);
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half)  // the warp's two 16-row tiles, one at a time
+      fold_rows_q8<DK, TU, GW == 1>(sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L,
+                                    j0 + 16 * half, lane,
+                                    static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
+                                    p.scale + head * size_t(DV) + r0, nullptr);
   } else {
     __syncwarp();
     merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,

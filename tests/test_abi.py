@@ -80,6 +80,9 @@ def test_state_bytes_layout():
     (dict(step_split=3), dlb.DL_ERR_ARG),
     (dict(step_split=4, d_v=64), dlb.DL_ERR_ARG),
     (dict(step_split=8), dlb.DL_ERR_ARG),
+    # an int8 base needs work items of at least 64 rows
+    (dict(step_split=4, base="q8"), dlb.DL_ERR_ARG),
+    (dict(step_split=2, d_v=64, base="q8"), dlb.DL_ERR_ARG),
 ])
 def test_state_bytes_rejects(bad, code):
     with pytest.raises(dlb.DeltaLogError) as e:

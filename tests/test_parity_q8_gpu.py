@@ -62,7 +62,7 @@ def test_q8_workloads(name, fused):
 
 def test_q8_serving_full_batch():
     # the benchmarked launch: B=512 H=32 d=128 L=16, ragged fills, fused
-    # merge, 64-row work items; more than two windows per sequence
+    # merge, one 128-row work item per head; more than two windows per sequence
     w = wl.WORKLOADS["gdn_serving"]
     heads = heads_covering_phases(w, 24)
     r = run_parity_q8(w, T=40, heads=heads, fused=True, snap_every=10, workers=None)
@@ -76,8 +76,8 @@ def test_q8_serving_full_batch():
     ("gdn2", 64, 128, "bf16"), ("gdn2", 128, 128, "f32"),
 ])
 def test_q8_shapes_dtypes_splits(variant, dk, dv, dtype, split):
-    if dv // split < 32:
-        pytest.skip("work items hold at least 32 rows")
+    if dv // split < 64:
+        pytest.skip("int8 work items hold at least 64 rows (32 per warp, two warps)")
     base = {"gdn": "gdn_qwen", "kda": "kda", "rwkv6": "rwkv6", "gdn2": "gdn2"}[variant]
     w = wl.WORKLOADS[base].replace(B=6, H=3, d_k=dk, d_v=dv, in_dtype=dtype, L=5, ragged=True,
                                    seed=31 + split)
