@@ -235,17 +235,23 @@ struct WarpRows {
   static constexpr int NV = 16 / RPI;
 };
 
+// Key column of the first of the four columns lane `lane` covers.
+template <int DK>
+__device__ __forceinline__ int gemv_col(int lane) {
+  return (lane % WarpRows<DK>::LPR) * 4;
+}
+
 // Row sums a_j = S_j . va and b_j = S_j . vb over the warp's rows in one pass
-// (a skipped unless WITH_A); returns them for the row `jl` this lane ends up
-// owning after the butterfly (lanes l and l^1 own the same row).
+// (a skipped unless WITH_A), given this lane's four columns of each vector
+// (a4 = va[gemv_col(lane) .. +3], likewise b4); returns them for the row
+// `jl` this lane ends up owning after the butterfly (lanes l and l^1 own the
+// same row).
 template <int DK, bool WITH_A>
-__device__ __forceinline__ void rows_gemv(const float* sS, int j0, int lane, const float* va,
-                                          const float* vb, float& a, float& b, int& jl) {
+__device__ __forceinline__ void rows_gemv4(const float* sS, int j0, int lane, float4 a4, float4 b4,
+                                           float& a, float& b, int& jl) {
   using G = WarpRows<DK>;
-  const int c0 = (lane % G::LPR) * 4;
+  const int c0 = gemv_col<DK>(lane);
   const int rsub = lane / G::LPR;
-  const float4 a4 = WITH_A ? *reinterpret_cast<const float4*>(va + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4 b4 = *reinterpret_cast<const float4*>(vb + c0);
   float pa[G::NV], pb[G::NV];
 #pragma unroll
   for (int pi = 0; pi < G::NV; ++pi) {
@@ -256,6 +262,15 @@ __device__ __forceinline__ void rows_gemv(const float* sS, int j0, int lane, con
   a = WITH_A ? reduce_rows<G::NV, G::LPR>(pa, lane) : 0.f;
   b = reduce_rows<G::NV, G::LPR>(pb, lane);
   jl = j0 + reduced_index<G::NV, G::LPR>(lane) * G::RPI + rsub;
+}
+
+// The same with va, vb read from shared memory (fp32 or bf16).
+template <int DK, bool WITH_A, typename TV>
+__device__ __forceinline__ void rows_gemv(const float* sS, int j0, int lane, const TV* va,
+                                          const TV* vb, float& a, float& b, int& jl) {
+  const int c0 = gemv_col<DK>(lane);
+  const float4 a4 = WITH_A ? load4(va + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+  rows_gemv4<DK, WITH_A>(sS, j0, lane, a4, load4(vb + c0), a, b, jl);
 }
 
 // The step's correction and readout for one row, given its base sums a, b:

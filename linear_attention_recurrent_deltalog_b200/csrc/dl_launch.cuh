@@ -75,11 +75,71 @@ cudaError_t launch_merge_rows(const MergeParams& p, const SeqList& list, unsigne
   return cudaGetLastError();
 }
 
+// SMs of the current device (cached per device).
+inline int sm_count() {
+  static std::atomic<int> cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+// CTAs of `kern` (threads, dynamic shared memory smem) that fit on one SM at
+// once, from its registers and shared memory, at most `cap`; 0 on error.
+template <typename Kern>
+inline int resident_ctas(Kern kern, int threads, size_t smem, int cap) {
+  int dev = 0, smem_sm = 0, reserved = 0, regs_sm = 0, threads_sm = 0;
+  cudaFuncAttributes fa{};
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) != cudaSuccess)
+    return 0;
+  const int warps = (threads + 31) / 32;
+  const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;  // allocation unit: 256 registers
+  int n = cap;
+  const int by_smem = int(size_t(smem_sm) / (smem + size_t(fa.sharedSizeBytes) + size_t(reserved)));
+  const int by_regs = regs_warp > 0 ? regs_sm / (regs_warp * warps) : n;
+  const int by_threads = threads_sm / (warps * 32);
+  n = by_smem < n ? by_smem : n;
+  n = by_regs < n ? by_regs : n;
+  n = by_threads < n ? by_threads : n;
+  return n;
+}
+
+// The int8 merge of d_v = 128 heads on TMEM: a persistent launch of as many
+// 288-thread CTAs as fit on the SMs (its shared memory keeps that at most
+// 512 / d_k per SM), each walking the listed heads.
+template <int VAR, int DK, typename TIn>
+cudaError_t launch_merge_q8_tmem(const MergeParams& p, const SeqList& list, unsigned nheads,
+                                 cudaStream_t s) {
+  static std::atomic<unsigned long long> done{0};
+  auto kern = dl_merge_q8_kernel<VAR, DK, TIn>;
+  cudaError_t e = prepare_kernel(kern, done);
+  if (e != cudaSuccess) return e;
+  const size_t smem = MergePipeLayout<VAR, DK, TIn>(p.L).total;
+  const int per_sm = resident_ctas(kern, kMergePipeThreads, smem, 512 / DK);
+  const int sms = sm_count();
+  if (per_sm <= 0 || sms <= 0) return cudaErrorInvalidConfiguration;
+  const unsigned cap = unsigned(per_sm) * unsigned(sms);
+  const unsigned grid = nheads < cap ? nheads : cap;
+  if (grid == 0) return cudaSuccess;
+  kern<<<grid, kMergePipeThreads, smem, s>>>(p, list, nheads);
+  return cudaGetLastError();
+}
+
 // Split heads into 64-row CTAs whenever no CTA has to read a fill another
-// CTA of the launch may reset (a listed merge, or materialize).
+// CTA of the launch may reset (a listed merge, or materialize).  An int8
+// base with d_v = 128 folds on TMEM, one CTA per head.
 template <int VAR, int DK, int DV, typename TIn, typename TB>
 cudaError_t launch_merge_t(const MergeParams& p, const SeqList& list, unsigned nheads,
                            cudaStream_t s) {
+  if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows)
+    return launch_merge_q8_tmem<VAR, DK, TIn>(p, list, nheads, s);
   if constexpr (DV >= 128) {
     if (p.use_list || p.mode == 2)
       return launch_merge_rows<VAR, DK, DV, DV / 2, TIn, TB>(p, list, nheads, s);
@@ -226,7 +286,10 @@ struct MergeSmem {
   size_t out;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    out = MergeLayout<VAR, DK, DV, DV, T, TB>(L).total;
+    if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows)
+      out = MergePipeLayout<VAR, DK, T>(L).total;
+    else
+      out = MergeLayout<VAR, DK, DV, DV, T, TB>(L).total;
     return cudaSuccess;
   }
 };

@@ -3,6 +3,7 @@
 
 #include "dl_common.cuh"
 #include "dl_q8.cuh"
+#include "dl_fold_tmem.cuh"
 
 namespace dl {
 
@@ -195,6 +196,224 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
 #pragma unroll
   for (int pi = 0; pi < NV; ++pi)
     *reinterpret_cast<float4*>(gO + size_t(j0 + pi * RPI + rsub) * DK + c0) = acc[pi];
+}
+
+// ------------------------------------- int8 merge / materialize on TMEM
+//
+// d_v = 128 heads of an int8 base, as a pipelined persistent kernel: each
+// CTA walks the heads blockIdx.x, blockIdx.x + gridDim.x, ...  A producer
+// warp streams the next head's codes, row scales and log entries into one of
+// two shared-memory stages while eight consumer warps fold the current head:
+// thread i of consumer warp w owns row 32 (w mod 4) + i and half of its key
+// channels.  The fold D = deq(codes) Diag(dec) + U Kt accumulates in tensor
+// memory (dl_fold_tmem.cuh), allocated once per CTA; the requantize (merge)
+// or the fp32 write (materialize) reads each row straight from TMEM.
+
+constexpr int kFoldThreads = 2 * kFoldRows;       // consumer threads
+constexpr int kMergePipeThreads = kFoldThreads + 32;  // plus the producer warp
+constexpr int kConsumerBar = 1;                   // named barrier of the consumers
+
+template <int VAR, int DK, typename TIn>
+struct MergePipeLayout {
+  using TU = typename LogU<VAR, TIn>::type;
+  // inside a stage (codes at 0)
+  size_t inU, inK, inG, inScale, stage;
+  size_t offA, offB, offDec, offMeta, offTmem, offBar, total;
+  __host__ __device__ explicit MergePipeLayout(int L) {
+    const size_t nch = size_t(q8_chunks(L));
+    inU = size_t(kFoldRows) * DK;                                    // codes [128][DK]
+    inK = inU + align_up(size_t(L) * kFoldRows * sizeof(TU), 128);   // u [4][L][32]
+    inG = inK + align_up(size_t(L) * DK * sizeof(TIn), 128);         // k [L][DK]
+    inScale = inG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128); // g
+    stage = inScale + align_up(size_t(kFoldRows) * 4, 128);          // row scales
+    offA = 2 * stage;                                                // A hi, lo (then row maxima)
+    offB = offA + 2 * nch * kFoldAStep;                              // B hi, lo
+    offDec = offB + 2 * nch * kFoldBStep<DK>;                        // decay, GDN factors
+    offMeta = offDec + align_up(size_t(kDecPadLen<DK> + 64) * 4, 128);
+    offTmem = offMeta + 32;
+    offBar = offTmem + 16;
+    const size_t need = offBar + 8 * 5;  // full[2], empty[2], mma
+    // at most 512 / DK CTAs per SM, so every CTA's TMEM allocation succeeds
+    // at once (228 KB of shared memory per SM, 1 KB reserved per CTA)
+    const size_t floor_bytes = (DK == 128) ? 49152 : 26624;
+    total = need > floor_bytes ? need : floor_bytes;
+  }
+};
+
+// What the producer tells the consumers about the head in a stage.
+struct MergeItem {
+  unsigned long long head;
+  int f;
+  int skip;  // nothing to fold (mode's filter) or an invalid fill
+};
+
+template <int VAR, int DK, typename TIn>
+__global__ void __launch_bounds__(kMergePipeThreads, 3)
+dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
+  using TU = typename LogU<VAR, TIn>::type;
+  constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
+  constexpr int DV = kFoldRows;
+  constexpr int NCOL = DK / 2;  // key channels per consumer thread
+  constexpr uint32_t kChunk = 32 * DK;  // codes of 32 rows
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int L = p.L;
+  const int GS = g_stride(VAR, L, DK);
+  const MergePipeLayout<VAR, DK, TIn> lay(L);
+  unsigned char* sA = smem + lay.offA;
+  unsigned char* sB = smem + lay.offB;
+  float* sAmax = reinterpret_cast<float*>(sA);                 // after the MMA: row maxima
+  float* sDec = reinterpret_cast<float*>(smem + lay.offDec);   // base decay at dec_pad indices
+  float* sFac = sDec + kDecPadLen<DK>;                           // GDN: e^{g_last - g_i}
+  MergeItem* sMeta = reinterpret_cast<MergeItem*>(smem + lay.offMeta);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + lay.offTmem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.offBar);
+  uint64_t* empty = full + 2;
+  uint64_t* barMma = full + 4;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(barMma, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(sTmem, DK);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+
+  if (warp == kFoldThreads / 32) {
+    // ---- producer: one lane issues every copy
+    if (lane == 0) {
+      for (unsigned j = 0;; ++j) {
+        const unsigned it = blockIdx.x + j * gridDim.x;
+        if (it >= nitems) break;
+        const int s = int(j & 1);
+        if (j >= 2 && !mbar_wait(&empty[s], ((j - 2) >> 1) & 1, p.err, -1)) break;
+        const unsigned li = it / unsigned(p.H);
+        const size_t head = p.use_list ? size_t(list.seq[li]) * size_t(p.H) + it % unsigned(p.H)
+                                       : size_t(it);
+        const int f = p.use_list ? int(list.f[li]) : p.fill[head];
+        int skip = 0;
+        if (f < 0 || f > L) {
+          if (p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
+          skip = 1;
+        } else if ((p.mode == 0 && f != L) || (p.mode == 1 && f == 0)) {
+          skip = 1;
+        }
+        sMeta[s] = MergeItem{head, f, skip};
+        if (skip) {
+          mbar_arrive(&full[s]);
+          continue;
+        }
+        unsigned char* st = smem + size_t(s) * lay.stage;
+        const uint32_t bu = uint32_t(f) * kURows * sizeof(TU);  // one 32-row block
+        const uint32_t bk = uint32_t(f) * DK * sizeof(TIn);
+        const uint32_t bg = f > 0 ? g_copy_bytes<VAR, DK>(f) : 0u;
+        const uint32_t bs = DV * 4u;
+        mbar_arrive_expect_tx(&full[s], 4 * kChunk + bu * uint32_t(DV / kURows) + bk + bg + bs);
+        const int8_t* gQ = static_cast<const int8_t*>(p.base) + head * size_t(DV) * DK;
+        for (int c = 0; c < 4; ++c)
+          tma_load_1d_stream(st + size_t(c) * kChunk, gQ + size_t(c) * kChunk, kChunk, &full[s]);
+        tma_load_1d(st + lay.inScale, p.scale + head * DV, bs, &full[s]);
+        if (f > 0) {
+          const TU* gU = static_cast<const TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
+          for (int rb = 0; rb < DV / kURows; ++rb)
+            tma_load_1d(st + lay.inU + size_t(rb) * L * kURows * sizeof(TU),
+                        gU + u_offset(0, rb * kURows, 0, L, DV), bu, &full[s]);
+          tma_load_1d(st + lay.inK, static_cast<const TIn*>(p.logK) + head * size_t(L) * DK, bk,
+                      &full[s]);
+          tma_load_1d(st + lay.inG, p.logG + head * size_t(GS), bg, &full[s]);
+        }
+      }
+    }
+  } else {
+    // ---- consumers
+    const int row = 32 * (warp & 3) + lane;  // this thread's value row
+    const int half = warp >> 2;              // which half of the row's channels
+    const int c0 = half * NCOL;
+    const uint32_t lane_addr = tmem_warp_addr(tmem, warp, 0);
+    uint32_t mma_phase = 0;
+    for (unsigned j = 0;; ++j) {
+      const unsigned it = blockIdx.x + j * gridDim.x;
+      if (it >= nitems) break;
+      const int s = int(j & 1);
+      if (!named_bar_and(kConsumerBar, kFoldThreads, mbar_wait(&full[s], (j >> 1) & 1, p.err, -1)))
+        break;
+      tc_fence_after();
+      const MergeItem m = sMeta[s];
+      if (!m.skip) {
+        const size_t head = size_t(m.head);
+        const int f = m.f;
+        const unsigned char* st = smem + size_t(s) * lay.stage;
+        const int8_t* sQ = reinterpret_cast<const int8_t*>(st);
+        const TU* sU = reinterpret_cast<const TU*>(st + lay.inU);
+        const TIn* sK = reinterpret_cast<const TIn*>(st + lay.inK);
+        const float* sG = reinterpret_cast<const float*>(st + lay.inG);
+        const float* sScale = reinterpret_cast<const float*>(st + lay.inScale);
+        for (int c = tid; c < DK; c += kFoldThreads)
+          sDec[dec_pad(c)] = expf((f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f);
+        if (GW == 1)
+          for (int e = tid; e < f; e += kFoldThreads) sFac[e] = expf(sG[f - 1] - sG[e]);
+        named_bar_sync(kConsumerBar, kFoldThreads);
+        const int nch = q8_chunks(f);
+        if (f > 0) {
+          if (tid < kFoldRows)  // A: one row per thread of the first four warps
+            stage_fold_a<TU>(sU, f, nch, L, sA, tid);
+          else                  // B: the other four warps
+            stage_fold_b<VAR, DK, TIn>(sK, sG, sG + size_t(f - 1) * GW, sFac, f, f, nch, sB,
+                                       tid - kFoldRows, kFoldThreads - kFoldRows);
+          fence_async_smem();
+        }
+        // D = the dequantized, decayed base rows
+        fold_init_q8<DK, NCOL, GW == 1>(sQ, sScale[row], sDec, row, c0, lane_addr);
+        tmem_wait_st();
+        tc_fence_before();
+        named_bar_sync(kConsumerBar, kFoldThreads);
+        if (nch > 0) {
+          if (tid == 0) {
+            tc_fence_after();
+            fold_issue<DK>(tmem, sA, sB, nch, barMma);
+          }
+          const bool done = named_bar_and(kConsumerBar, kFoldThreads,
+                                          mbar_wait(barMma, mma_phase, p.err, int(head)));
+          mma_phase ^= 1u;
+          tc_fence_after();
+          if (!done) break;
+        }
+        if (p.mode == 2) {
+          fold_store_f32<NCOL>(lane_addr, c0, p.out + (head * size_t(DV) + row) * DK);
+        } else {
+          sAmax[half * kFoldRows + row] = fold_amax<NCOL>(lane_addr, c0);
+          named_bar_sync(kConsumerBar, kFoldThreads);
+          const float amax = fmaxf(sAmax[row], sAmax[kFoldRows + row]);
+          const bool live = amax >= kTinyAmax;
+          const float inv = live ? __fdiv_rn(127.0f, amax) : 0.f;
+          fold_store_q8<DK, NCOL>(lane_addr, c0, row, inv,
+                                  static_cast<int8_t*>(p.base) + head * size_t(DV) * DK);
+          if (!half) p.scale[head * size_t(DV) + row] = live ? __fdiv_rn(amax, 127.0f) : 0.f;
+          // the log is emptied only once the merged rows are written
+          if (tid == 0) p.fill[head] = 0;
+        }
+        tc_fence_before();
+      }
+      // stage s, the operand buffers and TMEM are free again
+      named_bar_sync(kConsumerBar, kFoldThreads);
+      if (tid == 0) mbar_arrive(&empty[s]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, DK);
 }
 
 }  // namespace dl

@@ -121,6 +121,8 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   const int part = static_cast<int>(blockIdx.x % SPLIT);
   const int r0 = part * ROWS;  // first value row of this CTA
   const int h = static_cast<int>(head % static_cast<size_t>(p.H));
+  const TB* gS = static_cast<const TB*>(p.base) + (head * size_t(DV) + r0) * DK;
+
   const int f = step_fill(p, fp, head);
   if (f < 0 || f >= L) {  // the host never launches a step on a full log
     if (tid == 0 && p.err != nullptr && atomicCAS(p.err, 0, kDevErrFill) == 0) p.err[1] = int(head);
@@ -129,7 +131,6 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   const bool merge_now = FUSED && (f + 1 == L);
   const bool appender = (part == 0) && !merge_now;
 
-  const TB* gS = static_cast<const TB*>(p.base) + (head * size_t(DV) + r0) * DK;
   TU* gU = static_cast<TU*>(p.logU) + u_offset(head, 0, 0, L, DV);
   TIn* gK = static_cast<TIn*>(p.logK) + head * size_t(L) * DK;
   float* gG = p.logG + head * size_t(GS);
@@ -137,7 +138,9 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   // Warp 0 streams the tile; warp 1 fetches everything small (the step's
   // vectors and the f log entries).  Each thread reads the two per-head
   // scalars no bulk copy can carry (GDN's decay, beta) into registers, so
-  // no barrier waits on those loads.
+  // no barrier waits on those loads.  (Issuing the tile before the fill is
+  // read measured slower: the log copies, which gate the entry weights,
+  // then queue behind it.)
   const float dec_s = (GW == 1) ? __ldg(p.decay + head) : 0.f;
   const float beta_s = (VAR == kVarRWKV6 || VAR == kVarGDN2) ? 0.f : __ldg(p.beta + head);
   if (warp == 0 && lane == 0) {
@@ -256,33 +259,44 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
       sScal[1] = (VAR != kVarRWKV6 && p.kla) ? beta_s / (kk + p.kla_eps) : beta_s;  // eta -> beta
     }
   }
-  if (!__syncthreads_and(ok)) {
+  // ---- one pass over this warp's rows of S_b (16 fp32 rows, or 32 int8 rows).
+  // GDN's GEMV vectors are k_t and q_t as given, so with an fp32 base each
+  // warp forms S_b k and S_b q as soon as its rows land, before the barrier
+  // that publishes the other warps' entry weights (about 1 % faster on
+  // B200).  The vector-decay variants' GEMV vectors need the decay
+  // bookkeeping first; forming their columns per lane instead measured
+  // slower, so they wait for the barrier.
+  constexpr bool kEarlyGemv = (VAR == kVarGDN) && !Q8;
+  const int j0 = warp * Tl::kRowsPerWarp;  // local row index
+  uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
+  float a = 0.f, b = 0.f;
+  int jl = 0;  // local row this lane finishes
+  bool early_in = true;
+  if constexpr (kEarlyGemv) {
+    early_in = mbar_wait(barMine, 0, p.err, int(head));
+    if (early_in && ok) rows_gemv<DK, true>(sS, j0, lane, sKr, sQr, a, b, jl);
+  }
+  if (!__syncthreads_and(ok && early_in)) {
     mbar_wait(barLog, 0, nullptr, 0);
     for (int c = 0; c < Tl::kChunks; ++c) mbar_wait(&bars[c], 0, nullptr, 0);
     return;
   }
-
-  // ---- one pass over this warp's rows of S_b (16 fp32 rows, or 32 int8 rows)
-  const int j0 = warp * Tl::kRowsPerWarp;  // local row index
-  uint64_t* barMine = &bars[j0 / Tl::kChunkRows];
-  const bool mine = mbar_wait(barMine, 0, p.err, int(head));
-  // the int8 fused merge synchronises the whole CTA below, so there every
-  // warp has to know whether all tile chunks arrived
-  const bool all_in = (Q8 && merge_now) ? __syncthreads_and(mine) : mine;
-  if (!all_in) {
-    mbar_wait(barMine, 0, nullptr, 0);
-    return;
-  }
-  float a, b;
-  int jl;  // local row this lane finishes
   bool owner = true;  // the one lane that writes row jl (every lane for an int8 base)
-  if constexpr (Q8) {
-    rows_gemv_q8<DK>(sS, sScale, j0, lane, sVecH, a, b, jl);
-  } else {
-    rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, (VAR == kVarGDN) ? sk : sKh,
-                                    (VAR == kVarGDN) ? sq : sQh, a, b, jl);
-    owner = (lane & 1) == 0;
+  if constexpr (!kEarlyGemv) {
+    const bool mine = mbar_wait(barMine, 0, p.err, int(head));
+    // the int8 fused merge synchronises the whole CTA below, so there every
+    // warp has to know whether all tile chunks arrived
+    const bool all_in = (Q8 && merge_now) ? __syncthreads_and(mine) : mine;
+    if (!all_in) {
+      mbar_wait(barMine, 0, nullptr, 0);
+      return;
+    }
+    if constexpr (Q8)
+      rows_gemv_q8<DK>(sS, sScale, j0, lane, sVecH, a, b, jl);
+    else
+      rows_gemv<DK, VAR != kVarRWKV6>(sS, j0, lane, sKh, sQh, a, b, jl);
   }
+  if constexpr (!Q8) owner = (lane & 1) == 0;
   float u, o;
   const float vj = (VAR == kVarGDN2) ? sWg[jl] * to_f(sVr[jl]) : to_f(sVr[jl]);
   row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, vj, a, b, u, o);
