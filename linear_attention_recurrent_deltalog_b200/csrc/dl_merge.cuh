@@ -384,8 +384,11 @@ dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
             tc_fence_after();
             fold_issue<DK>(tmem, sA, sB, nch, barMma);
           }
-          const bool done = named_bar_and(kConsumerBar, kFoldThreads,
-                                          mbar_wait(barMma, mma_phase, p.err, int(head)));
+          // one thread polls the MMA's completion; the others sleep in the
+          // named barrier and order their TMEM reads after it with the fence
+          const bool done = named_bar_and(
+              kConsumerBar, kFoldThreads,
+              (tid == 0) ? mbar_wait(barMma, mma_phase, p.err, int(head)) : true);
           mma_phase ^= 1u;
           tc_fence_after();
           if (!done) break;

@@ -93,6 +93,15 @@ __host__ __device__ constexpr int fold_channel(int n, int j) {
   return (DK / 4) * (j >> 1) + 2 * n + (j & 1);
 }
 
+// The fp32 fold's order: lane 4g + t owns the channels 16 q + 4 t .. +3
+// (q = 0 .. DK/16 - 1) of its two rows, so the four lanes of a row read and
+// write 64 contiguous bytes at a time (fewer shared-memory bank conflicts on
+// an unswizzled fp32 tile than DK/4 contiguous channels per lane).
+template <int DK>
+__host__ __device__ constexpr int fold_channel_il(int n, int j) {
+  return 16 * (n >> 1) + 4 * (j >> 1) + 2 * (n & 1) + (j & 1);
+}
+
 // Slot of lane l's 16-byte B fragment for n-tile n in the staged array: the
 // lane index is XOR-ed with n mod 8, which leaves the fold's loads (one
 // n-tile, 32 lanes) conflict-free and spreads the staging stores over all
@@ -111,7 +120,10 @@ __host__ __device__ constexpr int kt_slot(int kc, int ntiles, int n, int l) {
 // them.  GDN's decay is one factor per entry, from sFac (filled by the
 // caller); the vector decays take it per channel.  All threads of the CTA
 // take part; the caller synchronises afterwards.
-template <int VAR, int DK, typename TIn>
+//
+// INTERLEAVED selects the channel order of an fp32 fold (fold_channel_il)
+// instead of fold_channel's.
+template <int VAR, int DK, typename TIn, bool INTERLEAVED = false>
 __device__ __forceinline__ void stage_kt_frags(const TIn* sK, const float* sG, const float* gLast,
                                                const float* sFac, int nlog, int nent, int nchunks,
                                                uint32_t* sB, int tid, int nt) {
@@ -120,9 +132,10 @@ __device__ __forceinline__ void stage_kt_frags(const TIn* sK, const float* sG, c
   for (int idx = tid; idx < nchunks * DK; idx += nt) {
     const int c = idx % DK;
     const int kc = idx / DK;
-    // inverse of fold_channel: c = CPL (j / 2) + 2 n + (j mod 2)
-    const int n = (c % CPL) >> 1;
-    const int j = 2 * (c / CPL) + (c & 1);
+    // inverse of fold_channel: c = CPL (j / 2) + 2 n + (j mod 2); of
+    // fold_channel_il: c = 16 (n / 2) + 4 (j / 2) + 2 (n mod 2) + (j mod 2)
+    const int n = INTERLEAVED ? 2 * (c >> 4) + ((c >> 1) & 1) : (c % CPL) >> 1;
+    const int j = INTERLEAVED ? 2 * ((c >> 2) & 3) + (c & 1) : 2 * (c / CPL) + (c & 1);
     float x[16];
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
@@ -151,6 +164,105 @@ __device__ __forceinline__ void stage_kt_frags(const TIn* sK, const float* sG, c
 __host__ __device__ constexpr int dec_pad(int c) { return c + ((c >> 5) << 2); }
 template <int DK>
 constexpr int kDecPadLen = DK + DK / 8;
+
+// acc += U Kt for the warp's 16 rows j0 .. j0+15 on the tensor cores:
+// U = the rows' u values for entries 0 .. nent-1 (zero beyond), split hi/lo
+// into A fragments in registers; Kt = the staged B fragments (stage_kt_frags)
+// of nchunks 16-entry chunks, each product formed as hi*hi + hi*lo + lo*hi.
+// Lane 4g + t holds rows j0+g and j0+g+8 over the key channels
+// [DK/4 t, DK/4 (t+1)) (fold_channel): acc[n][0..1] row g, channels
+// DK/4 t + 2n, +1; acc[n][2..3] the same of row g+8.
+template <int DK, typename TU>
+__device__ __forceinline__ void fold_mma_acc(float (&acc)[DK / 8][4], const TU* sU,
+                                             const uint32_t* sB, int nent, int nchunks, int L,
+                                             int j0, int lane) {
+  constexpr int NTILE = DK / 8;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int rows[2] = {j0 + g, j0 + g + 8};
+  const uint4* sB4 = reinterpret_cast<const uint4*>(sB);
+  for (int kc = 0; kc < nchunks; ++kc) {
+    const int e0 = 16 * kc + 2 * t;
+    float u[8];  // (g, e0), (g, e0+1), (g+8, e0), (g+8, e0+1), then the same at e0+8
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = e0 + (q & 1) + ((q & 4) ? 8 : 0);
+      u[q] = (e < nent) ? to_f(sU[su_offset(rows[(q >> 1) & 1], e, L)]) : 0.f;
+    }
+    uint32_t ah[4], al[4];
+    split_h2(u[0], u[1], ah[0], al[0]);  // a0: row g,   k 2t..
+    split_h2(u[2], u[3], ah[1], al[1]);  // a1: row g+8
+    split_h2(u[4], u[5], ah[2], al[2]);  // a2: row g,   k 2t+8..
+    split_h2(u[6], u[7], ah[3], al[3]);  // a3: row g+8
+#pragma unroll
+    for (int n = 0; n < NTILE; ++n) {
+      const uint4 bf = sB4[kt_slot(kc, NTILE, n, lane)];
+      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.x, bf.y);
+      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.z, bf.w);
+      mma_16816(acc[n], al[0], al[1], al[2], al[3], bf.x, bf.y);
+    }
+  }
+}
+
+// Writes the accumulators of fold_mma_acc as fp32 rows j0+g, j0+g+8 of
+// gOut (row-major, DK per row): 16-byte stores of DK/4 contiguous channels.
+template <int DK>
+__device__ __forceinline__ void fold_acc_store_f32(const float (&acc)[DK / 8][4], int j0, int lane,
+                                                   float* gOut) {
+  constexpr int WORDS = DK / 16;
+  const int g = lane >> 2;
+  const int cbase = (DK / 4) * (lane & 3);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float4* o = reinterpret_cast<float4*>(gOut + size_t(j0 + g + 8 * half) * DK + cbase);
+#pragma unroll
+    for (int v = 0; v < WORDS; ++v)
+      o[v] = make_float4(acc[2 * v][2 * half], acc[2 * v][2 * half + 1], acc[2 * v + 1][2 * half],
+                         acc[2 * v + 1][2 * half + 1]);
+  }
+}
+
+// The fp32 fold's accumulators (fold_channel_il order) from the warp's
+// staged fp32 rows j0+g, j0+g+8 of sS, times the base decay: one factor
+// `gamma` for every channel (SDEC), else e^{sGt[c]} per channel.
+template <int DK, bool SDEC>
+__device__ __forceinline__ void fold_init_f32(float (&acc)[DK / 8][4], const float* sS,
+                                              const float* sGt, float gamma, int j0, int lane) {
+  const int g = lane >> 2;
+  const int t = lane & 3;
+#pragma unroll
+  for (int q = 0; q < DK / 16; ++q) {
+    const int c = 16 * q + 4 * t;
+    float4 d = make_float4(gamma, gamma, gamma, gamma);
+    if (!SDEC) d = make_float4(expf(sGt[c]), expf(sGt[c + 1]), expf(sGt[c + 2]), expf(sGt[c + 3]));
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const float4 s4 = *reinterpret_cast<const float4*>(sS + size_t(j0 + g + 8 * half) * DK + c);
+      acc[2 * q][2 * half] = s4.x * d.x;
+      acc[2 * q][2 * half + 1] = s4.y * d.y;
+      acc[2 * q + 1][2 * half] = s4.z * d.z;
+      acc[2 * q + 1][2 * half + 1] = s4.w * d.w;
+    }
+  }
+}
+
+// Writes the fp32 fold's accumulators (fold_channel_il order) as rows j0+g,
+// j0+g+8 of gOut (row-major, DK per row).
+template <int DK>
+__device__ __forceinline__ void fold_store_f32_il(const float (&acc)[DK / 8][4], int j0, int lane,
+                                                  float* gOut) {
+  const int g = lane >> 2;
+  const int t = lane & 3;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float* o = gOut + size_t(j0 + g + 8 * half) * DK + 4 * t;
+#pragma unroll
+    for (int q = 0; q < DK / 16; ++q)
+      *reinterpret_cast<float4*>(o + 16 * q) =
+          make_float4(acc[2 * q][2 * half], acc[2 * q][2 * half + 1], acc[2 * q + 1][2 * half],
+                      acc[2 * q + 1][2 * half + 1]);
+  }
+}
 
 // Folds nent log entries into the warp's 16 rows of an int8 base on the
 // tensor cores, in one pass:
@@ -210,39 +322,14 @@ __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sSca
       }
     }
   }
-  const uint4* sB4 = reinterpret_cast<const uint4*>(sB);
-  for (int kc = 0; kc < nchunks; ++kc) {
-    const int e0 = 16 * kc + 2 * t;
-    float u[8];  // (g, e0), (g, e0+1), (g+8, e0), (g+8, e0+1), then the same at e0+8
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = e0 + (q & 1) + ((q & 4) ? 8 : 0);
-      u[q] = (e < nent) ? to_f(sU[su_offset(rows[(q >> 1) & 1], e, L)]) : 0.f;
-    }
-    uint32_t ah[4], al[4];
-    split_h2(u[0], u[1], ah[0], al[0]);  // a0: row g,   k 2t..
-    split_h2(u[2], u[3], ah[1], al[1]);  // a1: row g+8
-    split_h2(u[4], u[5], ah[2], al[2]);  // a2: row g,   k 2t+8..
-    split_h2(u[6], u[7], ah[3], al[3]);  // a3: row g+8
-#pragma unroll
-    for (int n = 0; n < NTILE; ++n) {
-      const uint4 bf = sB4[kt_slot(kc, NTILE, n, lane)];
-      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.x, bf.y);
-      mma_16816(acc[n], ah[0], ah[1], ah[2], ah[3], bf.z, bf.w);
-      mma_16816(acc[n], al[0], al[1], al[2], al[3], bf.x, bf.y);
-    }
+  fold_mma_acc<DK, TU>(acc, sU, sB, nent, nchunks, L, j0, lane);
+  if (gOut != nullptr) {
+    fold_acc_store_f32<DK>(acc, j0, lane, gOut);
+    return;
   }
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const int r = rows[half];
-    if (gOut != nullptr) {
-      float4* o = reinterpret_cast<float4*>(gOut + size_t(r) * DK + cbase);
-#pragma unroll
-      for (int v = 0; v < WORDS; ++v)
-        o[v] = make_float4(acc[2 * v][2 * half], acc[2 * v][2 * half + 1], acc[2 * v + 1][2 * half],
-                           acc[2 * v + 1][2 * half + 1]);
-      continue;
-    }
     float m = 0.f;
 #pragma unroll
     for (int n = 0; n < NTILE; ++n)

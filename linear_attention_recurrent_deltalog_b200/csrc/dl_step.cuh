@@ -65,12 +65,16 @@ struct StepLayout {
 // registers a thread), which the ~34 KB of shared memory of a 128-row head
 // allows anyway; the fold of the fused merge runs one 16-row tile at a time
 // so it needs no more.  The fp32 kernels keep the compiler's choice.
-template <typename TB, int THREADS, bool FOLDS>
-constexpr int kMinBlocks = std::is_same<TB, int8_t>::value ? 768 / THREADS : 1;
+// The fp32 step with the fused merge in 64-row items at d_k = 128 (the only
+// one with the tensor-core fold) is held to 5 CTAs per SM, what its shared
+// memory allows, so the fold's accumulators do not cost occupancy.
+template <typename TB, int THREADS, bool FOLDS, int DK>
+constexpr int kMinBlocks = std::is_same<TB, int8_t>::value ? 768 / THREADS
+                           : ((FOLDS && DK == 128 && THREADS == 128) ? 5 : 1);
 
 template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB, bool FUSED>
 __global__ void __launch_bounds__(StepTile<DK, ROWS, TB>::kThreads,
-                                  kMinBlocks<TB, StepTile<DK, ROWS, TB>::kThreads, FUSED>)
+                                  kMinBlocks<TB, StepTile<DK, ROWS, TB>::kThreads, FUSED, DK>)
 dl_step_kernel(const StepParams p, const FillParam fp) {
   using Tl = StepTile<DK, ROWS, TB>;
   using TU = typename LogU<VAR, TIn>::type;
@@ -326,9 +330,36 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
                                     static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
                                     p.scale + head * size_t(DV) + r0, nullptr);
   } else {
-    __syncwarp();
-    merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane,
-                                       static_cast<float*>(p.base) + (head * size_t(DV) + r0) * DK);
+    float* gRows = static_cast<float*>(p.base) + (head * size_t(DV) + r0) * DK;
+    const int nch = q8_chunks(f + 1);
+    // The fold runs on the FMA pipe unless the log is long (>= 32 entries) in
+    // a 64-row work item at d_k = 128 (where the staged key fragments of up to
+    // 64 entries fit in the tile's room): for short logs the tensor-core
+    // path's padding to 16 entries and its three CTA barriers cost more than
+    // the FMAs they save (measured on B200).
+    if (DK < 128 || ROWS != 64 || f + 1 < 32) {
+      __syncwarp();
+      merge_rows_fused<VAR, DK, TU, TIn>(sS, sU, sK, sG, sGt, sScal[2], f, L, j0, lane, gRows);
+      return;
+    }
+    // On the tensor cores (m16n8k16, fp16 hi/lo operands, fp32 accumulators):
+    // every warp first takes its decayed base rows into registers, then the
+    // CTA stages the decayed keys of the L entries as B fragments where the
+    // tile was, and each warp adds U Kt and writes its rows.
+    if constexpr (DK == 128 && ROWS == 64) {
+    float acc[DK / 8][4];
+    fold_init_f32<DK, GW == 1>(acc, sS, sGt, sScal[2], j0, lane);
+    __syncthreads();  // the tile is free; every warp's u_t is in slot f
+    if (GW == 1) {    // GDN: one decay factor per entry (sW's weights are no longer needed)
+      for (int e = tid; e < f; e += NT) sW[e] = expf(sGt[0] - sG[e]);
+      __syncthreads();
+    }
+    uint32_t* sB = reinterpret_cast<uint32_t*>(sS);
+    stage_kt_frags<VAR, DK, TIn, true>(sK, sG, sGt, sW, f, f + 1, nch, sB, tid, NT);
+    __syncthreads();
+    fold_mma_acc<DK, TU>(acc, sU, sB, f + 1, nch, L, j0, lane);
+    fold_store_f32_il<DK>(acc, j0, lane, gRows);
+    }
   }
 }
 
