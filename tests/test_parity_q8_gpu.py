@@ -86,6 +86,18 @@ def test_q8_shapes_dtypes_splits(variant, dk, dv, dtype, split):
         _check(r)
 
 
+@pytest.mark.parametrize("dk", [64, 128])
+def test_q8_large_batch_merge(dk):
+    # more than 4096 sequences merging at once: the TMEM merge reads each
+    # head's fill from the device instead of the launch's list (d_k = 64
+    # runs its MMAs with N = 64 over 64 TMEM columns)
+    w = wl.WORKLOADS["gdn_qwen"].replace(B=4200, H=1, d_k=dk, d_v=128, L=2, ragged=False, seed=47)
+    _check(run_parity_q8(w, T=5, heads=wl.sample_heads(w, 24), fused=False, snap_every=2))
+    w = wl.WORKLOADS["kda"].replace(B=4200, H=1, d_k=dk, d_v=128, L=3, ragged=False, seed=48)
+    _check(run_parity_q8(w, T=7, heads=wl.sample_heads(w, 24), fused=False, merge_all_at=(4,),
+                         snap_every=3))
+
+
 def test_q8_forced_merges():
     # merges of every non-empty log mid-window end those windows early
     w = wl.WORKLOADS["gdn_qwen"].replace(B=8, H=4, L=6, ragged=True, seed=41)
