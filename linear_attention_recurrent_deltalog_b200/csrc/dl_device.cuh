@@ -234,6 +234,19 @@ __device__ __forceinline__ void tma_load_1d_stream(void* dst, const void* src, u
       : "memory");
 }
 
+// Same, with an L2 evict-last policy: log entries, which every later step
+// reads again until the log is merged.
+__device__ __forceinline__ void tma_load_1d_keep(void* dst, const void* src, uint32_t bytes,
+                                                 uint64_t* bar) {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(policy));
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // --------------------------------------------------------- row reduction
 //
 // A warp covers rows of a d_v x d_k tile: LPR lanes per row, each lane

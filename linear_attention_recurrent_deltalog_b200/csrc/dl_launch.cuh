@@ -138,8 +138,12 @@ cudaError_t launch_merge_q8_tmem(const MergeParams& p, const SeqList& list, unsi
 template <int VAR, int DK, int DV, typename TIn, typename TB>
 cudaError_t launch_merge_t(const MergeParams& p, const SeqList& list, unsigned nheads,
                            cudaStream_t s) {
-  if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows)
-    return launch_merge_q8_tmem<VAR, DK, TIn>(p, list, nheads, s);
+  if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows) {
+    // long vector-decay logs whose two stages do not fit in shared memory
+    // take the per-warp fold below
+    if (MergePipeLayout<VAR, DK, TIn>(p.L).total <= size_t(kMaxSmemOptIn))
+      return launch_merge_q8_tmem<VAR, DK, TIn>(p, list, nheads, s);
+  }
   if constexpr (DV >= 128) {
     if (p.use_list || p.mode == 2)
       return launch_merge_rows<VAR, DK, DV, DV / 2, TIn, TB>(p, list, nheads, s);
@@ -286,10 +290,11 @@ struct MergeSmem {
   size_t out;
   template <int DK, int DV, typename T>
   cudaError_t run() {
-    if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows)
-      out = MergePipeLayout<VAR, DK, T>(L).total;
-    else
-      out = MergeLayout<VAR, DK, DV, DV, T, TB>(L).total;
+    out = MergeLayout<VAR, DK, DV, DV, T, TB>(L).total;
+    if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows) {
+      const size_t pipe = MergePipeLayout<VAR, DK, T>(L).total;
+      if (pipe <= size_t(kMaxSmemOptIn)) out = pipe;
+    }
     return cudaSuccess;
   }
 };

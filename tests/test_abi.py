@@ -242,3 +242,18 @@ def test_int8_code_swizzle_is_a_chunk_permutation(dk, dv):
     groups = (perm[:8, ::16] // 16) % 8          # rows 0..7, each logical chunk
     for j in range(dk // 16):
         assert len(set(groups[:, j].tolist())) == 8
+
+
+@pytest.mark.parametrize("variant", ["gdn", "kda", "gdn2", "rwkv6"])
+@pytest.mark.parametrize("L", [16, 48, 64])
+def test_q8_every_log_length_is_built(variant, L):
+    # the int8 merge takes the per-warp fold wherever its two-stage TMEM
+    # pipeline would not fit in shared memory (long vector-decay logs), so a
+    # state of every L up to 64 can be created (host-side check, no launch)
+    d = 64 if variant == "rwkv6" else 128
+    c = cfg(variant=variant, d_k=d, d_v=d, L=L, base="q8").c()
+    st = ctypes.c_void_p()
+    rc = dlb._lib.dl_state_create(ctypes.byref(c), ctypes.c_void_p(1 << 20), ctypes.c_void_p(2 << 20),
+                                  ctypes.c_void_p(3 << 20), ctypes.byref(st))
+    assert rc == dlb.DL_OK
+    assert dlb._lib.dl_state_destroy(st) == dlb.DL_OK

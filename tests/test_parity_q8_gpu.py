@@ -98,6 +98,14 @@ def test_q8_large_batch_merge(dk):
                          snap_every=3))
 
 
+def test_q8_long_vector_log():
+    # L = 64 with a vector decay: the merge takes the per-warp fold (the
+    # two-stage TMEM pipeline would not fit in shared memory)
+    w = wl.WORKLOADS["kda"].replace(B=3, H=2, L=64, ragged=True, seed=49)
+    _check(run_parity_q8(w, T=70, fused=False, snap_every=10))
+    _check(run_parity_q8(w, T=70, fused=True, snap_every=10))
+
+
 def test_q8_forced_merges():
     # merges of every non-empty log mid-window end those windows early
     w = wl.WORKLOADS["gdn_qwen"].replace(B=8, H=4, L=6, ragged=True, seed=41)
