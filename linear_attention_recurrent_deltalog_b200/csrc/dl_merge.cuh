@@ -33,8 +33,10 @@ struct MergeLayout {
 // DV / ROWS CTAs, as in the step).  With a list, the fills come from the
 // list and only part 0 empties the log, so split CTAs never race on it;
 // without a list the kernel runs unsplit and reads the device fill.
-// The int8 merge folds every CTA: compiled for 640 threads per SM (about
-// 100 registers, no spills).
+// It serves every fp32 base, and the int8 bases that the TMEM kernel below
+// does not take (d_v = 64 heads, and long vector-decay logs whose two
+// pipeline stages do not fit in shared memory); its int8 fold is per-warp
+// mma.sync, compiled for 640 threads per SM (about 100 registers, no spills).
 template <typename TB, int THREADS>
 constexpr int kMergeMinBlocks = std::is_same<TB, int8_t>::value ? 640 / THREADS : 1;
 
