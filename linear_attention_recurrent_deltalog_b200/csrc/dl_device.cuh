@@ -357,6 +357,39 @@ __device__ __forceinline__ uint32_t pack_codes4(uint32_t r0, uint32_t r1, uint32
   return __byte_perm(__byte_perm(r0, r1, 0x0040), __byte_perm(r2, r3, 0x0040), 0x5410);
 }
 
+// ------------------------------------------------- packed fp32 pairs
+//
+// sm_100 adds and multiplies two fp32 lanes with one instruction
+// (add/mul .rn.f32x2 on a 64-bit register pair); each lane is rounded
+// exactly as the scalar .rn operation rounds it, and an explicit rounding
+// mode keeps the compiler from fusing a multiply into a following add.  The
+// code conversions of an int8 row are dominated by such pairs.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// round_code_bits of two values: inv2 = f2_pack(inv, inv).
+__device__ __forceinline__ void round_code_bits2(float x0, float x1, uint64_t inv2, uint32_t& r0,
+                                                 uint32_t& r1) {
+  const uint64_t r = f2_add(f2_mul(f2_pack(x0, x1), inv2), f2_pack(12582912.0f, 12582912.0f));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(r));
+}
+
 // ------------------------------------------- int8 codes on the tensor cores
 //
 // The int8 base is multiplied on the tensor cores with warp-level

@@ -102,39 +102,43 @@ __device__ __forceinline__ void stage_fold_b(const TIn* sK, const float* sG, con
   }
 }
 
-// Sixteen int8 codes -> fp32, exactly: with the sign bit flipped each byte is
-// n = code + 128, placed as the low mantissa byte of 2^23 (0x4B0000nn), and
-// subtracting 2^23 + 128 leaves the code.
-__device__ __forceinline__ void codes16_to_f(uint4 q, float (&x)[16]) {
-  const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
-                         q.w ^ 0x80808080u};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      x[4 * i + k] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7650u + uint32_t(k))) - 8388736.0f;
-  }
-}
-
 // Writes columns c0 .. c0+NCOL-1 of row `row` of the dequantized, decayed
 // base into this thread's TMEM lane: x_c = (code_c * scale) * dec_c (SDEC:
 // one decay dec[0] for every c, folded into the scale first).  sDec: decay
-// per channel at dec_pad indices.
+// per channel at dec_pad indices (pairs of channels are adjacent there).
+// Codes -> fp32, exactly: with the sign bit flipped each byte is n = code +
+// 128, placed as the low mantissa byte of 2^23 (0x4B0000nn), and
+// subtracting 2^23 + 128 leaves the code; the subtraction and the scaling
+// run on packed pairs.
 template <int DK, int NCOL, bool SDEC>
 __device__ __forceinline__ void fold_init_q8(const int8_t* sQ, float scale, const float* sDec, int row,
                                              int c0, uint32_t lane_addr) {
-  const float sd = SDEC ? scale * sDec[0] : 0.f;
+  const float sd = SDEC ? scale * sDec[0] : scale;
+  const uint64_t s2 = f2_pack(sd, sd);
+  const uint64_t m2 = f2_pack(-8388736.0f, -8388736.0f);
 #pragma unroll 1
   for (int blk = 0; blk < NCOL / 32; ++blk) {
     const int cb = c0 + 32 * blk;
     float x[32];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float c16[16];
-      codes16_to_f(*reinterpret_cast<const uint4*>(sQ + q8_off<DK>(row, cb + 16 * h)), c16);
+      const uint4 q = *reinterpret_cast<const uint4*>(sQ + q8_off<DK>(row, cb + 16 * h));
+      const uint32_t w[4] = {q.x ^ 0x80808080u, q.y ^ 0x80808080u, q.z ^ 0x80808080u,
+                             q.w ^ 0x80808080u};
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        x[16 * h + i] = SDEC ? c16[i] * sd : (c16[i] * scale) * sDec[dec_pad(cb + 16 * h + i)];
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t wi = w[i >> 1];
+        const uint32_t k = uint32_t(2 * (i & 1));
+        const uint64_t c2 = f2_add(f2_pack(__uint_as_float(__byte_perm(wi, 0x4B000000u, 0x7650u + k)),
+                                           __uint_as_float(__byte_perm(wi, 0x4B000000u, 0x7651u + k))),
+                                   m2);  // the two codes, exactly
+        uint64_t x2 = f2_mul(c2, s2);
+        if (!SDEC) {
+          const float2 d = *reinterpret_cast<const float2*>(sDec + dec_pad(cb + 16 * h + 2 * i));
+          x2 = f2_mul(x2, f2_pack(d.x, d.y));
+        }
+        f2_unpack(x2, x[16 * h + 2 * i], x[16 * h + 2 * i + 1]);
+      }
     }
     tmem_st32(lane_addr + uint32_t(cb), x);
   }
@@ -181,6 +185,7 @@ __device__ __forceinline__ float fold_amax(uint32_t lane_addr, int c0) {
 template <int DK, int NCOL>
 __device__ __forceinline__ void fold_store_q8(uint32_t lane_addr, int c0, int row, float inv,
                                               int8_t* gCodes) {
+  const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
   for (int blk = 0; blk < NCOL / 32; ++blk) {
     const int cb = c0 + 32 * blk;
@@ -193,8 +198,10 @@ __device__ __forceinline__ void fold_store_q8(uint32_t lane_addr, int c0, int ro
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int i = 16 * h + 4 * k;
-        w[k] = pack_codes4(round_code_bits(v[i], inv), round_code_bits(v[i + 1], inv),
-                           round_code_bits(v[i + 2], inv), round_code_bits(v[i + 3], inv));
+        uint32_t r[4];
+        round_code_bits2(v[i], v[i + 1], inv2, r[0], r[1]);
+        round_code_bits2(v[i + 2], v[i + 3], inv2, r[2], r[3]);
+        w[k] = pack_codes4(r[0], r[1], r[2], r[3]);
       }
       *reinterpret_cast<uint4*>(gCodes + q8_off<DK>(row, cb + 16 * h)) =
           make_uint4(w[0], w[1], w[2], w[3]);

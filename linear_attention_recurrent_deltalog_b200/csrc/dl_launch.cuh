@@ -112,16 +112,16 @@ inline int resident_ctas(Kern kern, int threads, size_t smem, int cap) {
 }
 
 // The int8 merge of d_v = 128 heads on TMEM: a persistent launch of as many
-// 288-thread CTAs as fit on the SMs (its shared memory keeps that at most
-// 512 / d_k per SM), each walking the listed heads.
-template <int VAR, int DK, typename TIn>
+// 288-thread CTAs as fit on the SMs (at most 512 / d_k per SM, so every
+// TMEM allocation succeeds at once), each walking the listed heads.
+template <int VAR, int DK, typename TIn, int NS>
 cudaError_t launch_merge_q8_tmem(const MergeParams& p, const SeqList& list, unsigned nheads,
                                  cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
-  auto kern = dl_merge_q8_kernel<VAR, DK, TIn>;
+  auto kern = dl_merge_q8_kernel<VAR, DK, TIn, NS>;
   cudaError_t e = prepare_kernel(kern, done);
   if (e != cudaSuccess) return e;
-  const size_t smem = MergePipeLayout<VAR, DK, TIn>(p.L).total;
+  const size_t smem = MergePipeLayout<VAR, DK, TIn, NS>(p.L).total;
   const int per_sm = resident_ctas(kern, kMergePipeThreads, smem, 512 / DK);
   const int sms = sm_count();
   if (per_sm <= 0 || sms <= 0) return cudaErrorInvalidConfiguration;
@@ -139,10 +139,14 @@ template <int VAR, int DK, int DV, typename TIn, typename TB>
 cudaError_t launch_merge_t(const MergeParams& p, const SeqList& list, unsigned nheads,
                            cudaStream_t s) {
   if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows) {
-    // long vector-decay logs whose two stages do not fit in shared memory
-    // take the per-warp fold below
-    if (MergePipeLayout<VAR, DK, TIn>(p.L).total <= size_t(kMaxSmemOptIn))
-      return launch_merge_q8_tmem<VAR, DK, TIn>(p, list, nheads, s);
+    // Merge: one stage (4 CTAs per SM at d_k = 128).  Materialize writes
+    // twice the bytes per head of fp32 output and measured faster with two
+    // stages (3 CTAs per SM).  Long vector-decay logs whose stages do not fit
+    // in shared memory take the per-warp fold below.
+    if (p.mode == 2 && MergePipeLayout<VAR, DK, TIn, 2>(p.L).total <= size_t(kMaxSmemOptIn))
+      return launch_merge_q8_tmem<VAR, DK, TIn, 2>(p, list, nheads, s);
+    if (MergePipeLayout<VAR, DK, TIn, kMergeStages>(p.L).total <= size_t(kMaxSmemOptIn))
+      return launch_merge_q8_tmem<VAR, DK, TIn, kMergeStages>(p, list, nheads, s);
   }
   if constexpr (DV >= 128) {
     if (p.use_list || p.mode == 2)
@@ -292,7 +296,7 @@ struct MergeSmem {
   cudaError_t run() {
     out = MergeLayout<VAR, DK, DV, DV, T, TB>(L).total;
     if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows) {
-      const size_t pipe = MergePipeLayout<VAR, DK, T>(L).total;
+      const size_t pipe = MergePipeLayout<VAR, DK, T, kMergeStages>(L).total;
       if (pipe <= size_t(kMaxSmemOptIn)) out = pipe;
     }
     return cudaSuccess;

@@ -204,18 +204,26 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
 //
 // d_v = 128 heads of an int8 base, as a pipelined persistent kernel: each
 // CTA walks the heads blockIdx.x, blockIdx.x + gridDim.x, ...  A producer
-// warp streams the next head's codes, row scales and log entries into one of
-// two shared-memory stages while eight consumer warps fold the current head:
+// warp streams the next head's codes, row scales and log entries into a
+// shared-memory stage while eight consumer warps fold the current head:
 // thread i of consumer warp w owns row 32 (w mod 4) + i and half of its key
 // channels.  The fold D = deq(codes) Diag(dec) + U Kt accumulates in tensor
 // memory (dl_fold_tmem.cuh), allocated once per CTA; the requantize (merge)
-// or the fp32 write (materialize) reads each row straight from TMEM.
+// or the fp32 write (materialize) reads each row straight from TMEM.  A
+// stage is dead once its head's operands are staged and its base written
+// into TMEM (before the MMA), so the consumers hand it back there and the
+// producer loads the next head while they wait for the MMA and requantize:
+// with NS = 1 stage a CTA needs about 47 KB at d_k = 128, and 4 CTAs (the
+// 512 TMEM columns' worth) fit on an SM (merge on B200: 0.55 -> 0.65 of the
+// copy bandwidth against two stages and 3 CTAs; materialize, whose fp32
+// output is twice as large, stays faster with two).
 
 constexpr int kFoldThreads = 2 * kFoldRows;       // consumer threads
 constexpr int kMergePipeThreads = kFoldThreads + 32;  // plus the producer warp
 constexpr int kConsumerBar = 1;                   // named barrier of the consumers
+constexpr int kMergeStages = 1;                   // shared-memory stages of the pipeline
 
-template <int VAR, int DK, typename TIn>
+template <int VAR, int DK, typename TIn, int NS = 1>
 struct MergePipeLayout {
   using TU = typename LogU<VAR, TIn>::type;
   // inside a stage (codes at 0)
@@ -228,13 +236,13 @@ struct MergePipeLayout {
     inG = inK + align_up(size_t(L) * DK * sizeof(TIn), 128);         // k [L][DK]
     inScale = inG + align_up(size_t(g_stride(VAR, L, DK)) * 4, 128); // g
     stage = inScale + align_up(size_t(kFoldRows) * 4, 128);          // row scales
-    offA = 2 * stage;                                                // A hi, lo (then row maxima)
+    offA = NS * stage;                                               // A hi, lo (then row maxima)
     offB = offA + 2 * nch * kFoldAStep;                              // B hi, lo
     offDec = offB + 2 * nch * kFoldBStep<DK>;                        // decay, GDN factors
     offMeta = offDec + align_up(size_t(kDecPadLen<DK> + 64) * 4, 128);
     offTmem = offMeta + 32;
     offBar = offTmem + 16;
-    const size_t need = offBar + 8 * 5;  // full[2], empty[2], mma
+    const size_t need = offBar + 8 * (2 * NS + 1);  // full[NS], empty[NS], mma
     // at most 512 / DK CTAs per SM, so every CTA's TMEM allocation succeeds
     // at once (228 KB of shared memory per SM, 1 KB reserved per CTA)
     const size_t floor_bytes = (DK == 128) ? 49152 : 26624;
@@ -249,8 +257,8 @@ struct MergeItem {
   int skip;  // nothing to fold (mode's filter) or an invalid fill
 };
 
-template <int VAR, int DK, typename TIn>
-__global__ void __launch_bounds__(kMergePipeThreads, 3)
+template <int VAR, int DK, typename TIn, int NS>
+__global__ void __launch_bounds__(kMergePipeThreads, NS == 1 ? 4 : 3)
 dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
   using TU = typename LogU<VAR, TIn>::type;
   constexpr int GW = (VAR == kVarGDN) ? 1 : DK;
@@ -261,7 +269,7 @@ dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int L = p.L;
   const int GS = g_stride(VAR, L, DK);
-  const MergePipeLayout<VAR, DK, TIn> lay(L);
+  const MergePipeLayout<VAR, DK, TIn, NS> lay(L);
   unsigned char* sA = smem + lay.offA;
   unsigned char* sB = smem + lay.offB;
   float* sAmax = reinterpret_cast<float*>(sA);                 // after the MMA: row maxima
@@ -270,14 +278,14 @@ dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
   MergeItem* sMeta = reinterpret_cast<MergeItem*>(smem + lay.offMeta);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + lay.offTmem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.offBar);
-  uint64_t* empty = full + 2;
-  uint64_t* barMma = full + 4;
+  uint64_t* empty = full + NS;
+  uint64_t* barMma = full + 2 * NS;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -296,11 +304,13 @@ dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
   if (warp == kFoldThreads / 32) {
     // ---- producer: one lane issues every copy
     if (lane == 0) {
+      int lastj[NS];  // per stage, the last item announced on its full barrier
+      for (int s = 0; s < NS; ++s) lastj[s] = -1;
       for (unsigned j = 0;; ++j) {
         const unsigned it = blockIdx.x + j * gridDim.x;
         if (it >= nitems) break;
-        const int s = int(j & 1);
-        if (j >= 2 && !mbar_wait(&empty[s], ((j - 2) >> 1) & 1, p.err, -1)) break;
+        const int s = int(j % NS);
+        if (j >= NS && !mbar_wait(&empty[s], ((j - NS) / NS) & 1, p.err, -1)) break;
         const unsigned li = it / unsigned(p.H);
         const size_t head = p.use_list ? size_t(list.seq[li]) * size_t(p.H) + it % unsigned(p.H)
                                        : size_t(it);
@@ -313,6 +323,7 @@ dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
           skip = 1;
         }
         sMeta[s] = MergeItem{head, f, skip};
+        lastj[s] = int(j);
         if (skip) {
           mbar_arrive(&full[s]);
           continue;
@@ -337,6 +348,11 @@ dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
           tma_load_1d(st + lay.inG, p.logG + head * size_t(GS), bg, &full[s]);
         }
       }
+      // if the consumers stopped early (an error), no copy may still be
+      // landing in shared memory when the CTA exits: wait for each stage's
+      // last phase (already complete when every item was consumed)
+      for (int s = 0; s < NS; ++s)
+        if (lastj[s] >= 0) mbar_wait(&full[s], (unsigned(lastj[s]) / NS) & 1, nullptr, 0);
     }
   } else {
     // ---- consumers
@@ -348,72 +364,77 @@ dl_merge_q8_kernel(const MergeParams p, const SeqList list, unsigned nitems) {
     for (unsigned j = 0;; ++j) {
       const unsigned it = blockIdx.x + j * gridDim.x;
       if (it >= nitems) break;
-      const int s = int(j & 1);
-      if (!named_bar_and(kConsumerBar, kFoldThreads, mbar_wait(&full[s], (j >> 1) & 1, p.err, -1)))
+      const int s = int(j % NS);
+      if (!named_bar_and(kConsumerBar, kFoldThreads,
+                         mbar_wait(&full[s], (j / NS) & 1, p.err, -1)))
         break;
       tc_fence_after();
       const MergeItem m = sMeta[s];
-      if (!m.skip) {
-        const size_t head = size_t(m.head);
-        const int f = m.f;
-        const unsigned char* st = smem + size_t(s) * lay.stage;
-        const int8_t* sQ = reinterpret_cast<const int8_t*>(st);
-        const TU* sU = reinterpret_cast<const TU*>(st + lay.inU);
-        const TIn* sK = reinterpret_cast<const TIn*>(st + lay.inK);
-        const float* sG = reinterpret_cast<const float*>(st + lay.inG);
-        const float* sScale = reinterpret_cast<const float*>(st + lay.inScale);
-        for (int c = tid; c < DK; c += kFoldThreads)
-          sDec[dec_pad(c)] = expf((f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f);
-        if (GW == 1)
-          for (int e = tid; e < f; e += kFoldThreads) sFac[e] = expf(sG[f - 1] - sG[e]);
-        named_bar_sync(kConsumerBar, kFoldThreads);
-        const int nch = q8_chunks(f);
-        if (f > 0) {
-          if (tid < kFoldRows)  // A: one row per thread of the first four warps
-            stage_fold_a<TU>(sU, f, nch, L, sA, tid);
-          else                  // B: the other four warps
-            stage_fold_b<VAR, DK, TIn>(sK, sG, sG + size_t(f - 1) * GW, sFac, f, f, nch, sB,
-                                       tid - kFoldRows, kFoldThreads - kFoldRows);
-          fence_async_smem();
-        }
-        // D = the dequantized, decayed base rows
-        fold_init_q8<DK, NCOL, GW == 1>(sQ, sScale[row], sDec, row, c0, lane_addr);
-        tmem_wait_st();
-        tc_fence_before();
-        named_bar_sync(kConsumerBar, kFoldThreads);
-        if (nch > 0) {
-          if (tid == 0) {
-            tc_fence_after();
-            fold_issue<DK>(tmem, sA, sB, nch, barMma);
-          }
-          // one thread polls the MMA's completion; the others sleep in the
-          // named barrier and order their TMEM reads after it with the fence
-          const bool done = named_bar_and(
-              kConsumerBar, kFoldThreads,
-              (tid == 0) ? mbar_wait(barMma, mma_phase, p.err, int(head)) : true);
-          mma_phase ^= 1u;
-          tc_fence_after();
-          if (!done) break;
-        }
-        if (p.mode == 2) {
-          fold_store_f32<NCOL>(lane_addr, c0, p.out + (head * size_t(DV) + row) * DK);
-        } else {
-          sAmax[half * kFoldRows + row] = fold_amax<NCOL>(lane_addr, c0);
-          named_bar_sync(kConsumerBar, kFoldThreads);
-          const float amax = fmaxf(sAmax[row], sAmax[kFoldRows + row]);
-          const bool live = amax >= kTinyAmax;
-          const float inv = live ? __fdiv_rn(127.0f, amax) : 0.f;
-          fold_store_q8<DK, NCOL>(lane_addr, c0, row, inv,
-                                  static_cast<int8_t*>(p.base) + head * size_t(DV) * DK);
-          if (!half) p.scale[head * size_t(DV) + row] = live ? __fdiv_rn(amax, 127.0f) : 0.f;
-          // the log is emptied only once the merged rows are written
-          if (tid == 0) p.fill[head] = 0;
-        }
-        tc_fence_before();
+      if (m.skip) {
+        named_bar_sync(kConsumerBar, kFoldThreads);  // every consumer has read the item
+        if (tid == 0) mbar_arrive(&empty[s]);
+        continue;
       }
-      // stage s, the operand buffers and TMEM are free again
+      const size_t head = size_t(m.head);
+      const int f = m.f;
+      const unsigned char* st = smem + size_t(s) * lay.stage;
+      const int8_t* sQ = reinterpret_cast<const int8_t*>(st);
+      const TU* sU = reinterpret_cast<const TU*>(st + lay.inU);
+      const TIn* sK = reinterpret_cast<const TIn*>(st + lay.inK);
+      const float* sG = reinterpret_cast<const float*>(st + lay.inG);
+      const float* sScale = reinterpret_cast<const float*>(st + lay.inScale);
+      for (int c = tid; c < DK; c += kFoldThreads)
+        sDec[dec_pad(c)] = expf((f > 0) ? sG[size_t(f - 1) * GW + (GW > 1 ? c : 0)] : 0.f);
+      if (GW == 1)
+        for (int e = tid; e < f; e += kFoldThreads) sFac[e] = expf(sG[f - 1] - sG[e]);
       named_bar_sync(kConsumerBar, kFoldThreads);
+      const int nch = q8_chunks(f);
+      if (f > 0) {
+        if (tid < kFoldRows)  // A: one row per thread of the first four warps
+          stage_fold_a<TU>(sU, f, nch, L, sA, tid);
+        else                  // B: the other four warps
+          stage_fold_b<VAR, DK, TIn>(sK, sG, sG + size_t(f - 1) * GW, sFac, f, f, nch, sB,
+                                     tid - kFoldRows, kFoldThreads - kFoldRows);
+        fence_async_smem();
+      }
+      // D = the dequantized, decayed base rows
+      fold_init_q8<DK, NCOL, GW == 1>(sQ, sScale[row], sDec, row, c0, lane_addr);
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(kConsumerBar, kFoldThreads);
+      // the stage is no longer read: the producer may load the next head
       if (tid == 0) mbar_arrive(&empty[s]);
+      if (nch > 0) {
+        if (tid == 0) {
+          tc_fence_after();
+          fold_issue<DK>(tmem, sA, sB, nch, barMma);
+        }
+        // one thread polls the MMA's completion; the others sleep in the
+        // named barrier and order their TMEM reads after it with the fence
+        const bool done = named_bar_and(
+            kConsumerBar, kFoldThreads,
+            (tid == 0) ? mbar_wait(barMma, mma_phase, p.err, int(head)) : true);
+        mma_phase ^= 1u;
+        tc_fence_after();
+        if (!done) break;
+      }
+      if (p.mode == 2) {
+        fold_store_f32<NCOL>(lane_addr, c0, p.out + (head * size_t(DV) + row) * DK);
+      } else {
+        sAmax[half * kFoldRows + row] = fold_amax<NCOL>(lane_addr, c0);
+        named_bar_sync(kConsumerBar, kFoldThreads);
+        const float amax = fmaxf(sAmax[row], sAmax[kFoldRows + row]);
+        const bool live = amax >= kTinyAmax;
+        const float inv = live ? __fdiv_rn(127.0f, amax) : 0.f;
+        fold_store_q8<DK, NCOL>(lane_addr, c0, row, inv,
+                                static_cast<int8_t*>(p.base) + head * size_t(DV) * DK);
+        if (!half) p.scale[head * size_t(DV) + row] = live ? __fdiv_rn(amax, 127.0f) : 0.f;
+        // the log is emptied only once the merged rows are written
+        if (tid == 0) p.fill[head] = 0;
+      }
+      // the operand buffers, the row maxima and TMEM are free again
+      tc_fence_before();
+      named_bar_sync(kConsumerBar, kFoldThreads);
     }
   }
   tc_fence_before();

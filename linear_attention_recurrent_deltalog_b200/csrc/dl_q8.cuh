@@ -301,25 +301,25 @@ __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sSca
       w[4 * v + 2] = q.z;
       w[4 * v + 3] = q.w;
     }
-    const float sd = SDEC ? s * sDec[0] : 0.f;
+    // x = code * (scale * dec) (SDEC), else (code * scale) * dec_c, on
+    // packed pairs (an accumulator pair acc[n][2 half], +1 is a register pair)
+    const float sd = SDEC ? s * sDec[0] : s;
+    const uint64_t s2 = f2_pack(sd, sd);
 #pragma unroll
     for (int v = 0; v < WORDS; ++v) {
       uint32_t h01, h23;
       codes4_to_h2(w[v], h01, h23);
       const float2 c01 = __half22float2(bits_h2(h01));
       const float2 c23 = __half22float2(bits_h2(h23));
-      if (SDEC) {
-        acc[2 * v][2 * half] = c01.x * sd;
-        acc[2 * v][2 * half + 1] = c01.y * sd;
-        acc[2 * v + 1][2 * half] = c23.x * sd;
-        acc[2 * v + 1][2 * half + 1] = c23.y * sd;
-      } else {
+      uint64_t x01 = f2_mul(f2_pack(c01.x, c01.y), s2);
+      uint64_t x23 = f2_mul(f2_pack(c23.x, c23.y), s2);
+      if (!SDEC) {
         const float4 d4 = *reinterpret_cast<const float4*>(sDec + dec_pad(cbase + 4 * v));
-        acc[2 * v][2 * half] = (c01.x * s) * d4.x;
-        acc[2 * v][2 * half + 1] = (c01.y * s) * d4.y;
-        acc[2 * v + 1][2 * half] = (c23.x * s) * d4.z;
-        acc[2 * v + 1][2 * half + 1] = (c23.y * s) * d4.w;
+        x01 = f2_mul(x01, f2_pack(d4.x, d4.y));
+        x23 = f2_mul(x23, f2_pack(d4.z, d4.w));
       }
+      f2_unpack(x01, acc[2 * v][2 * half], acc[2 * v][2 * half + 1]);
+      f2_unpack(x23, acc[2 * v + 1][2 * half], acc[2 * v + 1][2 * half + 1]);
     }
   }
   fold_mma_acc<DK, TU>(acc, sU, sB, nent, nchunks, L, j0, lane);
@@ -338,13 +338,15 @@ __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sSca
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
     // rows below the tiny threshold store zero codes (inv = 0) and scale 0
     const float inv = (m >= kTinyAmax) ? __fdiv_rn(127.0f, m) : 0.f;
+    const uint64_t inv2 = f2_pack(inv, inv);
     uint32_t w[WORDS];
 #pragma unroll
-    for (int v = 0; v < WORDS; ++v)
-      w[v] = pack_codes4(round_code_bits(acc[2 * v][2 * half], inv),
-                         round_code_bits(acc[2 * v][2 * half + 1], inv),
-                         round_code_bits(acc[2 * v + 1][2 * half], inv),
-                         round_code_bits(acc[2 * v + 1][2 * half + 1], inv));
+    for (int v = 0; v < WORDS; ++v) {
+      uint32_t r[4];
+      round_code_bits2(acc[2 * v][2 * half], acc[2 * v][2 * half + 1], inv2, r[0], r[1]);
+      round_code_bits2(acc[2 * v + 1][2 * half], acc[2 * v + 1][2 * half + 1], inv2, r[2], r[3]);
+      w[v] = pack_codes4(r[0], r[1], r[2], r[3]);
+    }
 #pragma unroll
     for (int v = 0; v < WORDS / 4; ++v)
       *reinterpret_cast<uint4*>(gCodes + q8_off<DK>(r, cbase + 16 * v)) =
