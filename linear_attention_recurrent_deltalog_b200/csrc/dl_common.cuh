@@ -281,22 +281,13 @@ __device__ __forceinline__ void rows_gemv(const float* sS, int j0, int lane, con
 //   GDN-2: u = (w o v) - a - ck,         o = b + cq + (k.q) u  (vj is w_j v_j)
 //   RWKV6: u = v,                        o = b + cq + bonus v
 // sScal: [0] k.q or the RWKV6 bonus, [1] beta, [2] gamma = e^{g_t} (GDN).
-//
-// PAIR: lanes l and l^1 hold the same row (the fp32 GEMV's butterfly); from
-// kPairSplitF entries on, each of the two sums every other pair of entries
-// (lane parity 0: entries 0, 1, 4, 5, ...; parity 1: 2, 3, 6, 7, ...) and
-// one exchange adds the halves, which halves the row's serial chain.  Both
-// lanes end with the same bits (the final add commutes).
-constexpr int kPairSplitF = 12;
-template <int VAR, typename TU, bool PAIR>
+template <int VAR, typename TU>
 __device__ __forceinline__ void row_update(const TU* sU, int jl, int f, int L, const float* sW,
                                            const float* sZ, const float* sScal, float vj, float a,
-                                           float b, int lane, float& u, float& o) {
+                                           float b, float& u, float& o) {
   float ck0 = 0.f, ck1 = 0.f, cq0 = 0.f, cq1 = 0.f;
-  const bool split = PAIR && f >= kPairSplitF;
-  const int step = split ? 4 : 2;
-  int i = split ? 2 * (lane & 1) : 0;
-  for (; i + 1 < f; i += step) {
+  int i = 0;
+  for (; i + 1 < f; i += 2) {
     const float u0 = to_f(sU[su_offset(jl, i, L)]);
     const float u1 = to_f(sU[su_offset(jl, i + 1, L)]);
     if (VAR != kVarRWKV6) {
@@ -306,17 +297,13 @@ __device__ __forceinline__ void row_update(const TU* sU, int jl, int f, int L, c
     cq0 = fmaf(sZ[i], u0, cq0);
     cq1 = fmaf(sZ[i + 1], u1, cq1);
   }
-  if (i < f) {  // the last entry of an odd count (one lane of a split pair)
+  if (i < f) {
     const float u0 = to_f(sU[su_offset(jl, i, L)]);
     if (VAR != kVarRWKV6) ck0 = fmaf(sW[i], u0, ck0);
     cq0 = fmaf(sZ[i], u0, cq0);
   }
-  float ck = ck0 + ck1;
-  float cq = cq0 + cq1;
-  if (split) {
-    if (VAR != kVarRWKV6) ck += __shfl_xor_sync(0xffffffffu, ck, 1);
-    cq += __shfl_xor_sync(0xffffffffu, cq, 1);
-  }
+  const float ck = ck0 + ck1;
+  const float cq = cq0 + cq1;
   const float sdot = sScal[0];
   if (VAR == kVarGDN) {
     const float gamma = sScal[2];

@@ -306,7 +306,7 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   if constexpr (!Q8) owner = (lane & 1) == 0;
   float u, o;
   const float vj = (VAR == kVarGDN2) ? sWg[jl] * to_f(sVr[jl]) : to_f(sVr[jl]);
-  row_update<VAR, TU, !Q8>(sU, jl, f, L, sW, sZ, sScal, vj, a, b, lane, u, o);
+  row_update<VAR, TU>(sU, jl, f, L, sW, sZ, sScal, vj, a, b, u, o);
   if (owner) {
     p.o[head * DV + r0 + jl] = o;
     if (merge_now)
