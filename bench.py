@@ -57,6 +57,8 @@ _CSRC = "linear_attention_recurrent_deltalog_b200/csrc/"
 KERNEL_SOURCES = {
     "dl_step_kernel": ("dl_device.cuh", "dl_common.cuh", "dl_q8.cuh", "dl_step.cuh"),
     "dl_merge_kernel": ("dl_device.cuh", "dl_common.cuh", "dl_q8.cuh", "dl_merge.cuh"),
+    "dl_merge_q8_kernel": ("dl_device.cuh", "dl_common.cuh", "dl_q8.cuh", "dl_tmem.cuh",
+                           "dl_fold_tmem.cuh", "dl_merge.cuh"),
     "dl_eager_kernel": ("dl_device.cuh", "dl_common.cuh", "dl_eager.cuh"),
 }
 
