@@ -47,6 +47,17 @@ from linear_attention_recurrent_deltalog_b200 import workloads as wl  # noqa: E4
 METRIC = "decode state-update tokens/s (B=512,H=32,d=128); HBM GB/s vs 8 TB/s peak"
 UNIT = "tokens/s"
 RING = 16
+HOLD_CYCLES = 1_000_000  # ~0.5 ms of GPU spin before a device-timed region starts
+
+
+def hold_stream():
+    """A short GPU spin queued just before a device-timed region's start
+    event (and outside it): it holds the stream while the host queues the
+    region's first launches, so the region times its launches back to back
+    and not the host's latency to issue the first one after a synchronize
+    (nvbench's blocking-kernel practice).  The end-to-end region, whose host
+    copies belong to what it measures, does not use it."""
+    torch.cuda._sleep(HOLD_CYCLES)
 L2_BYTES = 126 * 2**20
 FALLBACK_HBM_GBS = 6650.0
 
@@ -399,6 +410,7 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
             q, k, v, dec, beta, wg = ring[i % len(ring)]
             st.step(q, k, v, dec, beta, wg if wg is not None else bonus, o)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        hold_stream()
         a.record(stream)
         st.merge(dlb.DL_MERGE_FULL)
         b.record(stream)
@@ -415,6 +427,7 @@ def measure_merge_materialize(cfg, w, ring, bonus, S0, device, stream, peak, rep
     st.materialize(out)
     torch.cuda.synchronize(device)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold_stream()
     a.record(stream)
     for _ in range(reps):
         st.materialize(out)
@@ -524,6 +537,7 @@ def run_ours(args, world, rank, local):
     dist_barrier(world)
     torch.cuda.synchronize(device)
     with ClockSampler(local) as clk:
+        hold_stream()  # the host needs ~60 us to issue a step
         start.record(stream)
         for i in range(args.steps):
             one_step(args.warmup + i, evs[i])
@@ -565,6 +579,7 @@ def run_ours(args, world, rank, local):
         dlb.dl_eager_step(cfg, S_e, q, k, v, dec, beta, wg if wg is not None else bonus, o)
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold_stream()
     e0.record(stream)
     for i in range(args.steps):
         q, k, v, dec, beta, wg = ring[i % RING]
@@ -793,6 +808,7 @@ def run_serving(args, world, rank, local):
     torch.cuda.synchronize(device)
     dist_barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hold_stream()
     a.record(stream)
     for i in range(args.steps):
         token_step(args.warmup + i)

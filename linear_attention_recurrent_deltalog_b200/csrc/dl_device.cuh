@@ -441,6 +441,26 @@ __device__ __forceinline__ void codes4_to_h2(uint32_t w, uint32_t& h01, uint32_t
 // a2 (row g, k 2t+8..2t+9), a3 (row g+8, k 2t+8..2t+9); b0 (k 2t..2t+1,
 // col g), b1 (k 2t+8..2t+9, col g); d0,d1 (row g, cols 2t, 2t+1), d2,d3
 // (row g+8, cols 2t, 2t+1).
+// The same with bf16 operands (both A and B bf16).
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// x0, x1 -> bf16 pairs hi = bf16(x), lo = bf16(x - hi): hi + lo carries 16
+// significant bits.
+__device__ __forceinline__ void split_bf2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 f = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - f.x, x1 - f.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(

@@ -204,6 +204,52 @@ __device__ __forceinline__ void fold_mma_acc(float (&acc)[DK / 8][4], const TU* 
   }
 }
 
+// The same product for GDN with bf16 keys, without staged key fragments:
+// GDN's decay factor depends on the entry alone, so U Kt = (U Diag(fac)) K,
+// and the factor goes with the u values (A, as bf16 hi/lo pairs: 16
+// significant bits, about 1e-5 relative) while the keys enter the MMA as the
+// log stores them (bf16, exact), read straight from the staged log sK
+// [entries][DK].  fac[e] for e < nlog (the decayed entries), 1 for the
+// step's own entry.  Each product is formed as hi*k + lo*k.
+template <int DK, typename TU>
+__device__ __forceinline__ void fold_mma_acc_gdn(float (&acc)[DK / 8][4], const TU* sU,
+                                                 const float* sFac, const __nv_bfloat16* sK,
+                                                 int nlog, int nent, int nchunks, int L, int j0,
+                                                 int lane) {
+  constexpr int NTILE = DK / 8;
+  const int g = lane >> 2;
+  const int t = lane & 3;
+  const int rows[2] = {j0 + g, j0 + g + 8};
+  const uint16_t* sKb = reinterpret_cast<const uint16_t*>(sK);
+  for (int kc = 0; kc < nchunks; ++kc) {
+    const int e0 = 16 * kc + 2 * t;
+    float u[8];  // as in fold_mma_acc, each times its entry's factor
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = e0 + (q & 1) + ((q & 4) ? 8 : 0);
+      const float fac = (e < nlog) ? sFac[e] : 1.f;
+      u[q] = (e < nent) ? to_f(sU[su_offset(rows[(q >> 1) & 1], e, L)]) * fac : 0.f;
+    }
+    uint32_t ah[4], al[4];
+    split_bf2(u[0], u[1], ah[0], al[0]);
+    split_bf2(u[2], u[3], ah[1], al[1]);
+    split_bf2(u[4], u[5], ah[2], al[2]);
+    split_bf2(u[6], u[7], ah[3], al[3]);
+    const int ek[4] = {e0, e0 + 1, e0 + 8, e0 + 9};
+#pragma unroll
+    for (int n = 0; n < NTILE; ++n) {
+      const int c = fold_channel<DK>(n, g);  // B column g of n-tile n
+      uint32_t kv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) kv[i] = (ek[i] < nent) ? uint32_t(sKb[size_t(ek[i]) * DK + c]) : 0u;
+      const uint32_t b0 = kv[0] | (kv[1] << 16);  // entries 2t, 2t+1
+      const uint32_t b1 = kv[2] | (kv[3] << 16);  // entries 2t+8, 2t+9
+      mma_16816_bf16(acc[n], ah[0], ah[1], ah[2], ah[3], b0, b1);
+      mma_16816_bf16(acc[n], al[0], al[1], al[2], al[3], b0, b1);
+    }
+  }
+}
+
 // Writes the accumulators of fold_mma_acc as fp32 rows j0+g, j0+g+8 of
 // gOut (row-major, DK per row): 16-byte stores of DK/4 contiguous channels.
 template <int DK>
@@ -274,11 +320,15 @@ __device__ __forceinline__ void fold_store_f32_il(const float (&acc)[DK / 8][4],
 // as fp32 (unswizzled); otherwise each row's absolute maximum is reduced
 // over its four lanes and the row is requantized straight from the
 // accumulators into gCodes (swizzled order) and gScale.
-template <int DK, typename TU, bool SDEC>
+// DIRECT (GDN with bf16 keys): no staged fragments; the product comes from
+// fold_mma_acc_gdn with sK (the staged log keys), sFac and nlog instead.
+template <int DK, typename TU, bool SDEC, bool DIRECT = false>
 __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sScale, const TU* sU,
                                              const uint32_t* sB, const float* sDec, int nent,
                                              int nchunks, int L, int j0, int lane, int8_t* gCodes,
-                                             float* gScale, float* gOut) {
+                                             float* gScale, float* gOut,
+                                             const __nv_bfloat16* sK = nullptr,
+                                             const float* sFac = nullptr, int nlog = 0) {
   constexpr int NTILE = DK / 8;      // n-tiles; lane holds 2 channels of each
   constexpr int CPL = DK / 4;        // contiguous channels per lane
   constexpr int WORDS = CPL / 4;     // 4-code words per lane per row
@@ -322,7 +372,10 @@ __device__ __forceinline__ void fold_rows_q8(const int8_t* sQ, const float* sSca
       f2_unpack(x23, acc[2 * v + 1][2 * half], acc[2 * v + 1][2 * half + 1]);
     }
   }
-  fold_mma_acc<DK, TU>(acc, sU, sB, nent, nchunks, L, j0, lane);
+  if constexpr (DIRECT)
+    fold_mma_acc_gdn<DK, TU>(acc, sU, sFac, sK, nlog, nent, nchunks, L, j0, lane);
+  else
+    fold_mma_acc<DK, TU>(acc, sU, sB, nent, nchunks, L, j0, lane);
   if (gOut != nullptr) {
     fold_acc_store_f32<DK>(acc, j0, lane, gOut);
     return;

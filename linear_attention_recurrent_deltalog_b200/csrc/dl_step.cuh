@@ -26,6 +26,13 @@ namespace dl {
 // base GEMVs as their rows land), a second barrier publishes them, and
 // each warp finishes its rows.
 
+// The int8 step's fused fold for GDN with bf16 keys multiplies by the staged
+// log keys directly (fold_mma_acc_gdn), so it needs no key fragments in
+// shared memory: 34 KB per CTA instead of 43 KB at L = 16, 6 CTAs per SM
+// instead of 5.  The other int8 fused steps stage them.
+template <int VAR, typename TIn>
+constexpr bool kQ8DirectFold = (VAR == kVarGDN) && std::is_same<TIn, __nv_bfloat16>::value;
+
 template <int VAR, int DK, int DV, int ROWS, typename TIn, typename TB = float,
           bool FUSED = true>
 struct StepLayout {
@@ -58,7 +65,7 @@ struct StepLayout {
     offVecH = offScale + (Q8 ? align_up(size_t(ROWS) * 4, 128) : 0);
     offDecF = offVecH + (Q8 ? align_up(size_t(4) * kVecHStride<DK> * 2, 128) : 0);
     offKt = offDecF + ((Q8 && FUSED) ? align_up(size_t(kDecPadLen<DK>) * 4, 128) : 0);
-    offBar = offKt + ((Q8 && FUSED) ? size_t(q8_chunks(L)) * DK * 64 : 0);
+    offBar = offKt + ((Q8 && FUSED && !kQ8DirectFold<VAR, TIn>) ? size_t(q8_chunks(L)) * DK * 64 : 0);
     total = offBar + 8 * (StepTile<DK, ROWS, TB>::kChunks + 1);
   }
 };
@@ -317,21 +324,25 @@ dl_step_kernel(const StepParams p, const FillParam fp) {
   if (!merge_now) return;
   if constexpr (Q8) {
     // every warp's u_t rows are in slot f; stage the decayed keys of the
-    // L entries and the base decay once for the CTA, then fold and requantize
+    // L entries (GDN with bf16 keys: only the per-entry factors) and the base
+    // decay once for the CTA, then fold and requantize
+    constexpr bool kDirect = kQ8DirectFold<VAR, TIn>;
     __syncthreads();
-    if (GW == 1) {  // GDN: one decay factor per entry (sW's weights are no longer needed)
+    if (GW == 1)  // GDN: one decay factor per entry (sW's weights are no longer needed)
       for (int e = tid; e < f; e += NT) sW[e] = expf(sGt[0] - sG[e]);
-      __syncthreads();
+    if constexpr (!kDirect) {
+      if (GW == 1) __syncthreads();
+      stage_kt_frags<VAR, DK, TIn>(sK, sG, sGt, sW, f, f + 1, q8_chunks(f + 1), sB, tid, NT);
     }
-    stage_kt_frags<VAR, DK, TIn>(sK, sG, sGt, sW, f, f + 1, q8_chunks(f + 1), sB, tid, NT);
     for (int c = tid; c < DK; c += NT) sDecF[dec_pad(c)] = (GW == 1) ? sScal[2] : expf(sGt[c]);
     __syncthreads();
 #pragma unroll 1
     for (int half = 0; half < 2; ++half)  // the warp's two 16-row tiles, one at a time
-      fold_rows_q8<DK, TU, GW == 1>(sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L,
-                                    j0 + 16 * half, lane,
-                                    static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
-                                    p.scale + head * size_t(DV) + r0, nullptr);
+      fold_rows_q8<DK, TU, GW == 1, kDirect>(
+          sS, sScale, sU, sB, sDecF, f + 1, q8_chunks(f + 1), L, j0 + 16 * half, lane,
+          static_cast<int8_t*>(p.base) + (head * size_t(DV) + r0) * DK,
+          p.scale + head * size_t(DV) + r0, nullptr, reinterpret_cast<const __nv_bfloat16*>(sK),
+          sW, f);
   } else {
     float* gRows = static_cast<float*>(p.base) + (head * size_t(DV) + r0) * DK;
     const int nch = q8_chunks(f + 1);
