@@ -125,11 +125,12 @@ __device__ __forceinline__ uint32_t g_copy_bytes(int f) {
 //   KDA  : W_i = sum_c k_i[c] k_t[c] e^{g_t[c] - g_i[c]},  Z_i the same with q_t
 //   GDN-2: as KDA, with k_t replaced by the gated key kgate o k_t in W_i
 //   RWKV6: Z_i = sum_c k_i[c] r_t[c] e^{g_{t-1}[c] - g_i[c]}
-// The vector-decay weights take CUDA's fast __expf / __logf (documented
-// error: a few ulp for the log-decay differences of a log, |x| < ~10, and
-// 2^-21.4 absolute for __logf near 1), about 1e-6 relative against the 1e-4
-// state tolerance; they sit on every CTA's critical path (d_k / LPE of each
-// per lane and entry).
+// The vector-decay weights take CUDA's fast __expf / __logf: CUDA documents
+// at most 2 + 1.17|x| ulp for __expf(x) (|x| stays within a log's few decay
+// steps) and 2^-21.4 absolute for __logf near 1, about 1e-6 relative against
+// the 1e-4 state tolerance.  Each lane takes d_k / LPE logs once and as many
+// exps per entry, on every CTA's critical path; the log-decays appended to
+// the log keep the accurate logf.
 // kin, qin: k_t and q_t (r_t) in shared memory (fp32 or the input type);
 // sK: the staged log keys [f][DK]; sG: the staged log-decay; dec: the
 // step's decay (one scalar for GDN, d_k values otherwise).  Requires f > 0.

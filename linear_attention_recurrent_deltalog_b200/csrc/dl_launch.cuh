@@ -140,8 +140,8 @@ cudaError_t launch_merge_t(const MergeParams& p, const SeqList& list, unsigned n
                            cudaStream_t s) {
   if constexpr (std::is_same<TB, int8_t>::value && DV == kFoldRows) {
     // Merge: one stage (4 CTAs per SM at d_k = 128).  Materialize writes
-    // twice the bytes per head of fp32 output and measured faster with two
-    // stages (3 CTAs per SM).  Long vector-decay logs whose stages do not fit
+    // fp32 rows, four times the requantized output per head, and measured
+    // faster with two stages (3 CTAs per SM).  Long vector-decay logs whose stages do not fit
     // in shared memory take the per-warp fold below.
     if (p.mode == 2 && MergePipeLayout<VAR, DK, TIn, 2>(p.L).total <= size_t(kMaxSmemOptIn))
       return launch_merge_q8_tmem<VAR, DK, TIn, 2>(p, list, nheads, s);

@@ -216,7 +216,7 @@ dl_merge_kernel(const MergeParams p, const SeqList list) {
 // with NS = 1 stage a CTA needs about 47 KB at d_k = 128, and 4 CTAs (the
 // 512 TMEM columns' worth) fit on an SM (merge on B200: 0.55 -> 0.65 of the
 // copy bandwidth against two stages and 3 CTAs; materialize, whose fp32
-// output is twice as large, stays faster with two).
+// output is four times as large, stays faster with two).
 
 constexpr int kFoldThreads = 2 * kFoldRows;       // consumer threads
 constexpr int kMergePipeThreads = kFoldThreads + 32;  // plus the producer warp
