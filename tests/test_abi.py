@@ -245,13 +245,18 @@ def test_int8_code_swizzle_is_a_chunk_permutation(dk, dv):
 
 
 @pytest.mark.parametrize("variant", ["gdn", "kda", "gdn2", "rwkv6"])
-@pytest.mark.parametrize("L", [16, 48, 64])
-def test_q8_every_log_length_is_built(variant, L):
-    # the int8 merge takes the per-warp fold wherever its two-stage TMEM
-    # pipeline would not fit in shared memory (long vector-decay logs), so a
-    # state of every L up to 64 can be created (host-side check, no launch)
+@pytest.mark.parametrize("L", [1, 16, 48, 64])
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("in_dtype", ["bf16", "f32"])
+def test_q8_every_log_length_is_built(variant, L, fused, in_dtype):
+    # the int8 merge takes the per-warp fold wherever its TMEM pipeline would
+    # not fit in shared memory (long vector-decay logs), and the fused step
+    # stages key fragments except for GDN with bf16 keys, so a state of every
+    # L up to 64 can be created in both merge modes and for both key types
+    # (host-side check of the kernels' shared memory, no launch)
     d = 64 if variant == "rwkv6" else 128
-    c = cfg(variant=variant, d_k=d, d_v=d, L=L, base="q8").c()
+    c = cfg(variant=variant, d_k=d, d_v=d, L=L, base="q8", fused_merge=fused,
+            in_dtype=in_dtype).c()
     st = ctypes.c_void_p()
     rc = dlb._lib.dl_state_create(ctypes.byref(c), ctypes.c_void_p(1 << 20), ctypes.c_void_p(2 << 20),
                                   ctypes.c_void_p(3 << 20), ctypes.byref(st))
