@@ -56,8 +56,11 @@ def hold_stream():
     region's first launches, so the region times its launches back to back
     and not the host's latency to issue the first one after a synchronize
     (nvbench's blocking-kernel practice).  The end-to-end region, whose host
-    copies belong to what it measures, does not use it."""
-    torch.cuda._sleep(HOLD_CYCLES)
+    copies belong to what it measures, does not use it.  Without torch's
+    spin helper the region simply starts unheld (slightly conservative)."""
+    sleep = getattr(torch.cuda, "_sleep", None)
+    if sleep is not None:
+        sleep(HOLD_CYCLES)
 L2_BYTES = 126 * 2**20
 FALLBACK_HBM_GBS = 6650.0
 
