@@ -71,3 +71,40 @@ def test_single_core_oracle_sample():
     w = bench.wl.WORKLOADS["gdn_tiny"]
     r = bench.oracle_single_core(w, target_s=0.05)
     assert r["cores"] == 1 and r["value"] > 0 and "sequences" in r["sample"]
+
+
+def test_traffic_records_match_the_sources():
+    # the committed full-size ncu records of the headline step and of the
+    # eager step are keyed by the hash of the sources they describe; the
+    # bench line reports them (roofline.traffic, the measured write
+    # reduction) only while that hash matches
+    import types
+    step = bench.traffic_record("dl_step_kernel", workload="gdn_serving", B=512, L=16,
+                                merge="fused", base="f32")
+    eager = bench.traffic_record("dl_eager_kernel", workload="gdn_serving", B=512)
+    assert step is not None and eager is not None
+    assert step["kernel_hash"] == bench.kernel_hash("dl_step_kernel")
+    assert len(step["launches"]) >= 3
+    assert step["bytes_per_launch"] == int(sum(x["dram_read"] + x["dram_write"]
+                                               for x in step["launches"]) / len(step["launches"]))
+    w = types.SimpleNamespace(name="gdn_serving", B=512)
+    args = types.SimpleNamespace(steps=1, merge="fused")
+    line = bench.write_bytes_line(w, args, dl_write_total=170_000 * 512,
+                                  eager_write=2_113_536 * 512, step_rec=step)
+    m = line["measured"]
+    assert m is not None and m["measured_reduction"] > 10.0
+    # another workload has no record
+    assert bench.traffic_record("dl_step_kernel", workload="gdn_serving", B=64) is None
+
+
+def test_traffic_record_of_changed_sources_is_not_reported(monkeypatch):
+    monkeypatch.setattr(bench, "kernel_hash", lambda kernel="dl_step_kernel": "0" * 16)
+    assert bench.traffic_record("dl_step_kernel", workload="gdn_serving", B=512, L=16,
+                                merge="fused", base="f32") is None
+
+
+def test_stream_hold_without_the_spin_helper(monkeypatch):
+    # the hold before a timed region is skipped, not fatal, without torch's helper
+    import torch
+    monkeypatch.delattr(torch.cuda, "_sleep", raising=False)
+    bench.hold_stream()
